@@ -1,0 +1,202 @@
+/*
+ * lsa.h -- C ABI of the Lookahead Sparse Attention (LSA) indexer hot path on B200.
+ *
+ * The operations follow the pages describing FlashMemory-DeepSeek-V4:
+ *   [SUMMARY] "技术摘要：通过前瞻性稀疏注意力机制实现的 FlashMemory-DeepSeek-V4"
+ *             (gist.science technical summary), §2.1 架构设计 (periodic trigger,
+ *             memory indexer, scoring, dynamic fetch, hierarchical selection),
+ *             §2.2 数据策展与标注 (cross-layer majority vote), §2.3 (BCE + focal loss),
+ *             §2.4 最优配置 (three indexer layers, OR mode).
+ *   [REVIEW]  "论文综述：FlashMemory-DeepSeek-V4 用前瞻稀疏注意力压缩超长上下文KV缓存"
+ *             (paper.oopus.info review), part 二 核心方法与创新.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every pointer is a DEVICE pointer unless the comment says "host".  The caller
+ *    owns every buffer, including workspaces; the library allocates no memory.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and never synchronises, prints, traps or aborts.
+ *  - Argument errors are detected on the host before anything is launched and
+ *    returned as LSA_ERR_INVALID_ARG / LSA_ERR_UNSUPPORTED / LSA_ERR_NOMEM (workspace
+ *    too small).  A failed launch returns LSA_ERR_CUDA.  lsa_last_error() gives a
+ *    one-line description of the last error on the calling thread.
+ *  - Conditions only the device can see (a fetch list longer than its capacity, an
+ *    entry index out of range) are reported through an optional device status word
+ *    (int32): the kernel raises it to the lsa_status code with atomicMax, so the
+ *    caller zeroes it first and reads it after synchronising.
+ *  - Per-(layer, sequence) tensors are stored LAYER-MAJOR: [L][B][...], so the slice
+ *    of one indexer layer is one contiguous [B][...] block.
+ *  - Bit sets are uint32 words; bit i of word j is entry 32*j + i; Nw = ceil(N/32);
+ *    bits at or past N are zero.
+ *  - Pointers must be 16-byte aligned; K_IComp must be 128-byte aligned.
+ */
+#ifndef LSA_H_
+#define LSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LSA_OK = 0,
+  LSA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer          */
+  LSA_ERR_UNSUPPORTED = 2,   /* dtype / shape combination not built                 */
+  LSA_ERR_CAPACITY = 3,      /* (device status) a list did not fit its capacity     */
+  LSA_ERR_NOMEM = 4,         /* workspace smaller than the *_workspace_bytes answer  */
+  LSA_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed                 */
+  LSA_ERR_TIMEOUT = 6,       /* (device status) a bounded wait gave up               */
+  LSA_ERR_RANGE = 7          /* (device status) an entry index was out of [0, N)     */
+} lsa_status;
+
+typedef enum { LSA_F32 = 0, LSA_BF16 = 1, LSA_E4M3 = 2 } lsa_dtype;
+
+/* Static string for a status code.  Never NULL. */
+const char* lsa_status_string(int status);
+
+/* Description of the last error returned on this thread ("" if none). */
+const char* lsa_last_error(void);
+
+/* ABI version of this header: 1. */
+int lsa_abi_version(void);
+
+/* ------------------------------------------------------------------------------------
+ * lsa_index_score -- low-rank indexer query + head-fused gated score + threshold.
+ *
+ * [SUMMARY] §2.1: every tau decode steps the memory indexer maps the hidden state
+ * h_t of the current token to a low-rank indexer query and scores every earlier
+ * compressed entry s with a head-fused, sigmoid-gated matching score I_{t,s}; entries
+ * with I >= 0.5 are fetched ([REVIEW] 二).  Per (layer l, sequence b):
+ *     c = h W_down[l]                    (rank r; rounded to bf16 when wdt = BF16)
+ *     q = c W_up[l]  -> [H][dI]          (rounded to bf16 when wdt = BF16)
+ *     w = h W_w[l]   -> [H]              (fp32, not rounded)
+ *     z_s = kscale_s * sum_h w_h * ReLU(q_h . khat_s) + bias[l]
+ *     I_s = sigmoid(z_s);  mask bit s = (z_s >= 0)  (<=> I_s >= 0.5)
+ *
+ * Sizes: B sequences, L indexer layers, N entries per sequence, D hidden, r rank,
+ *        H heads, dI head dim.
+ * Inputs (layer-major):
+ *   h       [L][B][D]        wdt (LSA_F32 or LSA_BF16)
+ *   W_down  [L][D][r]        wdt
+ *   W_up    [L][r][H*dI]     wdt
+ *   W_w     [L][D][H]        wdt
+ *   bias    [L]              fp32
+ *   K       [L][B][N][dI]    kdt (LSA_F32, LSA_BF16, or LSA_E4M3 codes)
+ *   kscale  [L][B][N]        fp32, > 0; required iff kdt = LSA_E4M3, else NULL
+ *   q_in    [L][B][H][dI]    wdt, optional: use this query instead of projecting
+ *   w_in    [L][B][H]        fp32, optional: use these head weights (needs q_in)
+ * Outputs (any may be NULL except mask):
+ *   q_out   [L][B][H][dI]    wdt: the projected query (ignored when q_in is given)
+ *   w_out   [L][B][H]        fp32
+ *   mask    [L][B][Nw]       uint32 bit set of marked entries
+ *   logit   [L][B][N]        fp32 z_s
+ *   score   [L][B][N]        fp32 I_s
+ * layer: -1 processes all L layers in one pass; 0 <= layer < L processes that layer
+ *   only and touches only that layer's slices of every output.
+ * workspace: at least lsa_index_score_workspace_bytes(...) bytes, 256-byte aligned;
+ *   contents are scratch and may be reused by the caller after the call completes.
+ * Supported: kdt LSA_F32 with wdt LSA_F32 (CUDA-core path); kdt LSA_BF16 or
+ *   LSA_E4M3 with wdt LSA_BF16 (tensor-core path: dI in {64,128,192,256} for bf16 and
+ *   {128,256} for e4m3, H a multiple of 16 up to 256).  Other combinations with
+ *   H*dI <= 16384 run on the CUDA-core path; anything else is LSA_ERR_UNSUPPORTED.
+ * ---------------------------------------------------------------------------------- */
+size_t lsa_index_score_workspace_bytes(int B, int L, int N, int D, int r, int H, int dI,
+                                       int wdt, int kdt);
+
+int lsa_index_score(int B, int L, int N, int D, int r, int H, int dI,
+                    int wdt, const void* h, const void* W_down, const void* W_up,
+                    const void* W_w, const float* bias,
+                    int kdt, const void* K, const float* kscale,
+                    int layer,
+                    const void* q_in, const float* w_in,
+                    void* q_out, float* w_out,
+                    uint32_t* mask, float* logit, float* score,
+                    void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * lsa_select_union -- multi-layer routing in OR mode ([SUMMARY] §2.4; [REVIEW] 二:
+ * an entry any indexer layer asks for is fetched).  For one layer's mask, per word:
+ *     new_l = mask_l & ~U;   U = U | mask_l
+ * so calling it for the layers in order leaves U = OR of all layers and new_l = the
+ * entries first asked for by layer l (what an incremental fetch must still move).
+ *   mask_l [B][Nw] in, U [B][Nw] in/out (zero it before the first layer),
+ *   new_l  [B][Nw] out or NULL.  Nw >= 0.
+ * ---------------------------------------------------------------------------------- */
+int lsa_select_union(int B, int Nw, const uint32_t* mask_l, uint32_t* U, uint32_t* new_l,
+                     void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * lsa_compact -- fetch list of a bit set ([SUMMARY] §2.1 dynamic fetch: every entry
+ * with I >= 0.5 is fetched).  For each sequence b:
+ *     count[b] = popcount(bits[b]);  idx[b][0..] = ascending indices of the set bits.
+ *   bits [B][Nw], idx [B][cap] int32, count [B] int32 (the true count, which may
+ *   exceed cap; then only the first cap indices are written and *status is raised to
+ *   LSA_ERR_CAPACITY).  status: device int32 or NULL.  N >= 0, cap >= 0.
+ * ---------------------------------------------------------------------------------- */
+int lsa_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32_t* count,
+                int32_t* status, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * lsa_topk -- fine top-k inside the fetched subset ([SUMMARY] §2.1 hierarchical
+ * selection: once the critical subset is in GPU memory, a top-k runs inside it).
+ * Candidate j of sequence b is entry e = idx[b][j], j < min(count[b], cap); its key is
+ *     max over layers l of logit[l][b][e]
+ * (for a fetched entry this equals the largest logit among the layers that marked it).
+ * Keys are ordered descending, equal keys by ascending entry index; the first
+ * min(k, n) are returned in ASCENDING ENTRY ORDER in topk[b][0..]; remaining slots are
+ * set to -1; topk_count[b] = min(k, n).
+ *   idx [B][cap] ascending (as written by lsa_compact), count [B],
+ *   logit [L][B][N] fp32, topk [B][k] int32, topk_count [B] int32 (may be NULL).
+ * workspace: lsa_topk_workspace_bytes(B, cap) bytes.
+ * ---------------------------------------------------------------------------------- */
+size_t lsa_topk_workspace_bytes(int B, int cap);
+
+int lsa_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
+             const float* logit, int32_t* topk, int32_t* topk_count,
+             void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * lsa_gather_cold -- cold pool -> hot pool copy of the fetched rows ([SUMMARY] §2.1:
+ * marked compressed KV entries move from the CPU cold pool into GPU memory; [REVIEW]
+ * 二: asynchronously, overlapped with compute).  For j < min(count[b], cap):
+ *     hot[b][j][0..row_bytes) = cold[b][idx[b][j]][0..row_bytes)
+ *   cold   HOST pointer [B][N][row_bytes], page-locked and mapped into the device
+ *          address space (cudaHostAlloc / pinned torch memory); read by the kernel
+ *          over the host link, no staging copy.
+ *   idx [B][cap], count [B], hot [B][cap][row_bytes] device.
+ *   row_bytes: a positive multiple of 16.  Indices outside [0, N) are skipped and
+ *   raise *status (if not NULL) to LSA_ERR_RANGE.
+ * Launch it on a side stream to overlap the host-link transfer with scoring.
+ * ---------------------------------------------------------------------------------- */
+int lsa_gather_cold(int B, int N, size_t row_bytes, const void* cold_host,
+                    const int32_t* idx, const int32_t* count, int cap, void* hot,
+                    int32_t* status, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * lsa_vote_labels -- cross-layer majority-vote golden labels and their loss
+ * ([SUMMARY] §2.2: softmax over the indexer logits, per-layer nucleus top-p, an entry
+ * is golden when at least theta of the L layers select it; §2.3 / [REVIEW] 二: BCE
+ * plus focal loss).  For each (layer l, position p):
+ *     pi = softmax_N(logits[l][p]);  S_{l,p} = nucleus: entries in descending pi
+ *     (equal pi: lower index first) whose preceding mass is < top_p.
+ *     count[p][s] = #{l : s in S_{l,p}};  golden[p] bit s = count >= theta.
+ *   logits [L][P][N] fp32, golden [P][Nw] uint32, counts [P][N] uint8 or NULL.
+ *   scores [P][N] fp32 probabilities in (0,1) or NULL; when given, loss[0] = mean BCE
+ *   and loss[1] = mean focal loss with exponent gamma over all P*N (device doubles).
+ * workspace: lsa_vote_labels_workspace_bytes(L, P, N) bytes.
+ * ---------------------------------------------------------------------------------- */
+size_t lsa_vote_labels_workspace_bytes(int L, int P, int N);
+
+int lsa_vote_labels(int L, int P, int N, const float* logits, float top_p, int theta,
+                    uint32_t* golden, uint8_t* counts,
+                    const float* scores, float gamma, double* loss,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H_ */

@@ -1,0 +1,127 @@
+"""Python binding of liblsa, the B200 (sm_100a) library for the Lookahead Sparse
+Attention indexer step: scoring, OR-union, compaction, cold->hot gather, top-k in the
+fetched set and cross-layer vote labels.
+
+The functions keep the C names and only marshal arguments: tensors become raw
+pointers, dtypes become lsa_dtype codes, and the current torch CUDA stream is passed
+unless one is given.  Every computation runs in liblsa's kernels; a nonzero status
+raises LsaError.  Shapes and layouts are documented in include/lsa.h.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _abi
+
+LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_UNSUPPORTED, LSA_ERR_CAPACITY = 0, 1, 2, 3
+LSA_ERR_NOMEM, LSA_ERR_CUDA, LSA_ERR_TIMEOUT, LSA_ERR_RANGE = 4, 5, 6, 7
+LSA_F32, LSA_BF16, LSA_E4M3 = 0, 1, 2
+
+
+class LsaError(RuntimeError):
+    def __init__(self, code: int, where: str, detail: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} ({detail})")
+
+
+def lib():
+    return _abi.load()
+
+
+def status_string(code: int) -> str:
+    return lib().lsa_status_string(code).decode()
+
+
+def dtype_code(t) -> int:
+    dt = t.dtype if isinstance(t, torch.Tensor) else t
+    if dt == torch.float32:
+        return LSA_F32
+    if dt == torch.bfloat16:
+        return LSA_BF16
+    if dt in (torch.uint8, torch.float8_e4m3fn):
+        return LSA_E4M3
+    raise TypeError(f"no lsa_dtype for {dt}")
+
+
+def _p(t):
+    """Raw pointer of a tensor (None -> NULL); plain ints pass through."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, where: str):
+    if rc != LSA_OK:
+        raise LsaError(rc, where, lib().lsa_last_error().decode())
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A 256-byte aligned device workspace (torch allocations are 512-byte aligned)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+# ----------------------------------------------------------------------------- scoring
+
+def lsa_index_score_workspace_bytes(B, L, N, D, r, H, dI, wdt, kdt) -> int:
+    return int(lib().lsa_index_score_workspace_bytes(B, L, N, D, r, H, dI, wdt, kdt))
+
+
+def lsa_index_score(B, L, N, D, r, H, dI, wdt, h, W_down, W_up, W_w, bias, kdt, K, kscale,
+                    layer, q_in, w_in, q_out, w_out, mask, logit, score, workspace, stream=None):
+    rc = lib().lsa_index_score(B, L, N, D, r, H, dI, wdt, _p(h), _p(W_down), _p(W_up), _p(W_w),
+                               _p(bias), kdt, _p(K), _p(kscale), layer, _p(q_in), _p(w_in),
+                               _p(q_out), _p(w_out), _p(mask), _p(logit), _p(score),
+                               _p(workspace), 0 if workspace is None else workspace.numel(),
+                               _stream(stream))
+    _check(rc, "lsa_index_score")
+
+
+# ----------------------------------------------------------------------------- selection
+
+def lsa_select_union(B, Nw, mask_l, U, new_l, stream=None):
+    _check(lib().lsa_select_union(B, Nw, _p(mask_l), _p(U), _p(new_l), _stream(stream)),
+           "lsa_select_union")
+
+
+def lsa_compact(B, N, bits, cap, idx, count, status=None, stream=None):
+    _check(lib().lsa_compact(B, N, _p(bits), cap, _p(idx), _p(count), _p(status), _stream(stream)),
+           "lsa_compact")
+
+
+def lsa_topk_workspace_bytes(B, cap) -> int:
+    return int(lib().lsa_topk_workspace_bytes(B, cap))
+
+
+def lsa_topk(B, L, N, k, idx, cap, count, logit, topk, topk_count, workspace, stream=None):
+    _check(lib().lsa_topk(B, L, N, k, _p(idx), cap, _p(count), _p(logit), _p(topk), _p(topk_count),
+                          _p(workspace), 0 if workspace is None else workspace.numel(),
+                          _stream(stream)), "lsa_topk")
+
+
+def lsa_gather_cold(B, N, row_bytes, cold_host, idx, count, cap, hot, status=None, stream=None):
+    _check(lib().lsa_gather_cold(B, N, row_bytes, _p(cold_host), _p(idx), _p(count), cap, _p(hot),
+                                 _p(status), _stream(stream)), "lsa_gather_cold")
+
+
+# ----------------------------------------------------------------------------- labels
+
+def lsa_vote_labels_workspace_bytes(L, P, N) -> int:
+    return int(lib().lsa_vote_labels_workspace_bytes(L, P, N))
+
+
+def lsa_vote_labels(L, P, N, logits, top_p, theta, golden, counts, scores, gamma, loss,
+                    workspace, stream=None):
+    _check(lib().lsa_vote_labels(L, P, N, _p(logits), float(top_p), theta, _p(golden), _p(counts),
+                                 _p(scores), float(gamma), _p(loss), _p(workspace),
+                                 0 if workspace is None else workspace.numel(), _stream(stream)),
+           "lsa_vote_labels")

@@ -1,0 +1,262 @@
+// The C ABI of liblsa: argument checks, workspace layout and dispatch to the kernels.
+// Every entry point is declared and documented in include/lsa.h.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <algorithm>
+
+#include "lsa_common.cuh"
+
+namespace lsa {
+
+static thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return LSA_OK;
+}
+
+static size_t esize(int dt) { return dt == LSA_F32 ? 4 : dt == LSA_BF16 ? 2 : 1; }
+static bool valid_dtype(int dt) { return dt == LSA_F32 || dt == LSA_BF16 || dt == LSA_E4M3; }
+
+// Workspace of lsa_index_score: regions in this order, each 1024-byte aligned.
+struct ScoreWs {
+  size_t partA, partW, partB, cbuf, q, w, qimg, wfold, diag, total;
+};
+
+static ScoreWs score_ws(int B, int L, int D, int r, int H, int dI, int wdt, int kdt) {
+  ScoreWs o{};
+  const size_t BL = static_cast<size_t>(B) * L;
+  const size_t SA = project_splits(D), SB = project_splits(r);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t at = off; off = align_up(off + bytes, 1024); return at; };
+  o.partA = take(SA * BL * r * 4);
+  o.partW = take(SA * BL * H * 4);
+  o.partB = take(SB * BL * H * dI * 4);
+  o.cbuf = take(BL * r * 4);
+  o.q = take(BL * H * dI * esize(wdt));
+  o.w = take(BL * H * 4);
+  const bool tc = tc_supported(H, dI, wdt, kdt);
+  o.qimg = take(tc ? BL * tc_image_bytes(H, dI, kdt) : 0);
+  o.wfold = take(tc ? BL * H * 4 : 0);
+  o.diag = take(16);
+  o.total = off;
+  return o;
+}
+
+}  // namespace lsa
+
+using namespace lsa;
+
+extern "C" {
+
+const char* lsa_status_string(int status) {
+  switch (status) {
+    case LSA_OK: return "ok";
+    case LSA_ERR_INVALID_ARG: return "invalid argument";
+    case LSA_ERR_UNSUPPORTED: return "unsupported dtype or shape";
+    case LSA_ERR_CAPACITY: return "list longer than its capacity";
+    case LSA_ERR_NOMEM: return "workspace too small";
+    case LSA_ERR_CUDA: return "CUDA error";
+    case LSA_ERR_TIMEOUT: return "bounded wait timed out";
+    case LSA_ERR_RANGE: return "entry index out of range";
+  }
+  return "unknown status";
+}
+
+const char* lsa_last_error(void) { return g_err; }
+
+int lsa_abi_version(void) { return 1; }
+
+size_t lsa_index_score_workspace_bytes(int B, int L, int N, int D, int r, int H, int dI, int wdt,
+                                       int kdt) {
+  (void)N;
+  if (B < 0 || L < 0 || D < 0 || r < 0 || H < 0 || dI < 0) return 0;
+  return score_ws(B, L, D, r, H, dI, wdt, kdt).total;
+}
+
+int lsa_index_score(int B, int L, int N, int D, int r, int H, int dI,
+                    int wdt, const void* h, const void* W_down, const void* W_up,
+                    const void* W_w, const float* bias,
+                    int kdt, const void* K, const float* kscale,
+                    int layer,
+                    const void* q_in, const float* w_in,
+                    void* q_out, float* w_out,
+                    uint32_t* mask, float* logit, float* score,
+                    void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  g_err[0] = 0;
+  if (B < 0 || L < 0 || N < 0 || D < 0 || r < 0 || H <= 0 || dI <= 0)
+    return fail(LSA_ERR_INVALID_ARG, "index_score: negative size or H/dI < 1");
+  if (wdt != LSA_F32 && wdt != LSA_BF16) return fail(LSA_ERR_UNSUPPORTED, "index_score: wdt %d", wdt);
+  if (!valid_dtype(kdt)) return fail(LSA_ERR_UNSUPPORTED, "index_score: kdt %d", kdt);
+  if (layer < -1 || layer >= L) return fail(LSA_ERR_INVALID_ARG, "index_score: layer %d of %d", layer, L);
+  if (B == 0 || L == 0) return LSA_OK;
+  if (w_in && !q_in) return fail(LSA_ERR_INVALID_ARG, "index_score: w_in needs q_in");
+  const bool need_q = q_in == nullptr, need_w = w_in == nullptr;
+  if (need_q && (D <= 0 || r <= 0 || !h || !W_down || !W_up))
+    return fail(LSA_ERR_INVALID_ARG, "index_score: projection needs h, W_down, W_up, D, r");
+  if (need_w && (D <= 0 || !h || !W_w))
+    return fail(LSA_ERR_INVALID_ARG, "index_score: head weights need h, W_w, D");
+  if (!bias) return fail(LSA_ERR_INVALID_ARG, "index_score: bias is null");
+  if (N > 0 && (!K || !mask)) return fail(LSA_ERR_INVALID_ARG, "index_score: K or mask is null");
+  if ((kdt == LSA_E4M3) != (kscale != nullptr))
+    return fail(LSA_ERR_INVALID_ARG, "index_score: kscale must be given exactly for e4m3 keys");
+  const void* ptrs[] = {h, W_down, W_up, W_w, bias, K, kscale, q_in, w_in, q_out, w_out, mask, logit, score};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return fail(LSA_ERR_INVALID_ARG, "index_score: pointer %p not 16-byte aligned", p);
+  const bool tc = tc_supported(H, dI, wdt, kdt);
+  if (!tc && static_cast<size_t>(H) * dI > 16384)
+    return fail(LSA_ERR_UNSUPPORTED, "index_score: H*dI=%d too large for the CUDA-core path", H * dI);
+  if (tc && !aligned(K, 128)) return fail(LSA_ERR_INVALID_ARG, "index_score: K must be 128-byte aligned");
+  const ScoreWs ws = score_ws(B, L, D, r, H, dI, wdt, kdt);
+  if (!workspace || workspace_bytes < ws.total || !aligned(workspace, 256))
+    return fail(LSA_ERR_NOMEM, "index_score: workspace %zu bytes (need %zu, 256-byte aligned)",
+                workspace_bytes, ws.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  const int l0 = layer < 0 ? 0 : layer, nL = layer < 0 ? L : 1;
+
+  int rc = LSA_OK;
+  if (need_q || need_w) {
+    ProjectArgs pa{};
+    pa.B = B; pa.L = L; pa.D = D; pa.r = r; pa.H = H; pa.dI = dI; pa.wdt = wdt; pa.l0 = l0; pa.nL = nL;
+    pa.h = h; pa.W_down = W_down; pa.W_up = W_up; pa.W_w = W_w;
+    pa.partA = reinterpret_cast<float*>(base + ws.partA);
+    pa.partW = reinterpret_cast<float*>(base + ws.partW);
+    pa.partB = reinterpret_cast<float*>(base + ws.partB);
+    pa.cbuf = reinterpret_cast<float*>(base + ws.cbuf);
+    pa.q_ws = base + ws.q;
+    pa.w_ws = reinterpret_cast<float*>(base + ws.w);
+    pa.q_out = q_out;
+    pa.w_out = w_out;
+    pa.do_q = need_q;
+    pa.do_w = need_w;
+    rc = launch_project(pa, st);
+    if (rc != LSA_OK) return rc;
+  }
+  if (N == 0) return LSA_OK;
+  ScoreArgs sa{};
+  sa.B = B; sa.L = L; sa.N = N; sa.H = H; sa.dI = dI; sa.wdt = wdt; sa.kdt = kdt; sa.l0 = l0; sa.nL = nL;
+  sa.q = need_q ? static_cast<const void*>(base + ws.q) : q_in;
+  sa.w = need_w ? reinterpret_cast<const float*>(base + ws.w) : w_in;
+  sa.bias = bias; sa.K = K; sa.kscale = kscale;
+  sa.mask = mask; sa.logit = logit; sa.score = score;
+  if (tc) {
+    TcArgs ta{};
+    ta.sc = sa;
+    ta.qimg = base + ws.qimg;
+    ta.wfold = reinterpret_cast<float*>(base + ws.wfold);
+    ta.diag = reinterpret_cast<int32_t*>(base + ws.diag);
+    return launch_score_tc(ta, st);
+  }
+  return launch_score_simt(sa, st);
+}
+
+int lsa_select_union(int B, int Nw, const uint32_t* mask_l, uint32_t* U, uint32_t* new_l,
+                     void* stream) {
+  g_err[0] = 0;
+  if (B < 0 || Nw < 0) return fail(LSA_ERR_INVALID_ARG, "select_union: negative size");
+  if (static_cast<size_t>(B) * Nw == 0) return LSA_OK;
+  if (!mask_l || !U) return fail(LSA_ERR_INVALID_ARG, "select_union: null pointer");
+  if (!aligned(mask_l, 16) || !aligned(U, 16) || (new_l && !aligned(new_l, 16)))
+    return fail(LSA_ERR_INVALID_ARG, "select_union: pointers must be 16-byte aligned");
+  return launch_union(B, Nw, mask_l, U, new_l, static_cast<cudaStream_t>(stream));
+}
+
+int lsa_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32_t* count,
+                int32_t* status, void* stream) {
+  g_err[0] = 0;
+  if (B < 0 || N < 0 || cap < 0) return fail(LSA_ERR_INVALID_ARG, "compact: negative size");
+  if (B == 0) return LSA_OK;
+  if (!count || (N > 0 && !bits) || (cap > 0 && !idx))
+    return fail(LSA_ERR_INVALID_ARG, "compact: null pointer");
+  if ((bits && !aligned(bits, 16)) || (idx && !aligned(idx, 16)) || !aligned(count, 4))
+    return fail(LSA_ERR_INVALID_ARG, "compact: misaligned pointer");
+  return launch_compact(B, N, bits, cap, idx, count, status, static_cast<cudaStream_t>(stream));
+}
+
+size_t lsa_topk_workspace_bytes(int B, int cap) {
+  if (B < 0 || cap < 0) return 0;
+  return align_up(static_cast<size_t>(B) * cap * 4, 256) + 256;
+}
+
+int lsa_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
+             const float* logit, int32_t* topk, int32_t* topk_count,
+             void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  if (B < 0 || L <= 0 || N < 0 || k < 0 || cap < 0)
+    return fail(LSA_ERR_INVALID_ARG, "topk: bad size (L must be >= 1)");
+  if (B == 0) return LSA_OK;
+  if (!count || (cap > 0 && !idx) || (k > 0 && !topk) || (N > 0 && !logit))
+    return fail(LSA_ERR_INVALID_ARG, "topk: null pointer");
+  if (workspace_bytes < lsa_topk_workspace_bytes(B, cap) || (cap > 0 && !workspace) ||
+      (workspace && !aligned(workspace, 256)))
+    return fail(LSA_ERR_NOMEM, "topk: workspace %zu bytes (need %zu)", workspace_bytes,
+                lsa_topk_workspace_bytes(B, cap));
+  return launch_topk(B, L, N, k, idx, cap, count, logit, topk, topk_count,
+                     static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+int lsa_gather_cold(int B, int N, size_t row_bytes, const void* cold_host,
+                    const int32_t* idx, const int32_t* count, int cap, void* hot,
+                    int32_t* status, void* stream) {
+  g_err[0] = 0;
+  if (B < 0 || N < 0 || cap < 0) return fail(LSA_ERR_INVALID_ARG, "gather_cold: negative size");
+  if (row_bytes == 0 || row_bytes % 16 != 0)
+    return fail(LSA_ERR_INVALID_ARG, "gather_cold: row_bytes %zu is not a positive multiple of 16", row_bytes);
+  if (B == 0 || cap == 0) return LSA_OK;
+  if (!cold_host || !idx || !count || !hot) return fail(LSA_ERR_INVALID_ARG, "gather_cold: null pointer");
+  if (!aligned(cold_host, 16) || !aligned(hot, 16) || !aligned(idx, 16))
+    return fail(LSA_ERR_INVALID_ARG, "gather_cold: pointers must be 16-byte aligned");
+  cudaPointerAttributes attr{};
+  if (cudaPointerGetAttributes(&attr, cold_host) != cudaSuccess || attr.type != cudaMemoryTypeHost ||
+      attr.devicePointer == nullptr) {
+    cudaGetLastError();
+    return fail(LSA_ERR_INVALID_ARG, "gather_cold: cold pool is not page-locked, mapped host memory");
+  }
+  return launch_gather(B, N, row_bytes, attr.devicePointer, idx, count, cap, hot, status,
+                       static_cast<cudaStream_t>(stream));
+}
+
+size_t lsa_vote_labels_workspace_bytes(int L, int P, int N) {
+  if (L < 0 || P < 0 || N < 0) return 0;
+  const size_t Nw = (static_cast<size_t>(N) + 31) / 32;
+  return align_up(static_cast<size_t>(L) * P * Nw * 4, 256) +
+         align_up(static_cast<size_t>(L) * P * 4 * 4, 256) + 256;
+}
+
+int lsa_vote_labels(int L, int P, int N, const float* logits, float top_p, int theta,
+                    uint32_t* golden, uint8_t* counts,
+                    const float* scores, float gamma, double* loss,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  if (L < 0 || P < 0 || N < 0) return fail(LSA_ERR_INVALID_ARG, "vote_labels: negative size");
+  if (!(top_p > 0.f && top_p <= 1.f)) return fail(LSA_ERR_INVALID_ARG, "vote_labels: top_p must be in (0, 1]");
+  if (static_cast<size_t>(P) * N == 0) return LSA_OK;
+  if ((L > 0 && !logits) || !golden) return fail(LSA_ERR_INVALID_ARG, "vote_labels: null pointer");
+  if (scores && !loss) return fail(LSA_ERR_INVALID_ARG, "vote_labels: scores given without loss output");
+  const size_t need = lsa_vote_labels_workspace_bytes(L, P, N);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+    return fail(LSA_ERR_NOMEM, "vote_labels: workspace %zu bytes (need %zu)", workspace_bytes, need);
+  const size_t Nw = (static_cast<size_t>(N) + 31) / 32;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  VoteArgs va{};
+  va.L = L; va.P = P; va.N = N; va.logits = logits; va.top_p = top_p; va.theta = theta;
+  va.golden = golden; va.counts = counts; va.scores = scores; va.gamma = gamma; va.loss = loss;
+  va.selbits = reinterpret_cast<uint32_t*>(base);
+  va.rowparam = reinterpret_cast<float*>(base + align_up(static_cast<size_t>(L) * P * Nw * 4, 256));
+  va.lossacc = reinterpret_cast<double*>(base + need - 256);
+  return launch_vote(va, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

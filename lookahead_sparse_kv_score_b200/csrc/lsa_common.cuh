@@ -1,0 +1,112 @@
+// Shared device helpers and internal launch declarations of liblsa.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "lsa.h"
+
+namespace lsa {
+
+// ------------------------------------------------------------------ host-side errors
+int fail(int code, const char* fmt, ...);   // records the message, returns code
+int check_launch(const char* what);        // LSA_OK or LSA_ERR_CUDA after a launch
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ------------------------------------------------------------------ device helpers
+__device__ __forceinline__ void raise_status(int32_t* status, int code) {
+  if (status != nullptr) atomicMax(status, code);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ float e4m3_to_float(uint8_t code) {
+  __nv_fp8_e4m3 v;
+  v.__x = code;
+  return static_cast<float>(v);   // exact: every e4m3 value is a float
+}
+
+// Element loaders for the three storage types.
+__device__ __forceinline__ float load_elem(const float* p, size_t i) { return p[i]; }
+__device__ __forceinline__ float load_elem(const __nv_bfloat16* p, size_t i) {
+  return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ float load_elem(const uint8_t* p, size_t i) { return e4m3_to_float(p[i]); }
+
+__device__ __forceinline__ float sigmoid_f(float z) { return 1.0f / (1.0f + __expf(-z)); }
+
+// ------------------------------------------------------------------ internal launches
+// Projection: fills q_ws ([L][B][H][dI], wdt) and w_ws ([L][B][H] fp32) for layers
+// l0 .. l0+nL-1.  Scratch regions come from the caller's workspace.
+struct ProjectArgs {
+  int B, L, D, r, H, dI, wdt, l0, nL;
+  const void *h, *W_down, *W_up, *W_w;
+  float *partA, *partW, *partB, *cbuf;
+  void* q_ws;
+  float* w_ws;
+  void* q_out;
+  float* w_out;
+  bool do_q, do_w;      // project the query / the head weights
+};
+int launch_project(const ProjectArgs& a, cudaStream_t s);
+int project_splits(int K);   // number of K-splits used for a reduction length K
+
+// CUDA-core scoring of layers l0 .. l0+nL-1.
+struct ScoreArgs {
+  int B, L, N, H, dI, wdt, kdt, l0, nL;
+  const void* q;        // [L][B][H][dI] wdt
+  const float* w;       // [L][B][H]
+  const float* bias;    // [L]
+  const void* K;        // [L][B][N][dI] kdt
+  const float* kscale;  // [L][B][N] or null
+  uint32_t* mask;
+  float* logit;
+  float* score;
+};
+int launch_score_simt(const ScoreArgs& a, cudaStream_t s);
+
+// Tensor-core scoring (tcgen05 + TMA).  qimg/wfold are workspace regions.
+struct TcArgs {
+  ScoreArgs sc;
+  uint8_t* qimg;        // [L][B][img_bytes], 1024-byte aligned
+  float* wfold;         // [L][B][H]
+  int32_t* diag;        // device diagnostic word (bounded-wait timeouts), may be null
+};
+size_t tc_image_bytes(int H, int dI, int kdt);
+bool tc_supported(int H, int dI, int wdt, int kdt);
+int launch_score_tc(const TcArgs& a, cudaStream_t s);
+
+// Selection.
+int launch_union(int B, int Nw, const uint32_t* m, uint32_t* U, uint32_t* nw, cudaStream_t s);
+int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32_t* count,
+                   int32_t* status, cudaStream_t s);
+int launch_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
+                const float* logit, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws,
+                cudaStream_t s);
+int launch_gather(int B, int N, size_t row_bytes, const void* cold_dev, const int32_t* idx,
+                  const int32_t* count, int cap, void* hot, int32_t* status, cudaStream_t s);
+
+struct VoteArgs {
+  int L, P, N;
+  const float* logits;
+  float top_p;
+  int theta;
+  uint32_t* golden;
+  uint8_t* counts;
+  const float* scores;
+  float gamma;
+  double* loss;
+  uint32_t* selbits;    // workspace [L][P][Nw]
+  float* rowparam;      // workspace [L][P][4]
+  double* lossacc;      // workspace [2]
+};
+int launch_vote(const VoteArgs& a, cudaStream_t s);
+
+}  // namespace lsa

@@ -1,0 +1,130 @@
+"""Shared test helpers: device inputs from the seeded generator, raw copies for the
+oracle, and the comparison rules (tolerance bands) used by the parity tests."""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from oracle import lsa_oracle as O
+from oracle import step as OS
+from synth import workloads as W
+
+# Tolerance on I = sigmoid(z) by key dtype; on z the slope of sigmoid at 0 is 1/4.
+TOL_I = {"f32": 1e-5, "bf16": 2e-3, "e4m3": 1e-2}
+
+
+def tol_z(kdtype: str) -> float:
+    return 4.0 * TOL_I[kdtype]
+
+
+def raw(t: torch.Tensor) -> np.ndarray:
+    """Device/host tensor -> numpy array of its storage (bf16 as uint16 bit patterns)."""
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
+    return t.numpy()
+
+
+def base_name(w: W.ScoreWorkload) -> str:
+    return w.name
+
+
+@dataclass
+class Inputs:
+    w: W.ScoreWorkload
+    h: torch.Tensor        # [L][B][D]
+    Wd: torch.Tensor       # [L][D][r]
+    Wu: torch.Tensor       # [L][r][H*dI]
+    Ww: torch.Tensor       # [L][D][H]
+    bias: torch.Tensor     # [L] fp32
+    K: torch.Tensor        # [L][B][N][dI]
+    kscale: torch.Tensor | None
+    direction: torch.Tensor
+
+
+def make_inputs(w: W.ScoreWorkload, device="cuda") -> Inputs:
+    """Inputs of workload w (possibly reduced with W.scaled: the first B sequences and
+    first N entries of the stored workload's streams)."""
+    bias, direction = W.load_params(w.name)
+    bias = bias[: w.L]
+    direction = direction[: w.B, : w.L]
+    h = W.hidden_states(w, device).transpose(0, 1).contiguous()
+    Wd, Wu, Ww = W.all_layer_weights(w, device)
+    kdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8}[w.kdtype]
+    K = torch.empty(w.L, w.B, w.N, w.dI, dtype=kdt, device=device)
+    ks = torch.empty(w.L, w.B, w.N, dtype=torch.float32, device=device) if w.kdtype == "e4m3" else None
+    for l in range(w.L):
+        for b in range(w.B):
+            k, s = W.keys(w, b, l, direction[b, l].double(), 0, w.N, device)
+            K[l, b] = k
+            if ks is not None:
+                ks[l, b] = s
+    return Inputs(w, h, Wd, Wu, Ww, bias.to(device), K, ks, direction)
+
+
+class OracleCache:
+    """Oracle results of (b, l) computed on demand from the raw inputs."""
+
+    def __init__(self, inp: Inputs):
+        self.inp = inp
+        self.w = inp.w
+        self._qw = {}
+        self._h = raw(inp.h)
+        self._Wd = [raw(inp.Wd[l]) for l in range(self.w.L)]
+        self._Wu = [raw(inp.Wu[l]) for l in range(self.w.L)]
+        self._Ww = [raw(inp.Ww[l]) for l in range(self.w.L)]
+
+    def qw(self, l, b):
+        if (l, b) not in self._qw:
+            self._qw[l, b] = OS.project(self._h[l, b], self._Wd[l], self._Wu[l], self._Ww[l],
+                                        self.w.H, self.w.dI, self.w.wdtype)
+        return self._qw[l, b]
+
+    def keys(self, l, b, entries=None):
+        K = self.inp.K[l, b] if entries is None else self.inp.K[l, b][entries]
+        s = None
+        if self.inp.kscale is not None:
+            s = raw(self.inp.kscale[l, b] if entries is None else self.inp.kscale[l, b][entries])
+        return OS.decode_keys(raw(K), s, self.w.kdtype)
+
+    def z(self, l, b, entries=None):
+        q, wv = self.qw(l, b)
+        return O.head_fused_logits(q, wv, float(raw(self.inp.bias)[l]), self.keys(l, b, entries))
+
+    def z_bound_from_q_ulp(self, l, b, entries=None):
+        """Bound on |z(q') - z(q)| when every bf16 element of q may move by one ulp:
+        sum_h |w_h| * sum_d ulp(q_hd) * |k_d|  (ReLU is 1-Lipschitz)."""
+        q, wv = self.qw(l, b)
+        ulp = np.where(q != 0, np.exp2(np.floor(np.log2(np.abs(q) + 1e-300)) - 7), 2.0 ** -133)
+        K = np.abs(self.keys(l, b, entries))
+        return (K @ ulp.T) @ np.abs(wv)
+
+
+def q_ulp_ok(q_cuda: np.ndarray, q_oracle: np.ndarray) -> np.ndarray:
+    """Elementwise: the CUDA bf16 query is within one bf16 ulp of the oracle's."""
+    ulp = np.where(q_oracle != 0, np.exp2(np.floor(np.log2(np.abs(q_oracle) + 1e-300)) - 7), 2.0 ** -133)
+    return np.abs(q_cuda - q_oracle) <= ulp * (1 + 1e-12)
+
+
+def unpack(words: torch.Tensor, n: int) -> np.ndarray:
+    return O.unpack_bits(raw(words).view(np.uint32), n)
+
+
+def band(z_oracle: np.ndarray, tz) -> np.ndarray:
+    """Entries whose oracle logit lies within the tolerance of the threshold."""
+    return np.abs(z_oracle) <= tz
+
+
+def assert_mask_parity(got: np.ndarray, z_oracle: np.ndarray, tz, what=""):
+    exp = O.threshold_mark(z_oracle)
+    bad = (got != exp) & ~band(z_oracle, tz)
+    assert not bad.any(), f"{what}: {int(bad.sum())} mask mismatches outside the band, e.g. {np.flatnonzero(bad)[:5]}"
+
+
+def sigmoid_tol_ok(score: np.ndarray, z_oracle: np.ndarray, tol_I) -> np.ndarray:
+    return np.abs(score - O.sigmoid(z_oracle)) <= tol_I

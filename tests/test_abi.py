@@ -1,0 +1,75 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every symbol the header
+declares, and rejects bad arguments on the host before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import lookahead_sparse_kv_score_b200 as lsa
+from lookahead_sparse_kv_score_b200 import _abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lsa.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lsa_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _abi.load()
+
+
+def test_header_declares_the_six_calls():
+    names = declared_functions()
+    for call in ("lsa_index_score", "lsa_select_union", "lsa_compact", "lsa_topk",
+                 "lsa_gather_cold", "lsa_vote_labels"):
+        assert call in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(_abi.SIGNATURES) == set(declared_functions())
+
+
+def test_status_strings_and_version(lib):
+    assert lib.lsa_abi_version() == 1
+    for code in range(8):
+        assert lib.lsa_status_string(code)
+    assert lsa.status_string(3) == "list longer than its capacity"
+
+
+def test_host_side_argument_errors(lib):
+    # Each of these returns before any CUDA call.
+    assert lib.lsa_select_union(-1, 4, None, None, None, None) == lsa.LSA_ERR_INVALID_ARG
+    assert lib.lsa_select_union(2, 4, None, None, None, None) == lsa.LSA_ERR_INVALID_ARG
+    assert lib.lsa_select_union(0, 4, None, None, None, None) == lsa.LSA_OK
+    assert lib.lsa_compact(1, 64, None, 8, None, None, None, None) == lsa.LSA_ERR_INVALID_ARG
+    assert lib.lsa_gather_cold(1, 4, 24, 16, 16, 16, 4, 16, None, None) == lsa.LSA_ERR_INVALID_ARG
+    assert b"multiple of 16" in lib.lsa_last_error()
+    assert lib.lsa_topk(1, 0, 10, 4, 16, 4, 16, 16, 16, None, None, 0, None) == lsa.LSA_ERR_INVALID_ARG
+    assert lib.lsa_vote_labels(2, 2, 8, 16, ctypes.c_float(1.5), 3, 16, None, None,
+                               ctypes.c_float(2.0), None, None, 0, None) == lsa.LSA_ERR_INVALID_ARG
+    args = [1, 1, 128, 64, 16, 8, 64]
+    rc = lib.lsa_index_score(*args, 7, None, None, None, None, None, 0, None, None, 0,
+                             None, None, None, None, None, None, None, None, 0, None)
+    assert rc == lsa.LSA_ERR_UNSUPPORTED
+    rc = lib.lsa_index_score(*args, 0, 256, 256, 256, 256, 256, 2, 256, None, 0,
+                             None, None, None, None, 256, None, None, None, 0, None)
+    assert rc == lsa.LSA_ERR_INVALID_ARG            # e4m3 keys without a scale
+    rc = lib.lsa_index_score(*args, 0, 256, 256, 256, 256, 256, 0, 256, None, 0,
+                             None, None, None, None, 256, None, None, None, 0, None)
+    assert rc == lsa.LSA_ERR_NOMEM                  # no workspace
+
+
+def test_workspace_queries(lib):
+    n = lib.lsa_index_score_workspace_bytes(32, 3, 262144, 4096, 512, 64, 128, 1, 2)
+    assert 0 < n < 64 << 20
+    assert lib.lsa_topk_workspace_bytes(32, 262144) >= 32 * 262144 * 4
+    assert lib.lsa_vote_labels_workspace_bytes(24, 64, 131072) >= 24 * 64 * 4096 * 4

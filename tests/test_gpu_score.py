@@ -1,0 +1,141 @@
+"""Parity of lsa_index_score (projection + head-fused score + threshold) with the fp64
+oracle on the same seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import lookahead_sparse_kv_score_b200 as lsa
+from lookahead_sparse_kv_score_b200 import build
+from synth import workloads as W
+
+import lsa_cases as C
+
+pytestmark = pytest.mark.gpu
+
+WDT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    build.build()
+    lsa.lib()
+
+
+def run_score(inp: C.Inputs, layer=-1, q_in=None, w_in=None, want_q=True, sentinel=False):
+    w = inp.w
+    Nw = (w.N + 31) // 32
+    dev = inp.K.device
+    fill = 0x5A5A5A5A if sentinel else 0
+    mask = torch.full((w.L, w.B, Nw), fill, dtype=torch.int32, device=dev)
+    logit = torch.full((w.L, w.B, w.N), float("nan"), device=dev)
+    score = torch.full((w.L, w.B, w.N), float("nan"), device=dev)
+    q_out = torch.zeros(w.L, w.B, w.H, w.dI, dtype=WDT[w.wdtype], device=dev) if want_q else None
+    w_out = torch.zeros(w.L, w.B, w.H, device=dev) if want_q else None
+    wdt, kdt = lsa.dtype_code(WDT[w.wdtype]), lsa.dtype_code(inp.K)
+    ws = lsa.workspace(lsa.lsa_index_score_workspace_bytes(w.B, w.L, w.N, w.D, w.r, w.H, w.dI, wdt, kdt))
+    lsa.lsa_index_score(w.B, w.L, w.N, w.D, w.r, w.H, w.dI, wdt, inp.h, inp.Wd, inp.Wu, inp.Ww, inp.bias,
+                        kdt, inp.K, inp.kscale, layer, q_in, w_in, q_out, w_out, mask, logit, score, ws)
+    torch.cuda.synchronize()
+    return dict(mask=mask, logit=logit, score=score, q=q_out, w=w_out)
+
+
+def oracle_query_tensors(inp, orc):
+    w = inp.w
+    q = torch.zeros(w.L, w.B, w.H, w.dI, dtype=torch.float64)
+    wv = torch.zeros(w.L, w.B, w.H, dtype=torch.float64)
+    for l in range(w.L):
+        for b in range(w.B):
+            qq, ww = orc.qw(l, b)
+            q[l, b] = torch.from_numpy(qq)
+            wv[l, b] = torch.from_numpy(ww)
+    # the oracle's q is bf16-valued for bf16 models, so the cast below is exact
+    return q.to(WDT[w.wdtype]).cuda(), wv.float().cuda()
+
+
+def check_layer_outputs(out, inp, orc, l, b, z_extra=0.0):
+    w = inp.w
+    z = orc.z(l, b)
+    tz = C.tol_z(w.kdtype) + z_extra
+    zc = out["logit"][l, b].double().cpu().numpy()
+    sc = out["score"][l, b].double().cpu().numpy()
+    assert np.all(np.abs(zc - z) <= tz), f"logit error {np.max(np.abs(zc - z) - tz)} over tolerance"
+    assert np.all(np.abs(sc - 1 / (1 + np.exp(-z))) <= C.TOL_I[w.kdtype] + np.asarray(z_extra) / 4)
+    got = C.unpack(out["mask"][l, b], w.N)
+    C.assert_mask_parity(got, z, tz, f"layer {l} seq {b}")
+    words = C.raw(out["mask"][l, b]).view(np.uint32)
+    if w.N % 32:
+        assert words[-1] >> (w.N % 32) == 0, "bits past N must be zero"
+
+
+def test_tiny_fp32_full_parity():
+    w = W.WORKLOADS["lsa_step_16k_tiny_fp32"]
+    inp = C.make_inputs(w)
+    orc = C.OracleCache(inp)
+    out = run_score(inp)
+    q, wv = orc.qw(0, 0)
+    np.testing.assert_allclose(out["q"][0, 0].double().cpu().numpy(), q, rtol=1e-5, atol=1e-5)
+    np.testing.assert_allclose(out["w"][0, 0].double().cpu().numpy(), wv, rtol=1e-5, atol=1e-5)
+    check_layer_outputs(out, inp, orc, 0, 0)
+    frac = float(C.unpack(out["mask"][0, 0], w.N).mean())
+    assert 0.05 < frac < 0.2
+
+
+def test_128k_bf16_projection_within_one_ulp():
+    w = W.WORKLOADS["lsa_step_128k_b1_bf16"]
+    inp = C.make_inputs(w)
+    orc = C.OracleCache(inp)
+    out = run_score(inp)
+    for l in range(w.L):
+        q, wv = orc.qw(l, 0)
+        qc = out["q"][l, 0].double().cpu().numpy()
+        ok = C.q_ulp_ok(qc, q)
+        assert ok.all(), f"layer {l}: {int((~ok).sum())} query elements off by more than 1 bf16 ulp"
+        np.testing.assert_allclose(out["w"][l, 0].double().cpu().numpy(), wv, rtol=1e-4, atol=1e-4)
+
+
+def test_128k_bf16_score_with_oracle_query():
+    w = W.WORKLOADS["lsa_step_128k_b1_bf16"]
+    inp = C.make_inputs(w)
+    orc = C.OracleCache(inp)
+    q_in, w_in = oracle_query_tensors(inp, orc)
+    out = run_score(inp, q_in=q_in, w_in=w_in, want_q=False)
+    for l in range(w.L):
+        check_layer_outputs(out, inp, orc, l, 0)
+
+
+def test_128k_bf16_end_to_end_with_query_bound():
+    """Projection inside the call: the logit may move by the effect of a one-ulp query
+    difference, bounded per entry by the oracle."""
+    w = W.WORKLOADS["lsa_step_128k_b1_bf16"]
+    inp = C.make_inputs(w)
+    orc = C.OracleCache(inp)
+    out = run_score(inp)
+    for l in range(w.L):
+        check_layer_outputs(out, inp, orc, l, 0, z_extra=orc.z_bound_from_q_ulp(l, 0))
+
+
+@pytest.mark.parametrize("N", [1, 31, 1000, 4097])
+def test_ragged_sizes_and_single_layer(N):
+    base = W.WORKLOADS["lsa_step_512k_b8_bf16"]
+    w = W.scaled(base, B=2, N=N)
+    inp = C.make_inputs(w)
+    orc = C.OracleCache(inp)
+    q_in, w_in = oracle_query_tensors(inp, orc)
+    out = run_score(inp, layer=1, q_in=q_in, w_in=w_in, want_q=False, sentinel=True)
+    for b in range(w.B):
+        check_layer_outputs(out, inp, orc, 1, b)
+    # the other layers' slices are untouched
+    assert bool((out["mask"][0] == 0x5A5A5A5A).all()) and bool((out["mask"][2] == 0x5A5A5A5A).all())
+    assert bool(torch.isnan(out["logit"][0]).all())
+
+
+def test_empty_sizes_are_no_ops():
+    w = W.scaled(W.WORKLOADS["lsa_step_16k_tiny_fp32"], N=0)
+    inp = C.make_inputs(w)
+    out = run_score(inp)
+    assert out["mask"].numel() == 0
+    w0 = W.scaled(W.WORKLOADS["lsa_step_16k_tiny_fp32"], B=0)
+    lsa.lsa_index_score(0, 1, 64, 512, 64, 8, 64, 0, None, None, None, None, None, 0, None, None,
+                        -1, None, None, None, None, None, None, None, None)
