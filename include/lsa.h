@@ -93,13 +93,15 @@ int lsa_abi_version(void);
  *   mask    [L][B][Nw]       uint32 bit set of marked entries
  *   logit   [L][B][N]        fp32 z_s
  *   score   [L][B][N]        fp32 I_s
+ * status: device int32 or NULL; raised to LSA_ERR_TIMEOUT if a bounded pipeline wait
+ *   inside the tensor-core kernel gave up (the outputs are then incomplete).
  * layer: -1 processes all L layers in one pass; 0 <= layer < L processes that layer
  *   only and touches only that layer's slices of every output.
  * workspace: at least lsa_index_score_workspace_bytes(...) bytes, 256-byte aligned;
  *   contents are scratch and may be reused by the caller after the call completes.
  * Supported: kdt LSA_F32 with wdt LSA_F32 (CUDA-core path); kdt LSA_BF16 or
  *   LSA_E4M3 with wdt LSA_BF16 (tensor-core path: dI in {64,128,192,256} for bf16 and
- *   {128,256} for e4m3, H a multiple of 16 up to 256).  Other combinations with
+ *   {128,256} for e4m3, H a multiple of 32 from 32 to 256).  Other combinations with
  *   H*dI <= 16384 run on the CUDA-core path; anything else is LSA_ERR_UNSUPPORTED.
  * ---------------------------------------------------------------------------------- */
 size_t lsa_index_score_workspace_bytes(int B, int L, int N, int D, int r, int H, int dI,
@@ -112,7 +114,7 @@ int lsa_index_score(int B, int L, int N, int D, int r, int H, int dI,
                     int layer,
                     const void* q_in, const float* w_in,
                     void* q_out, float* w_out,
-                    uint32_t* mask, float* logit, float* score,
+                    uint32_t* mask, float* logit, float* score, int32_t* status,
                     void* workspace, size_t workspace_bytes,
                     void* stream);
 

@@ -77,10 +77,11 @@ def lsa_index_score_workspace_bytes(B, L, N, D, r, H, dI, wdt, kdt) -> int:
 
 
 def lsa_index_score(B, L, N, D, r, H, dI, wdt, h, W_down, W_up, W_w, bias, kdt, K, kscale,
-                    layer, q_in, w_in, q_out, w_out, mask, logit, score, workspace, stream=None):
+                    layer, q_in, w_in, q_out, w_out, mask, logit, score, workspace, status=None,
+                    stream=None):
     rc = lib().lsa_index_score(B, L, N, D, r, H, dI, wdt, _p(h), _p(W_down), _p(W_up), _p(W_w),
                                _p(bias), kdt, _p(K), _p(kscale), layer, _p(q_in), _p(w_in),
-                               _p(q_out), _p(w_out), _p(mask), _p(logit), _p(score),
+                               _p(q_out), _p(w_out), _p(mask), _p(logit), _p(score), _p(status),
                                _p(workspace), 0 if workspace is None else workspace.numel(),
                                _stream(stream))
     _check(rc, "lsa_index_score")

@@ -20,7 +20,7 @@ SIGNATURES = {
     "lsa_index_score": (c_int, [c_int] * 7 + [c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                               c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p,
                                               c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
-                                              c_void_p, c_size_t, c_void_p]),
+                                              c_void_p, c_void_p, c_size_t, c_void_p]),
     "lsa_select_union": (c_int, [c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "lsa_compact": (c_int, [c_int, c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "lsa_topk_workspace_bytes": (c_size_t, [c_int, c_int]),

@@ -30,7 +30,7 @@ static bool valid_dtype(int dt) { return dt == LSA_F32 || dt == LSA_BF16 || dt =
 
 // Workspace of lsa_index_score: regions in this order, each 1024-byte aligned.
 struct ScoreWs {
-  size_t partA, partW, partB, cbuf, q, w, qimg, wfold, diag, total;
+  size_t partA, partW, partB, cbuf, q, w, qimg, wfold, total;
 };
 
 static ScoreWs score_ws(int B, int L, int D, int r, int H, int dI, int wdt, int kdt) {
@@ -48,7 +48,6 @@ static ScoreWs score_ws(int B, int L, int D, int r, int H, int dI, int wdt, int 
   const bool tc = tc_supported(H, dI, wdt, kdt);
   o.qimg = take(tc ? BL * tc_image_bytes(H, dI, kdt) : 0);
   o.wfold = take(tc ? BL * H * 4 : 0);
-  o.diag = take(16);
   o.total = off;
   return o;
 }
@@ -91,7 +90,7 @@ int lsa_index_score(int B, int L, int N, int D, int r, int H, int dI,
                     int layer,
                     const void* q_in, const float* w_in,
                     void* q_out, float* w_out,
-                    uint32_t* mask, float* logit, float* score,
+                    uint32_t* mask, float* logit, float* score, int32_t* status,
                     void* workspace, size_t workspace_bytes,
                     void* stream) {
   g_err[0] = 0;
@@ -156,7 +155,7 @@ int lsa_index_score(int B, int L, int N, int D, int r, int H, int dI,
     ta.sc = sa;
     ta.qimg = base + ws.qimg;
     ta.wfold = reinterpret_cast<float*>(base + ws.wfold);
-    ta.diag = reinterpret_cast<int32_t*>(base + ws.diag);
+    ta.status = status;
     return launch_score_tc(ta, st);
   }
   return launch_score_simt(sa, st);

@@ -77,7 +77,7 @@ struct TcArgs {
   ScoreArgs sc;
   uint8_t* qimg;        // [L][B][img_bytes], 1024-byte aligned
   float* wfold;         // [L][B][H]
-  int32_t* diag;        // device diagnostic word (bounded-wait timeouts), may be null
+  int32_t* status;      // caller's device status word (bounded-wait timeouts), may be null
 };
 size_t tc_image_bytes(int H, int dI, int kdt);
 bool tc_supported(int H, int dI, int wdt, int kdt);

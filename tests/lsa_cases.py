@@ -51,8 +51,11 @@ def make_inputs(w: W.ScoreWorkload, device="cuda") -> Inputs:
     """Inputs of workload w (possibly reduced with W.scaled: the first B sequences and
     first N entries of the stored workload's streams)."""
     bias, direction = W.load_params(w.name)
-    bias = bias[: w.L]
-    direction = direction[: w.B, : w.L]
+    return make_inputs_with(w, bias[: w.L], direction[: w.B, : w.L], device)
+
+
+def make_inputs_with(w: W.ScoreWorkload, bias, direction, device="cuda") -> Inputs:
+    """Inputs of workload w with a given per-layer bias and planted direction."""
     h = W.hidden_states(w, device).transpose(0, 1).contiguous()
     Wd, Wu, Ww = W.all_layer_weights(w, device)
     kdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8}[w.kdtype]

@@ -58,13 +58,13 @@ def test_host_side_argument_errors(lib):
                                ctypes.c_float(2.0), None, None, 0, None) == lsa.LSA_ERR_INVALID_ARG
     args = [1, 1, 128, 64, 16, 8, 64]
     rc = lib.lsa_index_score(*args, 7, None, None, None, None, None, 0, None, None, 0,
-                             None, None, None, None, None, None, None, None, 0, None)
+                             None, None, None, None, None, None, None, None, None, 0, None)
     assert rc == lsa.LSA_ERR_UNSUPPORTED
     rc = lib.lsa_index_score(*args, 0, 256, 256, 256, 256, 256, 2, 256, None, 0,
-                             None, None, None, None, 256, None, None, None, 0, None)
+                             None, None, None, None, 256, None, None, None, None, 0, None)
     assert rc == lsa.LSA_ERR_INVALID_ARG            # e4m3 keys without a scale
     rc = lib.lsa_index_score(*args, 0, 256, 256, 256, 256, 256, 0, 256, None, 0,
-                             None, None, None, None, 256, None, None, None, 0, None)
+                             None, None, None, None, 256, None, None, None, None, 0, None)
     assert rc == lsa.LSA_ERR_NOMEM                  # no workspace
 
 
