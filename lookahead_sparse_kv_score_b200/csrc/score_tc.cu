@@ -498,7 +498,7 @@ bool tc_supported(int H, int dI, int wdt, int kdt) {
   } else {
     return false;
   }
-  return tc_layout(H, dI, fp8).stages >= 3;
+  return tc_layout(H, dI, fp8).stages >= 2;
 }
 
 size_t tc_image_bytes(int H, int dI, int kdt) {

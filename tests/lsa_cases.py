@@ -99,19 +99,66 @@ class OracleCache:
         q, wv = self.qw(l, b)
         return O.head_fused_logits(q, wv, float(raw(self.inp.bias)[l]), self.keys(l, b, entries))
 
-    def z_bound_from_q_ulp(self, l, b, entries=None):
-        """Bound on |z(q') - z(q)| when every bf16 element of q may move by one ulp:
-        sum_h |w_h| * sum_d ulp(q_hd) * |k_d|  (ReLU is 1-Lipschitz)."""
+    def q_allowed(self, l, b):
+        """Per-element bound on |q_cuda - q_oracle| for an fp32-accumulating projection.
+
+        The device sums in fp32 with at most FP32_DEPTH sequential additions per output,
+        so |fl(sum) - sum| <= gamma * sum|terms| (gamma = depth * 2^-24 / (1 - depth * 2^-24)).
+        An element of c can round to a different bf16 value than the exact sum only when
+        the exact sum lies within that error of a rounding midpoint; such an element may
+        move by one ulp of c.  The perturbation of the pre-rounding q is then
+        (sum over those elements of ulp(c_i) |W_up[i, j]|) + gamma * sum|c_i W_up[i, j]|,
+        and rounding q to bf16 adds at most one ulp of q.  For fp32 models (no rounding)
+        the bound is the two fp32 summation errors alone."""
+        w = self.w
+        h = OS.decode(self._h[l, b], w.wdtype)
+        Wd = OS.decode(self._Wd[l], w.wdtype)
+        Wu = OS.decode(self._Wu[l], w.wdtype)
+        u = 2.0 ** -24
+        gam = FP32_DEPTH * u / (1 - FP32_DEPTH * u)
+        c_exact = h @ Wd
+        err_c = gam * (np.abs(h) @ np.abs(Wd))
+        if w.wdtype == "bf16":
+            c_r = O.round_to_bf16(c_exact)
+            ulp_c = bf16_ulp(c_r)
+            to_mid = np.abs(np.abs(c_exact - c_r) - ulp_c / 2)
+            dc = np.where(to_mid <= err_c, ulp_c, 0.0)
+        else:
+            c_r, dc = c_exact, err_c
+        err_q = dc @ np.abs(Wu) + gam * ((np.abs(c_r) + dc) @ np.abs(Wu))
+        q, _ = self.qw(l, b)
+        rnd = bf16_ulp(q) if w.wdtype == "bf16" else 0.0
+        return (err_q.reshape(q.shape) + rnd) * (1 + 1e-9)
+
+    def w_allowed(self, l, b):
+        """Bound on |w_cuda - w_oracle|: one fp32 summation error."""
+        w = self.w
+        h = OS.decode(self._h[l, b], w.wdtype)
+        Ww = OS.decode(self._Ww[l], w.wdtype)
+        u = 2.0 ** -24
+        return FP32_DEPTH * u / (1 - FP32_DEPTH * u) * (np.abs(h) @ np.abs(Ww))
+
+    def z_bound_from_q(self, l, b, entries=None):
+        """Bound on |z(q_cuda, w_cuda) - z(q_oracle, w_oracle)| (ReLU is 1-Lipschitz):
+        sum_h |w_h| sum_d allowed_hd |k_d|  +  sum_h dw_h (ReLU(q_h.k) + sum_d allowed_hd |k_d|)."""
         q, wv = self.qw(l, b)
-        ulp = np.where(q != 0, np.exp2(np.floor(np.log2(np.abs(q) + 1e-300)) - 7), 2.0 ** -133)
-        K = np.abs(self.keys(l, b, entries))
-        return (K @ ulp.T) @ np.abs(wv)
+        Kd = self.keys(l, b, entries)
+        dq = np.abs(Kd) @ self.q_allowed(l, b).T
+        return dq @ np.abs(wv) + (np.maximum(Kd @ q.T, 0) + dq) @ self.w_allowed(l, b)
 
 
-def q_ulp_ok(q_cuda: np.ndarray, q_oracle: np.ndarray) -> np.ndarray:
-    """Elementwise: the CUDA bf16 query is within one bf16 ulp of the oracle's."""
-    ulp = np.where(q_oracle != 0, np.exp2(np.floor(np.log2(np.abs(q_oracle) + 1e-300)) - 7), 2.0 ** -133)
-    return np.abs(q_cuda - q_oracle) <= ulp * (1 + 1e-12)
+FP32_DEPTH = 128   # longest chain of sequential fp32 additions in the projection kernels
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 values at |x| (2^-133 below the normal range)."""
+    x = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.where(x > 0, x, 1.0)))
+    return np.where(x >= 2.0 ** -126, np.exp2(e - 7), 2.0 ** -133)
+
+
+def q_within(q_cuda: np.ndarray, q_oracle: np.ndarray, allowed: np.ndarray) -> np.ndarray:
+    return np.abs(q_cuda - q_oracle) <= allowed
 
 
 def unpack(words: torch.Tensor, n: int) -> np.ndarray:

@@ -55,10 +55,17 @@ def oracle_query_tensors(inp, orc):
 
 
 def check_layer_outputs(out, inp, orc, l, b, z_extra=0.0):
+    """Logits, scores and mask of one (layer, sequence) against the oracle.  z_extra is a
+    per-entry bound for a query projected on the device (end-to-end runs); then the
+    worst case is checked against it and the typical error against the dtype tolerance."""
     w = inp.w
     z = orc.z(l, b)
     tz = C.tol_z(w.kdtype) + z_extra
     zc = out["logit"][l, b].double().cpu().numpy()
+    if np.ndim(z_extra) > 0:
+        dz = np.abs(zc - z)
+        assert np.median(dz) <= C.tol_z(w.kdtype) and np.quantile(dz, 0.99) <= 4 * C.tol_z(w.kdtype), \
+            f"typical logit error {np.median(dz)} / p99 {np.quantile(dz, 0.99)}"
     sc = out["score"][l, b].double().cpu().numpy()
     assert np.all(np.abs(zc - z) <= tz), f"logit error {np.max(np.abs(zc - z) - tz)} over tolerance"
     assert np.all(np.abs(sc - 1 / (1 + np.exp(-z))) <= C.TOL_I[w.kdtype] + np.asarray(z_extra) / 4)
@@ -82,7 +89,7 @@ def test_tiny_fp32_full_parity():
     assert 0.05 < frac < 0.2
 
 
-def test_128k_bf16_projection_within_one_ulp():
+def test_128k_bf16_projection_within_fp32_bound():
     w = W.WORKLOADS["lsa_step_128k_b1_bf16"]
     inp = C.make_inputs(w)
     orc = C.OracleCache(inp)
@@ -90,8 +97,8 @@ def test_128k_bf16_projection_within_one_ulp():
     for l in range(w.L):
         q, wv = orc.qw(l, 0)
         qc = out["q"][l, 0].double().cpu().numpy()
-        ok = C.q_ulp_ok(qc, q)
-        assert ok.all(), f"layer {l}: {int((~ok).sum())} query elements off by more than 1 bf16 ulp"
+        ok = C.q_within(qc, q, orc.q_allowed(l, 0))
+        assert ok.all(), f"layer {l}: {int((~ok).sum())} query elements outside the bound"
         np.testing.assert_allclose(out["w"][l, 0].double().cpu().numpy(), wv, rtol=1e-4, atol=1e-4)
 
 
@@ -106,14 +113,14 @@ def test_128k_bf16_score_with_oracle_query():
 
 
 def test_128k_bf16_end_to_end_with_query_bound():
-    """Projection inside the call: the logit may move by the effect of a one-ulp query
-    difference, bounded per entry by the oracle."""
+    """Projection inside the call: the logit may move by the effect of the query's fp32
+    accumulation and bf16 rounding, bounded per entry by the oracle."""
     w = W.WORKLOADS["lsa_step_128k_b1_bf16"]
     inp = C.make_inputs(w)
     orc = C.OracleCache(inp)
     out = run_score(inp)
     for l in range(w.L):
-        check_layer_outputs(out, inp, orc, l, 0, z_extra=orc.z_bound_from_q_ulp(l, 0))
+        check_layer_outputs(out, inp, orc, l, 0, z_extra=orc.z_bound_from_q(l, 0))
 
 
 @pytest.mark.parametrize("N", [1, 31, 1000, 4097])

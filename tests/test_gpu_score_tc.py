@@ -43,7 +43,7 @@ def test_fp8_end_to_end_with_query_bound():
     out = run_score(inp)
     for l in range(w.L):
         for b in range(w.B):
-            check_layer_outputs(out, inp, orc, l, b, z_extra=orc.z_bound_from_q_ulp(l, b))
+            check_layer_outputs(out, inp, orc, l, b, z_extra=orc.z_bound_from_q(l, b))
 
 
 @pytest.mark.parametrize("H,dI,kdt", [(48, 128, "bf16"), (64, 64, "e4m3"), (32, 64, "bf16"), (64, 256, "bf16")])
@@ -98,12 +98,16 @@ def _full_size_check(name, samples_per_unit=192, seqs=None):
         assert not ((bits[ent] != (z >= 0)) & (np.abs(z) > tz)).any()
     del out
     out = run_score(inp, want_q=True)
+    marked = {l: [] for l in range(w.L)}
     for l, b in units:
         q, _ = orc.qw(l, b)
-        assert C.q_ulp_ok(out["q"][l, b].double().cpu().numpy(), q).all()
+        assert C.q_within(out["q"][l, b].double().cpu().numpy(), q, orc.q_allowed(l, b)).all()
         bits = C.unpack(out["mask"][l, b], w.N)
         assert np.array_equal(bits, (out["logit"][l, b] >= 0).cpu().numpy())
-        assert 0.01 < bits.mean() < 0.5
+        marked[l].append(bits.mean())
+    # the bias is calibrated on pooled sequences (10% of a sample); single sequences vary
+    for l in range(w.L):
+        assert 0.02 < float(np.mean(marked[l])) < 0.3, marked[l]
     return out
 
 
