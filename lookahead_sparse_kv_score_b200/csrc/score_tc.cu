@@ -18,16 +18,22 @@
 // max |q_h / s_h| <= 448, then split as hi = e4m3(q/s), lo = e4m3(q/s - hi).  A bf16
 // value has 8 significant bits and the residual after a 4-bit e4m3 rounding has at
 // most 4, so hi + lo reproduces q/s exactly unless lo falls below the e4m3 subnormal
-// range (|q| < 2^-10 s_h).  The MMA runs the key tile against hi and then against lo
-// into the same accumulator, and s_h > 0 folds into the head weight:
-// w_h ReLU(s_h x) = (w_h s_h) ReLU(x).
+// range (|q| < 2^-10 s_h).  The B operand stacks the hi rows and the lo rows (N = 2H),
+// so one MMA gives both dot products and the epilogue adds them; s_h > 0 folds into
+// the head weight: w_h ReLU(s_h x) = (w_h s_h) ReLU(x).
 //
-// Pipeline (one persistent CTA per SM, 6 warps):
-//   warp 0       TMA producer: key tiles into an S-stage ring, query images into two
-//                slots (one per (sequence, layer) change).
-//   warp 1       TMEM allocation and the single-thread MMA issuer; two accumulators
-//                so the epilogue of tile i overlaps the MMA of tile i+1.
-//   warps 2..5   epilogue, one per TMEM lane quadrant (warp id mod 4).
+// Pipeline (one persistent CTA per SM, 12 warps).  Issuing a tcgen05.mma or a commit
+// costs a single thread on the order of a hundred cycles, comparable to the MMA's own
+// work at these small N, so the CTA runs two independent pipelines over the even and
+// the odd tiles of its range:
+//   warps 0, 1   TMA producers (one per pipeline) into that pipeline's half of the
+//                key-tile ring; warp 0 also loads the query image into one of two
+//                slots at each (sequence, layer) change.
+//   warps 2, 3   single-thread MMA issuers; warp 2 also owns the TMEM allocation.
+//                Each pipeline has two accumulators (one when N > 128).
+//   warps 4..11  two epilogue groups of four warps (one per TMEM lane quadrant).
+// Per-tile bookkeeping is incremental (no integer division on the critical path) and
+// the MMA descriptors are formed by adding constant offsets to a base descriptor.
 // Every mbarrier wait is bounded by a time limit; on expiry the kernel records
 // LSA_ERR_TIMEOUT in the status word, drains what it issued and frees its TMEM.
 #include <cuda.h>
@@ -40,7 +46,6 @@ namespace lsa {
 namespace {
 
 constexpr int kTileM = 128;
-constexpr int kThreads = 192;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
@@ -155,24 +160,6 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-}
-
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row core
 // groups 1024 bytes apart (stride byte offset), descriptor version 1.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
@@ -194,14 +181,23 @@ __host__ __device__ constexpr uint32_t instr_desc(bool fp8, int n) {
          | (static_cast<uint32_t>(kTileM >> 4) << 24);   // M >> 4
 }
 
+
 // ------------------------------------------------------------------ layout constants
+// Accumulator columns per tile: H for bf16; 2H for fp8 (hi heads then lo heads).
+template <bool kFp8, int kH>
+struct TcShape {
+  static constexpr int kN = kFp8 ? 2 * kH : kH;               // MMA N
+  static constexpr int kNumAcc = kN <= 128 ? 4 : 2;           // TMEM accumulators
+  static constexpr int kThreads = 128 + 128 * kNumAcc;        // 4 role warps + one epilogue group per accumulator
+  static constexpr int kTmemCols = kNumAcc * kN;              // 128, 256 or 512
+};
+
 struct TcLayout {
   int chunks;       // 128-byte K chunks of one key row
   int a_bytes;      // one key tile (128 rows)
-  int img_bytes;    // one query image (hi+lo for fp8)
+  int img_bytes;    // one query image (hi and lo rows for fp8)
   int ksteps;       // MMA instructions per tile
-  int stages;       // key-tile ring depth
-  int tmem_cols;    // allocated TMEM columns (2 accumulators)
+  int stages;       // key-tile ring depth (even; half per pipeline)
   size_t smem;      // dynamic shared memory
 };
 
@@ -211,13 +207,11 @@ __host__ __device__ inline TcLayout tc_layout(int H, int dI, bool fp8) {
   t.chunks = row_bytes / 128;
   t.a_bytes = kTileM * row_bytes;
   t.img_bytes = (fp8 ? 2 : 1) * H * row_bytes;
-  t.ksteps = (fp8 ? 2 : 1) * row_bytes / 32;
-  int cols = 32;
-  while (cols < 2 * H) cols *= 2;
-  t.tmem_cols = cols;
-  const int fixed = 2 * t.img_bytes + 2 * H * 4 + 1024 /*barriers*/ + 1024 /*alignment*/;
+  t.ksteps = row_bytes / 32;
+  const int fixed = 2 * t.img_bytes + 1024 /*barriers*/ + 1024 /*alignment*/;
   int s = (kSmemLimit - fixed) / t.a_bytes;
-  t.stages = s > 8 ? 8 : s;
+  s = s > 8 ? 8 : s;
+  t.stages = s & ~1;
   t.smem = static_cast<size_t>(t.stages) * t.a_bytes + fixed;
   return t;
 }
@@ -234,40 +228,70 @@ struct TcParams {
   int32_t* status;         // device status word or null
 };
 
-template <bool kFp8>
-__global__ void __launch_bounds__(kThreads, 1)
+// Two 32-column TMEM loads of this thread's lane, one wait.
+__device__ __forceinline__ void tmem_ld32x2(uint32_t t0, uint32_t t1, float (&v0)[32], float (&v1)[32]) {
+  uint32_t r[64];
+#define LSA_LD32(base, off)                                                                              \
+  asm volatile(                                                                                          \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "                                                          \
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "                          \
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"        \
+      : "=r"(r[base + 0]), "=r"(r[base + 1]), "=r"(r[base + 2]), "=r"(r[base + 3]), "=r"(r[base + 4]),  \
+        "=r"(r[base + 5]), "=r"(r[base + 6]), "=r"(r[base + 7]), "=r"(r[base + 8]), "=r"(r[base + 9]),  \
+        "=r"(r[base + 10]), "=r"(r[base + 11]), "=r"(r[base + 12]), "=r"(r[base + 13]),                 \
+        "=r"(r[base + 14]), "=r"(r[base + 15]), "=r"(r[base + 16]), "=r"(r[base + 17]),                 \
+        "=r"(r[base + 18]), "=r"(r[base + 19]), "=r"(r[base + 20]), "=r"(r[base + 21]),                 \
+        "=r"(r[base + 22]), "=r"(r[base + 23]), "=r"(r[base + 24]), "=r"(r[base + 25]),                 \
+        "=r"(r[base + 26]), "=r"(r[base + 27]), "=r"(r[base + 28]), "=r"(r[base + 29]),                 \
+        "=r"(r[base + 30]), "=r"(r[base + 31])                                                           \
+      : "r"(off))
+  LSA_LD32(0, t0);
+  LSA_LD32(32, t1);
+#undef LSA_LD32
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int j = 0; j < 32; ++j) { v0[j] = __uint_as_float(r[j]); v1[j] = __uint_as_float(r[32 + j]); }
+}
+
+// Two pipelines per CTA, split by local tile parity p: producer warp p and MMA warp 2+p.
+// Local tile i uses accumulator i % kNumAcc, drained by epilogue group i % kNumAcc
+// (warps 4+4g .. 7+4g).  The pipelines share the query slots (loaded by producer 0 and
+// released by both MMA issuers) and nothing else.
+template <bool kFp8, int kH>
+__global__ void __launch_bounds__(TcShape<kFp8, kH>::kThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
+  using S = TcShape<kFp8, kH>;
+  constexpr int kN = S::kN, kNumAcc = S::kNumAcc;
   extern __shared__ uint8_t smem_raw[];
-  const TcLayout lay = tc_layout(p.H, p.dI, kFp8);
+  const TcLayout lay = tc_layout(kH, p.dI, kFp8);
+  const int S2 = lay.stages / 2;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* a_ring = smem;                                                   // [stages][a_bytes]
   uint8_t* q_slot = a_ring + static_cast<size_t>(lay.stages) * lay.a_bytes;  // [2][img_bytes]
-  float* wf_slot = reinterpret_cast<float*>(q_slot + 2 * lay.img_bytes);     // [2][H]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(wf_slot + 2 * p.H);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(q_slot + 2 * lay.img_bytes);
   uint64_t* full = bars;                    // [8]
   uint64_t* empty = bars + 8;               // [8]
   uint64_t* qfull = bars + 16;              // [2]
   uint64_t* qempty = bars + 18;             // [2]
-  uint64_t* tfull = bars + 20;              // [2]
-  uint64_t* tempty = bars + 22;             // [2]
-  uint64_t* drain = bars + 24;              // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 26);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 27);
+  uint64_t* tfull = bars + 20;              // [4]
+  uint64_t* tempty = bars + 24;             // [4]
+  uint64_t* drain = bars + 28;              // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 30);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 31);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < lay.stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&qfull[s], 1);
-      mbar_init(&qempty[s], 1 + 4);     // MMA commit + four epilogue warps
-      mbar_init(&tfull[s], 1);
-      mbar_init(&tempty[s], 4);         // four epilogue warps
+      mbar_init(&qempty[s], 2);         // both MMA issuers
+      mbar_init(&drain[s], 1);
     }
-    mbar_init(drain, 1);
+    for (int a = 0; a < kNumAcc; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) tmem_alloc(tmem_slot, lay.tmem_cols);
+  if (warp == 2) tmem_alloc(tmem_slot, S::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -275,50 +299,61 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
 
   const long long T = static_cast<long long>(p.nUnits) * p.tiles_per_unit;
   const long long t_begin = T * blockIdx.x / gridDim.x, t_end = T * (blockIdx.x + 1) / gridDim.x;
+  const int n_local = static_cast<int>(t_end - t_begin);
+  const int unit0 = static_cast<int>(t_begin / p.tiles_per_unit);
+  const int tile0 = static_cast<int>(t_begin - static_cast<long long>(unit0) * p.tiles_per_unit);
   const int Nw = (p.N + 31) / 32;
+  const int uabs0 = p.l0 * p.B;
 
-  if (warp == 0 && lane == 0) {
-    // ---------------------------------------------------------------- producer
+  if (warp < 2 && lane == 0) {
+    // ---------------------------------------------------------------- producers
+    // Producer pp loads the key tiles of parity pp into stages [pp*S2, pp*S2+S2);
+    // producer 0 also loads the query image at every unit change.
+    const int pp = warp;
     const uint64_t policy = evict_first_policy();
-    long long cur = -1;
-    int k = -1;
-    long long issued = 0;
-    for (long long t = t_begin; t < t_end; ++t, ++issued) {
-      const long long unit = t / p.tiles_per_unit;
-      const int n0 = static_cast<int>(t - unit * p.tiles_per_unit) * kTileM;
-      const int uabs = p.l0 * p.B + static_cast<int>(unit);
-      if (unit != cur) {
+    int unit = unit0, tile = tile0, cur = -1, k = -1;
+    int j = 0, s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int i = 0; i < n_local && ok; ++i) {
+      if (pp == 0 && unit != cur) {
         cur = unit;
         ++k;
         const int slot = k & 1;
-        if (!mbar_wait(&qempty[slot], ((k >> 1) & 1) ^ 1, abort_flag)) break;
-        mbar_expect_tx(&qfull[slot], lay.img_bytes + p.H * 4);
-        bulk_load(q_slot + slot * lay.img_bytes, p.qimg + static_cast<size_t>(uabs) * lay.img_bytes,
+        if (!(ok = mbar_wait(&qempty[slot], ((k >> 1) & 1) ^ 1, abort_flag))) break;
+        mbar_expect_tx(&qfull[slot], lay.img_bytes);
+        bulk_load(q_slot + slot * lay.img_bytes, p.qimg + static_cast<size_t>(uabs0 + unit) * lay.img_bytes,
                   lay.img_bytes, &qfull[slot]);
-        bulk_load(wf_slot + slot * p.H, p.wfold + static_cast<size_t>(uabs) * p.H, p.H * 4, &qfull[slot]);
       }
-      const int s = static_cast<int>(issued % lay.stages);
-      if (!mbar_wait(&empty[s], ((issued / lay.stages) & 1) ^ 1, abort_flag)) break;
-      mbar_expect_tx(&full[s], lay.a_bytes);
-      uint8_t* dst = a_ring + static_cast<size_t>(s) * lay.a_bytes;
-      for (int c = 0; c < lay.chunks; ++c)
-        tma_load_3d(dst + c * (kTileM * 128), &kmap, c * (kFp8 ? 128 : 64), n0, uabs, &full[s], policy);
+      if ((i & 1) == pp) {
+        const int st = pp * S2 + s;
+        if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag))) break;
+        mbar_expect_tx(&full[st], lay.a_bytes);
+        uint8_t* dst = a_ring + static_cast<size_t>(st) * lay.a_bytes;
+        for (int c = 0; c < lay.chunks; ++c)
+          tma_load_3d(dst + c * (kTileM * 128), &kmap, c * (kFp8 ? 128 : 64), tile * kTileM, uabs0 + unit,
+                      &full[st], policy);
+        ++j;
+        if (++s == S2) { s = 0; ph ^= 1; }
+      }
+      if (++tile == p.tiles_per_unit) { tile = 0; ++unit; }
     }
     // drain: every key tile this thread issued has landed before the CTA exits
-    for (long long j = std::max(0ll, issued - lay.stages); j < issued; ++j) {
-      const int s = static_cast<int>(j % lay.stages);
+    for (int jj = j > S2 ? j - S2 : 0; jj < j; ++jj) {
       volatile int no_abort = 0;
-      if (!mbar_wait(&full[s], (j / lay.stages) & 1, &no_abort)) break;
+      if (!mbar_wait(&full[pp * S2 + jj % S2], (jj / S2) & 1, &no_abort)) break;
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------------------------------------------------------- MMA issuer
-    const uint32_t idesc = instr_desc(kFp8, p.H);
-    long long cur = -1;
-    int k = -1, slot = 0;
-    long long i = 0;
+  } else if ((warp == 2 || warp == 3) && lane == 0) {
+    // ---------------------------------------------------------------- MMA issuers
+    const int pp = warp - 2;
+    const uint32_t idesc = instr_desc(kFp8, kN);
+    const uint64_t dhi = smem_desc(0);
+    const uint32_t a_ring_u = smem_u32(a_ring), q_slot_u = smem_u32(q_slot);
+    int unit = unit0, tile = tile0, cur = -1, k = -1, slot = 0;
+    int s = 0;
+    uint32_t ph = 0, aph = 0;     // aph: phase bit of each accumulator
     bool ok = true;
-    for (long long t = t_begin; t < t_end && ok; ++t, ++i) {
-      const long long unit = t / p.tiles_per_unit;
+    for (int i = 0; i < n_local; ++i) {
       if (unit != cur) {
         if (cur != -1) mma_commit(&qempty[slot]);
         cur = unit;
@@ -326,73 +361,112 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
         slot = k & 1;
         if (!(ok = mbar_wait(&qfull[slot], (k >> 1) & 1, abort_flag))) break;
       }
-      const int acc = static_cast<int>(i & 1);
-      if (!(ok = mbar_wait(&tempty[acc], ((i >> 1) & 1) ^ 1, abort_flag))) break;
-      tc_fence_after();
-      const int s = static_cast<int>(i % lay.stages);
-      if (!(ok = mbar_wait(&full[s], (i / lay.stages) & 1, abort_flag))) break;
-      tc_fence_after();
-      const uint32_t a_base = smem_u32(a_ring + static_cast<size_t>(s) * lay.a_bytes);
-      const uint32_t b_base = smem_u32(q_slot + slot * lay.img_bytes);
-      const uint32_t d_tmem = tmem_base + acc * p.H;
-      const int steps_per_pass = lay.chunks * 4;     // 32-byte K steps over one key row
-      for (int ks = 0; ks < lay.ksteps; ++ks) {
-        const int ka = ks % steps_per_pass;           // fp8: second pass re-reads the same key tile
-        const uint32_t a_addr = a_base + (ka >> 2) * (kTileM * 128) + (ka & 3) * 32;
-        const uint32_t b_addr = b_base + (ks >> 2) * (p.H * 128) + (ks & 3) * 32;
-        mma<kFp8>(d_tmem, smem_desc(a_addr), smem_desc(b_addr), idesc, ks > 0 ? 1u : 0u);
+      if ((i & 1) == pp) {
+        const int a = i % kNumAcc;
+        const int st = pp * S2 + s;
+        if (!(ok = mbar_wait(&tempty[a], ((aph >> a) & 1) ^ 1, abort_flag))) break;
+        if (!(ok = mbar_wait(&full[st], ph, abort_flag))) break;
+        tc_fence_after();
+        const uint64_t adesc = dhi | (((a_ring_u + st * lay.a_bytes) >> 4) & 0x3FFFu);
+        const uint64_t bdesc = dhi | (((q_slot_u + slot * lay.img_bytes) >> 4) & 0x3FFFu);
+        const uint32_t d_tmem = tmem_base + a * kN;
+        for (int ks = 0; ks < lay.ksteps; ++ks) {
+          const uint32_t aoff = ((ks >> 2) * (kTileM * 128) + (ks & 3) * 32) >> 4;
+          const uint32_t boff = ((ks >> 2) * (kN * 128) + (ks & 3) * 32) >> 4;
+          mma<kFp8>(d_tmem, adesc + aoff, bdesc + boff, idesc, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&empty[st]);
+        mma_commit(&tfull[a]);
+        aph ^= 1u << a;
+        if (++s == S2) { s = 0; ph ^= 1; }
       }
-      mma_commit(&empty[s]);
-      mma_commit(&tfull[acc]);
+      if (++tile == p.tiles_per_unit) { tile = 0; ++unit; }
     }
     if (cur != -1 && ok) mma_commit(&qempty[slot]);
     // drain: all MMAs issued by this thread have completed
-    mma_commit(drain);
+    mma_commit(&drain[pp]);
     volatile int no_abort = 0;
-    mbar_wait(drain, 0, &no_abort);
-  } else if (warp >= 2) {
+    mbar_wait(&drain[pp], 0, &no_abort);
+  } else if (warp >= 4) {
     // ---------------------------------------------------------------- epilogue
-    const int quad = warp & 3;
+    const int g = (warp - 4) >> 2;            // accumulator: local tiles i = g, g + kNumAcc, ...
+    const int quad = warp & 3;                // TMEM lane quadrant of this warp
     const int row = quad * 32 + lane;
-    long long cur = -1;
-    int k = -1, slot = 0;
+    int unit = unit0, tile = tile0 + g;
+    while (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
+    int cur = -1;
     float bias_l = 0.f;
-    long long i = 0;
-    for (long long t = t_begin; t < t_end; ++t, ++i) {
-      const long long unit = t / p.tiles_per_unit;
-      const int n0 = static_cast<int>(t - unit * p.tiles_per_unit) * kTileM;
-      const size_t uabs = static_cast<size_t>(p.l0) * p.B + static_cast<size_t>(unit);
+    const float4* wf4 = nullptr;
+    uint32_t aph = 0;
+    // per-entry scale of the next tile, loaded one tile ahead
+    float ks_next = 1.f;
+    if (kFp8 && g < n_local) {
+      const int n = tile * kTileM + row;
+      if (n < p.N) ks_next = __ldg(p.kscale + static_cast<size_t>(uabs0 + unit) * p.N + n);
+    }
+    for (int i = g; i < n_local; i += kNumAcc) {
+      const size_t uabs = static_cast<size_t>(uabs0 + unit);
       if (unit != cur) {
-        if (cur != -1) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&qempty[slot]);
-        }
         cur = unit;
-        ++k;
-        slot = k & 1;
-        bias_l = p.bias[p.l0 + static_cast<int>(unit / p.B)];
-        if (!__all_sync(0xffffffffu, mbar_wait(&qfull[slot], (k >> 1) & 1, abort_flag))) break;
+        bias_l = __ldg(p.bias + p.l0 + unit / p.B);
+        wf4 = reinterpret_cast<const float4*>(p.wfold + uabs * kH);
       }
+      const int n0 = tile * kTileM;
       const int n = n0 + row;
       const bool valid = n < p.N;
-      float ks = 1.f;
-      if (kFp8 && valid) ks = p.kscale[uabs * p.N + n];
-      const int acc = static_cast<int>(i & 1);
-      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], (i >> 1) & 1, abort_flag))) break;
-      tc_fence_after();
-      float z = 0.f;
-      const float* wf = wf_slot + slot * p.H;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * p.H;
-      for (int c0 = 0; c0 < p.H; c0 += 32) {
-        float v[32];
-        tmem_ld32(taddr + c0, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) z = fmaf(wf[c0 + j], fmaxf(v[j], 0.f), z);
+      const float ks = ks_next;
+      // advance to this group's next tile and prefetch its scale
+      const int cur_tile = tile;
+      tile += kNumAcc;
+      while (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
+      if (kFp8 && i + kNumAcc < n_local) {
+        const int nn = tile * kTileM + row;
+        ks_next = nn < p.N ? __ldg(p.kscale + static_cast<size_t>(uabs0 + unit) * p.N + nn) : 1.f;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
-      z = fmaf(z, ks, bias_l);
+      (void)cur_tile;
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[g], aph, abort_flag))) break;
+      aph ^= 1;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + g * kN;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      constexpr int kStep = kFp8 ? 32 : (kH >= 64 ? 64 : 32);
+#pragma unroll
+      for (int c0 = 0; c0 < kH; c0 += kStep) {
+        float v0[32], v1[32];
+        if constexpr (kFp8) {
+          tmem_ld32x2(taddr + c0, taddr + kH + c0, v0, v1);         // hi heads, lo heads
+        } else if constexpr (kStep == 64) {
+          tmem_ld32x2(taddr + c0, taddr + c0 + 32, v0, v1);         // two head chunks
+        } else {
+          tmem_ld32x2(taddr + c0, taddr + c0, v0, v1);
+        }
+        if (c0 + kStep >= kH) {              // last load of this tile: release the accumulator
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[g]);
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 w = __ldg(wf4 + c0 / 4 + q4);
+          const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int jj = 4 * q4 + e;
+            const float x = kFp8 ? v0[jj] + v1[jj] : v0[jj];
+            acc[e] = fmaf(wv[e], fmaxf(x, 0.f), acc[e]);
+          }
+        }
+        if constexpr (!kFp8 && kStep == 64) {
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 w = __ldg(wf4 + (c0 + 32) / 4 + q4);
+            const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[e] = fmaf(wv[e], fmaxf(v1[4 * q4 + e], 0.f), acc[e]);
+          }
+        }
+      }
+      const float z = fmaf((acc[0] + acc[1]) + (acc[2] + acc[3]), ks, bias_l);
       if (valid) {
         if (p.logit) p.logit[uabs * p.N + n] = z;
         if (p.score) p.score[uabs * p.N + n] = sigmoid_f(z);
@@ -401,71 +475,78 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
       const int word = (n0 + quad * 32) >> 5;
       if (lane == 0 && word < Nw) p.mask[uabs * Nw + word] = bits;
     }
-    if (cur != -1) {      // warp-uniform: every lane left the loop at the same tile
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&qempty[slot]);
-    }
   }
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) raise_status(p.status, LSA_ERR_TIMEOUT);
-  if (warp == 1) {
+  if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, lay.tmem_cols);
+    tmem_dealloc(tmem_base, S::kTmemCols);
   }
 }
 
 // ------------------------------------------------------------------ query images
-// One block per (layer, sequence).  bf16: the query rows in the 128-byte-swizzled
-// K-major layout the MMA reads (16-byte unit j of row h stored at unit j ^ (h % 8)).
-// fp8: per-head power-of-two scale, hi and lo e4m3 rows in the same layout, and the
-// folded head weights w_h * s_h.
-template <bool kFp8>
-__global__ void build_qimg_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
-                                  int B, int H, int dI, int l0, uint8_t* __restrict__ img,
-                                  float* __restrict__ wfold) {
-  const size_t uabs = static_cast<size_t>(l0) * B + blockIdx.x;
-  const __nv_bfloat16* qu = q + uabs * H * dI;
-  const int row_bytes = kFp8 ? dI : 2 * dI;
-  const int img_bytes = (kFp8 ? 2 : 1) * H * row_bytes;
-  uint8_t* out = img + uabs * img_bytes;
-  if constexpr (!kFp8) {
-    for (int e = threadIdx.x; e < H * dI; e += blockDim.x) {
-      const int h = e / dI, d = e % dI;
-      const int c = d / 64, j = (d % 64) / 8, x = d % 8;
-      const size_t off = static_cast<size_t>(c) * H * 128 + h * 128 + ((j ^ (h & 7)) * 16) + x * 2;
-      *reinterpret_cast<__nv_bfloat16*>(out + off) = qu[e];
-    }
-    for (int h = threadIdx.x; h < H; h += blockDim.x) wfold[uabs * H + h] = w[uabs * H + h];
-  } else {
-    // one warp per head
-    const int lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-    const size_t lo_base = static_cast<size_t>(H) * dI;
-    for (int h = threadIdx.x >> 5; h < H; h += nwarps) {
-      float amax = 0.f;
-      for (int d = lane; d < dI; d += 32) amax = fmaxf(amax, fabsf(__bfloat162float(qu[h * dI + d])));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      // smallest power of two s with amax <= 448 s
-      int e = 0;
-      if (amax > 0.f) {
-        e = static_cast<int>(ceilf(log2f(amax / 448.f)));
-        while (amax > ldexpf(448.f, e)) ++e;
-        while (e > -126 && amax <= ldexpf(448.f, e - 1)) --e;
-      }
-      const float inv = ldexpf(1.f, -e);
-      for (int d = lane; d < dI; d += 32) {
-        const float x = __bfloat162float(qu[h * dI + d]) * inv;   // exact (power of two)
-        const __nv_fp8_e4m3 hi(x);
-        const __nv_fp8_e4m3 lo(x - static_cast<float>(hi));
-        const int c = d / 128, j = (d % 128) / 16, xx = d % 16;
-        const size_t off = static_cast<size_t>(c) * H * 128 + h * 128 + ((j ^ (h & 7)) * 16) + xx;
-        out[off] = hi.__x;
-        out[lo_base + off] = lo.__x;
-      }
-      if (lane == 0) wfold[uabs * H + h] = w[uabs * H + h] * ldexpf(1.f, e);
-    }
+// bf16: the query rows in the 128-byte-swizzled K-major layout the MMA reads (16-byte
+// unit j of row h stored at unit j ^ (h % 8)); one 16-byte unit per thread.
+__global__ void build_qimg_bf16_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
+                                       int B, int H, int dI, int l0, uint8_t* __restrict__ img,
+                                       float* __restrict__ wfold) {
+  const size_t uabs = static_cast<size_t>(l0) * B + blockIdx.y;
+  const int units = H * dI / 8;
+  const int u = blockIdx.x * blockDim.x + threadIdx.x;
+  if (u < units) {
+    const int h = u / (dI / 8), d0 = (u % (dI / 8)) * 8;
+    const int c = d0 / 64, j = (d0 % 64) / 8;
+    const uint4 v = *reinterpret_cast<const uint4*>(q + uabs * H * dI + static_cast<size_t>(h) * dI + d0);
+    *reinterpret_cast<uint4*>(img + uabs * H * dI * 2 + static_cast<size_t>(c) * H * 128 + h * 128 +
+                              ((j ^ (h & 7)) * 16)) = v;
   }
+  if (blockIdx.x == 0)
+    for (int hh = threadIdx.x; hh < H; hh += blockDim.x) wfold[uabs * H + hh] = w[uabs * H + hh];
+}
+
+// fp8: one warp per head: power-of-two scale s_h with max|q_h / s_h| <= 448, hi and lo
+// e4m3 values, and the folded head weight w_h * s_h.  In each 128-byte K chunk the
+// image holds 2H rows: row h = hi of head h, row H + h = lo of head h, swizzled like
+// the bf16 image.  Each lane handles four consecutive elements of the head row.
+__global__ void build_qimg_fp8_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
+                                      int B, int H, int dI, int l0, uint8_t* __restrict__ img,
+                                      float* __restrict__ wfold) {
+  const size_t uabs = static_cast<size_t>(l0) * B + blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (h >= H) return;
+  const __nv_bfloat16* qr = q + (uabs * H + h) * dI;
+  uint8_t* out = img + uabs * 2 * H * dI;
+  float amax = 0.f;
+  for (int d = lane * 4; d < dI; d += 128)
+    for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(__bfloat162float(qr[d + e])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  int ex = 0;   // smallest power of two s = 2^ex with amax <= 448 s
+  if (amax > 0.f) {
+    ex = static_cast<int>(ceilf(log2f(amax / 448.f)));
+    while (amax > ldexpf(448.f, ex)) ++ex;
+    while (ex > -126 && amax <= ldexpf(448.f, ex - 1)) --ex;
+  }
+  const float inv = ldexpf(1.f, -ex);
+  const int rows = 2 * H;
+  for (int d = lane * 4; d < dI; d += 128) {
+    uint32_t hi4 = 0, lo4 = 0;
+    for (int e = 0; e < 4; ++e) {
+      const float x = __bfloat162float(qr[d + e]) * inv;   // exact (power of two)
+      const __nv_fp8_e4m3 hi(x);
+      const __nv_fp8_e4m3 lo(x - static_cast<float>(hi));
+      hi4 |= static_cast<uint32_t>(hi.__x) << (8 * e);
+      lo4 |= static_cast<uint32_t>(lo.__x) << (8 * e);
+    }
+    const int c = d / 128, j = (d % 128) / 16, x = d % 16;
+    const size_t chunk = static_cast<size_t>(c) * rows * 128;
+    const int rh = h, rl = H + h;
+    *reinterpret_cast<uint32_t*>(out + chunk + rh * 128 + ((j ^ (rh & 7)) * 16) + x) = hi4;
+    *reinterpret_cast<uint32_t*>(out + chunk + rl * 128 + ((j ^ (rl & 7)) * 16) + x) = lo4;
+  }
+  if (lane == 0) wfold[uabs * H + h] = w[uabs * H + h] * ldexpf(1.f, ex);
 }
 
 // ------------------------------------------------------------------ tensor map
@@ -476,21 +557,43 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   if (!fn) {
-    void* p = nullptr;
+    void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
   }
   return fn;
+}
+
+template <bool kFp8, int kH>
+int launch_kernel(const CUtensorMap& map, const TcParams& p, const TcLayout& lay, int grid, cudaStream_t st) {
+  auto kern = score_tc_kernel<kFp8, kH>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.smem);
+  kern<<<grid, TcShape<kFp8, kH>::kThreads, lay.smem, st>>>(map, p);
+  return check_launch("score_tc");
+}
+
+template <bool kFp8>
+int launch_h(const CUtensorMap& map, const TcParams& p, const TcLayout& lay, int grid, cudaStream_t st) {
+  switch (p.H) {
+    case 32: return launch_kernel<kFp8, 32>(map, p, lay, grid, st);
+    case 64: return launch_kernel<kFp8, 64>(map, p, lay, grid, st);
+    case 128: return launch_kernel<kFp8, 128>(map, p, lay, grid, st);
+    case 256:
+      if constexpr (!kFp8) return launch_kernel<false, 256>(map, p, lay, grid, st);
+      break;
+  }
+  return fail(LSA_ERR_UNSUPPORTED, "score_tc: H=%d", p.H);
 }
 
 }  // namespace
 
 bool tc_supported(int H, int dI, int wdt, int kdt) {
   if (wdt != LSA_BF16) return false;
-  if (H < 32 || H > 256 || H % 32 != 0) return false;
+  if (H != 32 && H != 64 && H != 128 && H != 256) return false;
   const bool fp8 = kdt == LSA_E4M3;
+  if (fp8 && H > 128) return false;   // hi and lo heads share one MMA: N = 2H <= 256
   if (kdt == LSA_BF16) {
     if (dI % 64 != 0 || dI < 64 || dI > 256) return false;
   } else if (fp8) {
@@ -511,12 +614,13 @@ int launch_score_tc(const TcArgs& a, cudaStream_t st) {
   const bool fp8 = s.kdt == LSA_E4M3;
   const TcLayout lay = tc_layout(s.H, s.dI, fp8);
   // query images and folded head weights for the processed layers
+  const dim3 ig(fp8 ? (s.H + 7) / 8 : (s.H * s.dI / 8 + 255) / 256, s.B * s.nL);
   if (fp8)
-    build_qimg_kernel<true><<<s.B * s.nL, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(s.q), s.w, s.B, s.H,
-                                                        s.dI, s.l0, a.qimg, a.wfold);
+    build_qimg_fp8_kernel<<<ig, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(s.q), s.w, s.B, s.H, s.dI,
+                                              s.l0, a.qimg, a.wfold);
   else
-    build_qimg_kernel<false><<<s.B * s.nL, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(s.q), s.w, s.B,
-                                                         s.H, s.dI, s.l0, a.qimg, a.wfold);
+    build_qimg_bf16_kernel<<<ig, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(s.q), s.w, s.B, s.H, s.dI,
+                                               s.l0, a.qimg, a.wfold);
   int rc = check_launch("score_tc/query image");
   if (rc != LSA_OK) return rc;
 
@@ -545,14 +649,7 @@ int launch_score_tc(const TcArgs& a, cudaStream_t st) {
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long tiles = static_cast<long long>(p.nUnits) * p.tiles_per_unit;
   const int grid = static_cast<int>(std::min<long long>(sms, tiles));
-  if (fp8) {
-    cudaFuncSetAttribute(score_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.smem);
-    score_tc_kernel<true><<<grid, kThreads, lay.smem, st>>>(map, p);
-  } else {
-    cudaFuncSetAttribute(score_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.smem);
-    score_tc_kernel<false><<<grid, kThreads, lay.smem, st>>>(map, p);
-  }
-  return check_launch("score_tc");
+  return fp8 ? launch_h<true>(map, p, lay, grid, st) : launch_h<false>(map, p, lay, grid, st);
 }
 
 }  // namespace lsa
