@@ -25,7 +25,8 @@ Readings taken where the pages are silent (each is listed in the design notes):
   * nucleus: descending probability, equal probability -> lower index first; the
     smallest prefix whose mass reaches top_p (an entry is in it iff the mass strictly
     before it is < top_p).
-  * loss: mean BCE and mean focal loss (gamma, no alpha), reported separately.
+  * loss: mean BCE and mean focal loss (gamma, no alpha), reported separately, with
+    probabilities clamped to [2^-20, 1 - 2^-20].
 """
 from __future__ import annotations
 
@@ -238,13 +239,19 @@ def vote_labels(logits, top_p: float, theta: int):
     return count >= theta, count
 
 
-def bce_focal(prob, label, gamma: float):
+PROB_EPS = 2.0 ** -20   # probabilities are clamped to [PROB_EPS, 1 - PROB_EPS]
+
+
+def bce_focal(prob, label, gamma: float, eps: float = PROB_EPS):
     """Mean binary cross-entropy and mean focal loss ([SUMMARY] §2.3 loss; [REVIEW] 二).
 
+    p = clamp(prob, eps, 1 - eps)   (sigmoid scores saturate to exactly 0 or 1 in fp32,
+                                     where an unclamped log would be infinite; eps is a
+                                     power of two, exact in fp32 and fp64)
     BCE = -mean[y ln p + (1-y) ln(1-p)];
     FL  = -mean[y (1-p)^gamma ln p + (1-y) p^gamma ln(1-p)].
     """
-    p = np.asarray(prob, dtype=np.float64)
+    p = np.clip(np.asarray(prob, dtype=np.float64), eps, 1.0 - eps)
     y = np.asarray(label, dtype=np.float64)
     with np.errstate(divide="ignore", invalid="ignore"):
         lp = np.where(y > 0, np.log(p), 0.0)

@@ -293,8 +293,12 @@ def test_bce_focal_closed_forms():
     bce, fl = O.bce_focal([0.8, 0.2], [1, 0], 2.0)
     assert bce == pytest.approx(-math.log(0.8), rel=1e-14)
     assert fl == pytest.approx(0.04 * -math.log(0.8), rel=1e-14)
-    bce, fl = O.bce_focal([1 - 1e-12, 1e-12], [1, 0], 2.0)
+    bce, fl = O.bce_focal([1 - 1e-12, 1e-12], [1, 0], 2.0, eps=1e-15)
     assert bce == pytest.approx(1e-12, rel=1e-3)
+    # clamping: a saturated wrong score costs -ln(2^-20) = 20 ln 2, not infinity
+    bce, fl = O.bce_focal([0.0, 1.0], [1, 0], 2.0)
+    assert bce == pytest.approx(20 * math.log(2), rel=1e-12)
+    assert fl == pytest.approx((1 - 2.0 ** -20) ** 2 * 20 * math.log(2), rel=1e-12)
     bce, fl = O.bce_focal([0.9, 0.3], [1, 1], 0.0)                 # gamma = 0: FL == BCE
     assert fl == pytest.approx(bce, rel=1e-15)
 
