@@ -1,0 +1,544 @@
+#!/usr/bin/env python
+"""Benchmark of one Lookahead Sparse Attention indexer trigger on B200.
+
+One step = the whole indexer path for a batch of B sequences and the three indexer
+layers: low-rank query projection, head-fused gated score + threshold (tcgen05), OR-union,
+fetch-list compaction, cold-pool -> hot-pool gather of the newly fetched compressed-KV
+rows over the host link (on a side stream, overlapped with the next layer's scoring),
+compaction of the union and the top-k inside the fetched set.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own batch (weak scaling, no collective on the data
+path); the timed region is bracketed by a barrier and a synchronisation, and the time
+is the maximum over ranks.  Rank 0 prints one JSON line.  `--impl reference` times the
+fp64 CPU oracle on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import workloads as W  # noqa: E402
+
+METRIC = "LSA entries scored+selected/sec at 1M ctx (B=32, 3 layers); % of roofline"
+UNIT = "entry-layer scorings/s"
+DEFAULT_WORKLOAD = "lsa_step_1m_b32_fp8"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "score_tc_fp8_1m_b32_traffic.txt")
+SCORE_SRC = os.path.join(ROOT, "lookahead_sparse_kv_score_b200", "csrc", "score_tc.cu")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences per GPU (default: the workload's B); smaller batches are for profiling")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- ranks
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_pg(world: int, local: int, backend: str):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local) if backend == "nccl" else None)
+    return dist
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job(units_local: int, ms_local: float, dist, device):
+    """(total units over ranks, max device time over ranks in ms, whole-job units/s)."""
+    if dist is None:
+        return units_local, ms_local, units_local / (ms_local * 1e-3)
+    t = torch.tensor([float(units_local)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    ms = max_over_ranks(ms_local, dist, device)
+    units = int(t.item())
+    return units, ms, units / (ms * 1e-3)
+
+
+def barrier(dist, device):
+    if dist is not None:
+        dist.barrier(device_ids=[device.index] if device.type == "cuda" else None)
+
+
+# ----------------------------------------------------------------------------- inputs
+
+def device_inputs(w: W.ScoreWorkload, device):
+    """All inputs of the scoring step, generated on the device from the seeded streams."""
+    bias, direction = W.load_params(w.name)
+    h = W.hidden_states(w, device).transpose(0, 1).contiguous()           # [L][B][D]
+    Wd, Wu, Ww = W.all_layer_weights(w, device)
+    kdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8}[w.kdtype]
+    K = torch.empty(w.L, w.B, w.N, w.dI, dtype=kdt, device=device)
+    ks = torch.empty(w.L, w.B, w.N, dtype=torch.float32, device=device) if w.kdtype == "e4m3" else None
+    for l in range(w.L):
+        for b in range(w.B):
+            k, s = W.keys(w, b, l, direction[b, l].double(), 0, w.N, device)
+            K[l, b] = k
+            if ks is not None:
+                ks[l, b] = s
+    return dict(h=h, Wd=Wd, Wu=Wu, Ww=Ww, bias=bias.to(device), K=K, kscale=ks)
+
+
+def cold_pool(w: W.ScoreWorkload, device, chunk_rows=1 << 15):
+    """Pinned, device-mapped host memory [B][N][row_bytes] filled with the seeded rows."""
+    cold = torch.empty(w.B, w.N, w.row_bytes, dtype=torch.uint8, pin_memory=True)
+    for b in range(w.B):
+        for s0 in range(0, w.N, chunk_rows):
+            n = min(chunk_rows, w.N - s0)
+            cold[b, s0:s0 + n].copy_(W.cold_rows(w, b, s0, n, device), non_blocking=False)
+    return cold
+
+
+# ----------------------------------------------------------------------------- the step
+
+class Trigger:
+    """Buffers and streams of one indexer trigger; run() enqueues one step."""
+
+    def __init__(self, lsa, w: W.ScoreWorkload, inp, cold, device):
+        self.lsa, self.w, self.inp, self.cold, self.dev = lsa, w, inp, cold, device
+        B, L, N = w.B, w.L, w.N
+        self.Nw = (N + 31) // 32
+        self.cap = N
+        self.wdt = lsa.dtype_code(inp["h"])
+        self.kdt = lsa.dtype_code(inp["K"])
+        self.q = torch.empty(L, B, w.H, w.dI, dtype=inp["h"].dtype, device=device)
+        self.wv = torch.empty(L, B, w.H, dtype=torch.float32, device=device)
+        self.mask = torch.empty(L, B, self.Nw, dtype=torch.int32, device=device)
+        self.logit = torch.empty(L, B, N, dtype=torch.float32, device=device)
+        self.U = torch.zeros(B, self.Nw, dtype=torch.int32, device=device)
+        self.new = torch.empty(L, B, self.Nw, dtype=torch.int32, device=device)
+        self.idx_new = torch.empty(L, B, self.cap, dtype=torch.int32, device=device)
+        self.cnt_new = torch.zeros(L, B, dtype=torch.int32, device=device)
+        self.hot = torch.empty(L, B, self.cap, w.row_bytes, dtype=torch.uint8, device=device)
+        self.idx_U = torch.empty(B, N, dtype=torch.int32, device=device)
+        self.cnt_U = torch.zeros(B, dtype=torch.int32, device=device)
+        self.topk = torch.empty(B, w.k, dtype=torch.int32, device=device)
+        self.topk_cnt = torch.zeros(B, dtype=torch.int32, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.ws_proj = lsa.workspace(lsa.lsa_index_project_workspace_bytes(B, L, w.D, w.r, w.H, w.dI, self.wdt),
+                                     device)
+        self.ws_score = lsa.workspace(lsa.lsa_index_score_workspace_bytes(B, L, N, w.D, w.r, w.H, w.dI,
+                                                                          self.wdt, self.kdt), device)
+        self.ws_topk = lsa.workspace(lsa.lsa_topk_workspace_bytes(B, N), device)
+        self.main = torch.cuda.Stream(device)
+        self.side = torch.cuda.Stream(device)
+        self.timing = []     # per step: [(score_start, score_end, gather_start, gather_end) per layer]
+
+    def run(self, record=False):
+        """One trigger.  The three layers are scored in one launch (HBM-bound, ~1 ms) before
+        the gathers start: the gathers are host-link-bound (tens of ms) and occupy every SM,
+        so running them beside the scoring would only slow the scoring down.  Union,
+        compaction and top-k run on the main stream while the side stream gathers."""
+        lsa, w, inp = self.lsa, self.w, self.inp
+        B, L, N = w.B, w.L, w.N
+        m, sd = self.main, self.side
+        e = [torch.cuda.Event(enable_timing=record) for _ in range(2 + 2 * L)]
+        lsa.lsa_index_project(B, L, w.D, w.r, w.H, w.dI, self.wdt, inp["h"], inp["Wd"], inp["Wu"], inp["Ww"], -1,
+                              self.q, self.wv, self.ws_proj, stream=m)
+        if record:
+            e[0].record(m)
+        lsa.lsa_index_score(B, L, N, w.D, w.r, w.H, w.dI, self.wdt, None, None, None, None, inp["bias"],
+                            self.kdt, inp["K"], inp["kscale"], -1, self.q, self.wv, None, None,
+                            self.mask, self.logit, None, self.ws_score, status=self.status, stream=m)
+        if record:
+            e[1].record(m)
+        with torch.cuda.stream(m):
+            self.U.zero_()
+        for l in range(L):
+            lsa.lsa_select_union(B, self.Nw, self.mask[l], self.U, self.new[l], stream=m)
+            lsa.lsa_compact(B, N, self.new[l], self.cap, self.idx_new[l], self.cnt_new[l], self.status, stream=m)
+            ready = torch.cuda.Event()
+            ready.record(m)
+            sd.wait_event(ready)
+            if record:
+                e[2 + 2 * l].record(sd)
+            lsa.lsa_gather_cold(B, N, w.row_bytes, self.cold, self.idx_new[l], self.cnt_new[l], self.cap,
+                                self.hot[l], self.status, stream=sd)
+            if record:
+                e[3 + 2 * l].record(sd)
+        lsa.lsa_compact(B, N, self.U, N, self.idx_U, self.cnt_U, self.status, stream=m)
+        lsa.lsa_topk(B, L, N, w.k, self.idx_U, N, self.cnt_U, self.logit, self.topk, self.topk_cnt, self.ws_topk,
+                     stream=m)
+        done = torch.cuda.Event()
+        done.record(sd)
+        m.wait_event(done)
+        if record:
+            self.timing.append(e)
+
+    def kernel_times_ms(self):
+        """(score launch per step, gather launches per step) in ms."""
+        L = self.w.L
+        score = [e[0].elapsed_time(e[1]) for e in self.timing]
+        gather = [sum(e[2 + 2 * l].elapsed_time(e[3 + 2 * l]) for l in range(L)) for e in self.timing]
+        return score, gather
+
+
+# ----------------------------------------------------------------------------- measurements
+
+def host_link_gbs(device, nbytes=1 << 30, reps=5) -> float:
+    """Pinned host -> device copy bandwidth (the host link's measured peak here)."""
+    src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    best = 0.0
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dst.copy_(src, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        best = max(best, nbytes / (a.elapsed_time(b) * 1e-3) / 1e9)
+    del src, dst
+    return best
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = tempfile.mktemp(suffix=".csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), "measured"
+    return 6650.0, "fallback"
+
+
+def traffic_per_launch():
+    """DRAM bytes per score launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    kv = {}
+    for line in open(PROFILE_TRAFFIC):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    sha = hashlib.sha256(open(SCORE_SRC, "rb").read()).hexdigest()
+    if kv.get("source_sha256") != sha:
+        return None
+    try:
+        return int(kv["dram_bytes_read_per_launch"]) + int(kv["dram_bytes_write_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ----------------------------------------------------------------------------- oracle
+
+def oracle_sample_step(w: W.ScoreWorkload, raw_inputs, seqs):
+    """The oracle's indexer step on sequences `seqs` (all layers, all entries)."""
+    from oracle import lsa_oracle as O
+    from oracle import step as OS
+    units = 0
+    for b in seqs:
+        zs, marks = [], []
+        for l in range(w.L):
+            h, Wd, Wu, Ww, K, ks, bias = raw_inputs(l, b)
+            q, wv = OS.project(h, Wd, Wu, Ww, w.H, w.dI, w.wdtype)
+            z, _, mark = OS.score_layer(q, wv, bias, K, ks, w.kdtype)
+            zs.append(z)
+            marks.append(mark)
+            units += len(z)
+        OS.select(marks, zs, w.k)
+    return units
+
+
+def raw_from_device(inp, w, seqs, n_entries):
+    """Host copies (storage bytes) of the inputs of the sampled sequences."""
+    def raw(t):
+        t = t.detach().cpu().contiguous()
+        if t.dtype == torch.bfloat16:
+            return t.view(torch.int16).numpy().view(np.uint16)
+        return t.numpy()
+    cache = {}
+    Wd = [raw(inp["Wd"][l]) for l in range(w.L)]
+    Wu = [raw(inp["Wu"][l]) for l in range(w.L)]
+    Ww = [raw(inp["Ww"][l]) for l in range(w.L)]
+    bias = raw(inp["bias"])
+    for l in range(w.L):
+        for b in seqs:
+            ks = raw(inp["kscale"][l, b, :n_entries]) if inp["kscale"] is not None else None
+            cache[l, b] = (raw(inp["h"][l, b]), Wd[l], Wu[l], Ww[l], raw(inp["K"][l, b, :n_entries]), ks,
+                           float(bias[l]))
+    return lambda l, b: cache[l, b]
+
+
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=os.cpu_count() or 1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(inp, w, seqs=(0, 1)):
+    raw_inputs = raw_from_device(inp, w, seqs, w.N)
+    t0 = time.perf_counter()
+    units = oracle_sample_step(w, raw_inputs, seqs)
+    dt = time.perf_counter() - t0
+    return {"value": units / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"sequences {list(seqs)} of {w.B}, all {w.L} layers, all {w.N} entries "
+                      f"({units} entry-layer scorings, then union, compaction and top-k) in {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- arms
+
+def reference_arm(args):
+    rank, world, _ = dist_setup()
+    if rank != 0:
+        return 0
+    w = W.WORKLOADS[args.workload]
+    n_entries = min(w.N, 1 << 17)
+    seqs = (0,)
+    wsample = W.scaled(w, B=1, N=n_entries)
+    bias, direction = W.load_params(w.name)
+    h = W.hidden_states(wsample).transpose(0, 1).contiguous()
+    Wd, Wu, Ww = W.all_layer_weights(w)
+    kdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8}[w.kdtype]
+    K = torch.empty(w.L, 1, n_entries, w.dI, dtype=kdt)
+    ks = torch.empty(w.L, 1, n_entries, dtype=torch.float32) if w.kdtype == "e4m3" else None
+    for l in range(w.L):
+        k, s = W.keys(w, 0, l, direction[0, l].double(), 0, n_entries)
+        K[l, 0] = k
+        if ks is not None:
+            ks[l, 0] = s
+    inp = dict(h=h, Wd=Wd, Wu=Wu, Ww=Ww, bias=bias, K=K, kscale=ks)
+    raw_inputs = raw_from_device(inp, wsample, seqs, n_entries)
+    for _ in range(args.warmup):
+        oracle_sample_step(wsample, raw_inputs, seqs)
+    t0 = time.perf_counter()
+    units = 0
+    for _ in range(args.steps):
+        units += oracle_sample_step(wsample, raw_inputs, seqs)
+    dt = time.perf_counter() - t0
+    value = units / dt
+    sample = (f"sequence 0 of {w.B}, all {w.L} layers, first {n_entries} of {w.N} entries per step "
+              f"({units // max(args.steps, 1)} entry-layer scorings, then union, compaction and top-k)")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / max(args.steps, 1) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "layers": w.L, "N": w.N, "H_I": w.H, "d_I": w.dI,
+                       "top_k": w.k, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def our_arm(args):
+    import lookahead_sparse_kv_score_b200 as lsa
+    rank, world, local = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_pg(world, local, "nccl")
+    lsa.lib()
+    w = W.WORKLOADS[args.workload]
+    if args.batch is not None:
+        w = W.scaled(w, B=args.batch)
+    args.e2e_steps = max(1, args.e2e_steps)
+
+    inp = device_inputs(w, device)
+    cold = cold_pool(w, device)
+    trig = Trigger(lsa, w, inp, cold, device)
+    torch.cuda.synchronize()
+
+    for _ in range(max(args.warmup, 0)):
+        trig.run()
+    torch.cuda.synchronize()
+    trig.status.zero_()
+    launches0 = lsa.kernel_launches()
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(trig.main)
+    for _ in range(args.steps):
+        trig.run(record=True)
+    t_end.record(trig.main)
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    clk = clocks.stop()
+    launches = lsa.kernel_launches() - launches0
+    ms_local = t_start.elapsed_time(t_end)
+    status = int(trig.status.item())
+    if status != 0:
+        raise SystemExit(f"device status {status} ({lsa.status_string(status)}) during the timed region")
+
+    units, ms, value = whole_job(w.B * w.L * w.N * args.steps, ms_local, dist, device)
+    score_ms, gather_ms = trig.kernel_times_ms()
+    score_avg = statistics.mean(score_ms)
+    gather_avg = statistics.mean(gather_ms)
+    fetched_rows = int(trig.cnt_new.sum().item())          # rows moved by the last step
+    # algorithmic bytes of one scoring launch (all layers): the keys and their scales
+    key_bytes = w.L * w.B * w.N * (w.dI * trig.inp["K"].element_size() + (4 if w.kdtype == "e4m3" else 0))
+    hbm_peak, peak_kind = measured_peaks()
+    achieved = key_bytes / (score_avg * 1e-3) / 1e9
+    link = host_link_gbs(device)
+    gather_gbs = fetched_rows * w.row_bytes / (gather_ms[-1] * 1e-3) / 1e9
+
+    # end to end: inputs from pinned host memory every step, result read back
+    h_host = inp["h"].cpu().pin_memory()
+    K_host = inp["K"].cpu().pin_memory()
+    ks_host = inp["kscale"].cpu().pin_memory() if inp["kscale"] is not None else None
+    topk_host = torch.empty_like(trig.topk, device="cpu").pin_memory()
+    cnt_host = torch.empty_like(trig.topk_cnt, device="cpu").pin_memory()
+    h2d = h_host.numel() * h_host.element_size() + K_host.numel() * K_host.element_size() + \
+        (ks_host.numel() * 4 if ks_host is not None else 0)
+    d2h = topk_host.numel() * 4 + cnt_host.numel() * 4
+
+    def e2e_step():
+        with torch.cuda.stream(trig.main):
+            inp["h"].copy_(h_host, non_blocking=True)
+            inp["K"].copy_(K_host, non_blocking=True)
+            if ks_host is not None:
+                inp["kscale"].copy_(ks_host, non_blocking=True)
+        trig.run()
+        with torch.cuda.stream(trig.main):
+            topk_host.copy_(trig.topk, non_blocking=True)
+            cnt_host.copy_(trig.topk_cnt, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(trig.main)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(trig.main)
+    torch.cuda.synchronize()
+    _, e2e_ms, e2e_value = whole_job(w.B * w.L * w.N * args.e2e_steps, e0.elapsed_time(e1), dist, device)
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(inp, w)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.kdtype, "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "layers": w.L, "N": w.N, "D": w.D, "r": w.r, "H_I": w.H,
+                       "d_I": w.dI, "top_k": w.k, "row_bytes": w.row_bytes,
+                       "l2": "inputs larger than L2 (keys %.2f GB)" % (key_bytes / 1e9),
+                       "parallelism": f"replica per GPU x{world}"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": traffic_per_launch(),
+                         "kernel": "score_tc (lsa_index_score, all layers in one launch)",
+                         "bytes_per_launch": key_bytes, "launch_ms": score_avg, "peak_kind": peak_kind},
+            "cpu_baseline": base,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms / args.e2e_steps},
+            "clocks": clk,
+            "gpu_launches": launches,
+            "roofline_gather": {"bound": "host_link", "achieved": gather_gbs, "peak": link, "unit": "GB/s",
+                                "frac": gather_gbs / link, "traffic": None,
+                                "kernel": "gather_cold (zero-copy reads of pinned host rows)",
+                                "bytes_per_step": fetched_rows * w.row_bytes, "rows_per_step": fetched_rows,
+                                "ms_per_step": gather_avg,
+                                "peak_kind": "measured here: pinned host->device cudaMemcpy, 1 GiB"},
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return reference_arm(args)
+    return our_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

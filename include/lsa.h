@@ -62,6 +62,10 @@ const char* lsa_last_error(void);
 /* ABI version of this header: 1. */
 int lsa_abi_version(void);
 
+/* Number of kernels this library has launched in this process (all threads).  A
+ * diagnostic for callers that account for device work; it never resets. */
+unsigned long long lsa_kernel_launches(void);
+
 /* ------------------------------------------------------------------------------------
  * lsa_index_score -- low-rank indexer query + head-fused gated score + threshold.
  *
@@ -117,6 +121,23 @@ int lsa_index_score(int B, int L, int N, int D, int r, int H, int dI,
                     uint32_t* mask, float* logit, float* score, int32_t* status,
                     void* workspace, size_t workspace_bytes,
                     void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * lsa_index_project -- the low-rank indexer query alone (the first half of
+ * lsa_index_score, [SUMMARY] §2.1 memory indexer / §2.3 low-rank query projections):
+ *     q_out[l][b] = (h[l][b] W_down[l]) W_up[l]   (bf16 rounding at c and q for BF16)
+ *     w_out[l][b] = h[l][b] W_w[l]                 (fp32)
+ * Same layouts and dtypes as lsa_index_score; q_out [L][B][H][dI] in wdt and
+ * w_out [L][B][H] fp32 are required.  Feed them to lsa_index_score as q_in / w_in to
+ * score several times against one query, or to time the scoring on its own.
+ * workspace: lsa_index_project_workspace_bytes(...) bytes, 256-byte aligned.
+ * ---------------------------------------------------------------------------------- */
+size_t lsa_index_project_workspace_bytes(int B, int L, int D, int r, int H, int dI, int wdt);
+
+int lsa_index_project(int B, int L, int D, int r, int H, int dI, int wdt, const void* h,
+                      const void* W_down, const void* W_up, const void* W_w, int layer,
+                      void* q_out, float* w_out, void* workspace, size_t workspace_bytes,
+                      void* stream);
 
 /* ------------------------------------------------------------------------------------
  * lsa_select_union -- multi-layer routing in OR mode ([SUMMARY] §2.4; [REVIEW] 二:

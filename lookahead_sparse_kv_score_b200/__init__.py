@@ -70,7 +70,24 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
+def kernel_launches() -> int:
+    """Kernels liblsa has launched in this process so far."""
+    return int(lib().lsa_kernel_launches())
+
+
 # ----------------------------------------------------------------------------- scoring
+
+def lsa_index_project_workspace_bytes(B, L, D, r, H, dI, wdt) -> int:
+    return int(lib().lsa_index_project_workspace_bytes(B, L, D, r, H, dI, wdt))
+
+
+def lsa_index_project(B, L, D, r, H, dI, wdt, h, W_down, W_up, W_w, layer, q_out, w_out,
+                      workspace, stream=None):
+    _check(lib().lsa_index_project(B, L, D, r, H, dI, wdt, _p(h), _p(W_down), _p(W_up), _p(W_w),
+                                   layer, _p(q_out), _p(w_out), _p(workspace),
+                                   0 if workspace is None else workspace.numel(), _stream(stream)),
+           "lsa_index_project")
+
 
 def lsa_index_score_workspace_bytes(B, L, N, D, r, H, dI, wdt, kdt) -> int:
     return int(lib().lsa_index_score_workspace_bytes(B, L, N, D, r, H, dI, wdt, kdt))

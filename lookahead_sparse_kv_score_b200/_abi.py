@@ -16,6 +16,10 @@ SIGNATURES = {
     "lsa_status_string": (c_char_p, [c_int]),
     "lsa_last_error": (c_char_p, []),
     "lsa_abi_version": (c_int, []),
+    "lsa_kernel_launches": (ctypes.c_ulonglong, []),
+    "lsa_index_project_workspace_bytes": (c_size_t, [c_int] * 7),
+    "lsa_index_project": (c_int, [c_int] * 7 + [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
+                                               c_void_p, c_void_p, c_size_t, c_void_p]),
     "lsa_index_score_workspace_bytes": (c_size_t, [c_int] * 9),
     "lsa_index_score": (c_int, [c_int] * 7 + [c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                               c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p,

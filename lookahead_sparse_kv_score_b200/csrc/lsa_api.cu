@@ -4,12 +4,14 @@
 #include <stdio.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "lsa_common.cuh"
 
 namespace lsa {
 
 static thread_local char g_err[512] = "";
+static std::atomic<unsigned long long> g_launches{0};
 
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -19,9 +21,10 @@ int fail(int code, const char* fmt, ...) {
   return code;
 }
 
-int check_launch(const char* what) {
+int check_launch(const char* what, int kernels) {
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  g_launches.fetch_add(static_cast<unsigned long long>(kernels), std::memory_order_relaxed);
   return LSA_OK;
 }
 
@@ -75,6 +78,48 @@ const char* lsa_status_string(int status) {
 const char* lsa_last_error(void) { return g_err; }
 
 int lsa_abi_version(void) { return 1; }
+
+unsigned long long lsa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t lsa_index_project_workspace_bytes(int B, int L, int D, int r, int H, int dI, int wdt) {
+  if (B < 0 || L < 0 || D < 0 || r < 0 || H < 0 || dI < 0) return 0;
+  const ScoreWs ws = score_ws(B, L, D, r, H, dI, wdt, LSA_F32);
+  return ws.q;   // the projection scratch regions come first
+}
+
+int lsa_index_project(int B, int L, int D, int r, int H, int dI, int wdt, const void* h,
+                      const void* W_down, const void* W_up, const void* W_w, int layer,
+                      void* q_out, float* w_out, void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  if (B < 0 || L < 0 || D <= 0 || r <= 0 || H <= 0 || dI <= 0)
+    return fail(LSA_ERR_INVALID_ARG, "index_project: bad size");
+  if (wdt != LSA_F32 && wdt != LSA_BF16) return fail(LSA_ERR_UNSUPPORTED, "index_project: wdt %d", wdt);
+  if (layer < -1 || layer >= L) return fail(LSA_ERR_INVALID_ARG, "index_project: layer %d of %d", layer, L);
+  if (B == 0 || L == 0) return LSA_OK;
+  if (!h || !W_down || !W_up || !W_w || !q_out || !w_out)
+    return fail(LSA_ERR_INVALID_ARG, "index_project: null pointer");
+  const void* ptrs[] = {h, W_down, W_up, W_w, q_out, w_out};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return fail(LSA_ERR_INVALID_ARG, "index_project: pointer %p not 16-byte aligned", p);
+  const ScoreWs ws = score_ws(B, L, D, r, H, dI, wdt, LSA_F32);
+  if (!workspace || workspace_bytes < ws.q || !aligned(workspace, 256))
+    return fail(LSA_ERR_NOMEM, "index_project: workspace %zu bytes (need %zu)", workspace_bytes, ws.q);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  ProjectArgs pa{};
+  pa.B = B; pa.L = L; pa.D = D; pa.r = r; pa.H = H; pa.dI = dI; pa.wdt = wdt;
+  pa.l0 = layer < 0 ? 0 : layer; pa.nL = layer < 0 ? L : 1;
+  pa.h = h; pa.W_down = W_down; pa.W_up = W_up; pa.W_w = W_w;
+  pa.partA = reinterpret_cast<float*>(base + ws.partA);
+  pa.partW = reinterpret_cast<float*>(base + ws.partW);
+  pa.partB = reinterpret_cast<float*>(base + ws.partB);
+  pa.cbuf = reinterpret_cast<float*>(base + ws.cbuf);
+  pa.q_ws = q_out;          // written directly into the caller's buffers
+  pa.w_ws = w_out;
+  pa.q_out = nullptr;
+  pa.w_out = nullptr;
+  pa.do_q = pa.do_w = true;
+  return launch_project(pa, static_cast<cudaStream_t>(stream));
+}
 
 size_t lsa_index_score_workspace_bytes(int B, int L, int N, int D, int r, int H, int dI, int wdt,
                                        int kdt) {

@@ -13,7 +13,8 @@ namespace lsa {
 
 // ------------------------------------------------------------------ host-side errors
 int fail(int code, const char* fmt, ...);   // records the message, returns code
-int check_launch(const char* what);        // LSA_OK or LSA_ERR_CUDA after a launch
+int check_launch(const char* what, int kernels = 1);   // LSA_OK or LSA_ERR_CUDA after launching
+                                                        // `kernels` kernels (counted when OK)
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }

@@ -116,7 +116,7 @@ int project_typed(const ProjectArgs& a, cudaStream_t st) {
     reduce_splits<float><<<(unsigned)((nw + 255) / 256), 256, 0, st>>>(
         a.partW, SA, nw, 0, a.w_ws + woff, a.w_out ? a.w_out + woff : nullptr, nullptr);
   }
-  if (!a.do_q) return check_launch("project");
+  if (!a.do_q) return check_launch("project", a.do_w ? 2 : 0);
   // c = h W_down (rounded to bf16 for bf16 models)
   skinny_partial<WT, WT><<<dim3((a.r + kCols - 1) / kCols, SA, a.nL), 256, 0, st>>>(
       h, static_cast<const WT*>(a.W_down), a.B, a.D, a.r, a.l0, a.partA);
@@ -131,7 +131,7 @@ int project_typed(const ProjectArgs& a, cudaStream_t st) {
   reduce_splits<WT><<<gq, 256, 0, st>>>(a.partB, SB, nq, rb, nullptr,
                                         static_cast<WT*>(a.q_ws) + qoff,
                                         a.q_out ? static_cast<WT*>(a.q_out) + qoff : nullptr);
-  return check_launch("project");
+  return check_launch("project", (a.do_w ? 2 : 0) + 4);
 }
 
 }  // namespace
