@@ -182,6 +182,27 @@ int lsa_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int3
              void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * lsa_topk_noalloc -- lsa_topk without a workspace argument.  The pages have no
+ * counterpart of this call: it exists for callers that cannot allocate device memory
+ * when they call the library, such as a plugin inside a host framework that owns every
+ * device allocation and exposes no allocator, or a latency-critical loop whose memory
+ * is fixed once at start-up.  Arguments, results and errors are those of lsa_topk.
+ *   Scratch: a file-scope device array of 2^23 uint32 slots (32 MiB) that every GPU
+ *   which loads this part of the library's device code keeps until the process exits.  B * cap must not exceed
+ *   8,388,608; larger calls return LSA_ERR_NOMEM and launch nothing.
+ *   Set-up: the first call on each device resolves the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call before any
+ *   stream capture.
+ *   Sharing: all calls on a device use the same array, which keeps the last call's
+ *   contents (nothing needs clearing: a call writes each slot before reading it).
+ *   Calls that overlap on the GPU (for example on two streams) race on the array;
+ *   serialise them.
+ *   Allocation: no cudaMalloc, cudaFree or allocating library routine is called.
+ * ---------------------------------------------------------------------------------- */
+int lsa_topk_noalloc(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
+                     const float* logit, int32_t* topk, int32_t* topk_count, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * lsa_gather_cold -- cold pool -> hot pool copy of the fetched rows ([SUMMARY] §2.1:
  * marked compressed KV entries move from the CPU cold pool into GPU memory; [REVIEW]
  * 二: asynchronously, overlapped with compute).  For j < min(count[b], cap):

@@ -126,6 +126,12 @@ def lsa_topk(B, L, N, k, idx, cap, count, logit, topk, topk_count, workspace, st
                           _stream(stream)), "lsa_topk")
 
 
+def lsa_topk_noalloc(B, L, N, k, idx, cap, count, logit, topk, topk_count, stream=None):
+    """lsa_topk with its scratch in the library's built-in device array (no workspace)."""
+    _check(lib().lsa_topk_noalloc(B, L, N, k, _p(idx), cap, _p(count), _p(logit), _p(topk), _p(topk_count),
+                                  _stream(stream)), "lsa_topk_noalloc")
+
+
 def lsa_gather_cold(B, N, row_bytes, cold_host, idx, count, cap, hot, status=None, stream=None):
     _check(lib().lsa_gather_cold(B, N, row_bytes, _p(cold_host), _p(idx), _p(count), cap, _p(hot),
                                  _p(status), _stream(stream)), "lsa_gather_cold")

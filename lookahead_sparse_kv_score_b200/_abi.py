@@ -30,6 +30,8 @@ SIGNATURES = {
     "lsa_topk_workspace_bytes": (c_size_t, [c_int, c_int]),
     "lsa_topk": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
                          c_void_p, c_void_p, c_size_t, c_void_p]),
+    "lsa_topk_noalloc": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
+                                 c_void_p, c_void_p]),
     "lsa_gather_cold": (c_int, [c_int, c_int, c_size_t, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
                                 c_void_p, c_void_p]),
     "lsa_vote_labels_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
