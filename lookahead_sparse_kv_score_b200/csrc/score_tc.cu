@@ -257,7 +257,7 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t t0, uint32_t t1, float (&v0
 // Local tile i uses accumulator i % kNumAcc, drained by epilogue group i % kNumAcc
 // (warps 4+4g .. 7+4g).  The pipelines share the query slots (loaded by producer 0 and
 // released by both MMA issuers) and nothing else.
-template <bool kFp8, int kH>
+template <bool kFp8, int kH, int kKSteps>
 __global__ void __launch_bounds__(TcShape<kFp8, kH>::kThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
   using S = TcShape<kFp8, kH>;
@@ -305,39 +305,50 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
   const int Nw = (p.N + 31) / 32;
   const int uabs0 = p.l0 * p.B;
 
+  // Local tile i of this CTA belongs to unit (i + t_begin) / tiles_per_unit; query slot
+  // k = unit - unit0 of every unit in the range is loaded once by producer 0 and
+  // released by both MMA issuers, in unit order.
+  const int k_last = n_local > 0 ? static_cast<int>((t_end - 1) / p.tiles_per_unit) - unit0 : -1;
   if (warp < 2 && lane == 0) {
     // ---------------------------------------------------------------- producers
-    // Producer pp loads the key tiles of parity pp into stages [pp*S2, pp*S2+S2);
-    // producer 0 also loads the query image at every unit change.
+    // Producer pp loads the key tiles of parity pp (local tiles pp, pp+2, ...) into
+    // stages [pp*S2, pp*S2+S2); producer 0 also loads the query image of every unit.
     const int pp = warp;
     const uint64_t policy = evict_first_policy();
-    int unit = unit0, tile = tile0, cur = -1, k = -1;
+    int unit = unit0, tile = tile0 + pp;
+    if (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
+    int kq = -1;                              // last query slot loaded (producer 0)
+    auto load_q_through = [&](int k_to) -> bool {
+      while (kq < k_to) {
+        ++kq;
+        const int slot = kq & 1;
+        if (!mbar_wait(&qempty[slot], ((kq >> 1) & 1) ^ 1, abort_flag)) return false;
+        mbar_expect_tx(&qfull[slot], lay.img_bytes);
+        bulk_load(q_slot + slot * lay.img_bytes, p.qimg + static_cast<size_t>(uabs0 + unit0 + kq) * lay.img_bytes,
+                  lay.img_bytes, &qfull[slot]);
+      }
+      return true;
+    };
     int j = 0, s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (int i = 0; i < n_local && ok; ++i) {
-      if (pp == 0 && unit != cur) {
-        cur = unit;
-        ++k;
-        const int slot = k & 1;
-        if (!(ok = mbar_wait(&qempty[slot], ((k >> 1) & 1) ^ 1, abort_flag))) break;
-        mbar_expect_tx(&qfull[slot], lay.img_bytes);
-        bulk_load(q_slot + slot * lay.img_bytes, p.qimg + static_cast<size_t>(uabs0 + unit) * lay.img_bytes,
-                  lay.img_bytes, &qfull[slot]);
-      }
-      if ((i & 1) == pp) {
-        const int st = pp * S2 + s;
-        if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag))) break;
-        mbar_expect_tx(&full[st], lay.a_bytes);
-        uint8_t* dst = a_ring + static_cast<size_t>(st) * lay.a_bytes;
-        for (int c = 0; c < lay.chunks; ++c)
-          tma_load_3d(dst + c * (kTileM * 128), &kmap, c * (kFp8 ? 128 : 64), tile * kTileM, uabs0 + unit,
-                      &full[st], policy);
-        ++j;
-        if (++s == S2) { s = 0; ph ^= 1; }
-      }
-      if (++tile == p.tiles_per_unit) { tile = 0; ++unit; }
+    for (int i = pp; i < n_local; i += 2) {
+      if (pp == 0 && !(ok = load_q_through(unit - unit0))) break;
+      const int st = pp * S2 + s;
+      if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag))) break;
+      mbar_expect_tx(&full[st], lay.a_bytes);
+      uint8_t* dst = a_ring + static_cast<size_t>(st) * lay.a_bytes;
+#pragma unroll
+      for (int c = 0; c < kKSteps / 4; ++c)     // 128-byte K chunks of a key row
+        tma_load_3d(dst + c * (kTileM * 128), &kmap, c * (kFp8 ? 128 : 64), tile * kTileM, uabs0 + unit,
+                    &full[st], policy);
+      ++j;
+      if (++s == S2) { s = 0; ph ^= 1; }
+      tile += 2;
+      if (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
+      if (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
     }
+    if (pp == 0 && ok) load_q_through(k_last);
     // drain: every key tile this thread issued has landed before the CTA exits
     for (int jj = j > S2 ? j - S2 : 0; jj < j; ++jj) {
       volatile int no_abort = 0;
@@ -349,40 +360,46 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
     const uint32_t idesc = instr_desc(kFp8, kN);
     const uint64_t dhi = smem_desc(0);
     const uint32_t a_ring_u = smem_u32(a_ring), q_slot_u = smem_u32(q_slot);
-    int unit = unit0, tile = tile0, cur = -1, k = -1, slot = 0;
+    int unit = unit0, tile = tile0 + pp;
+    if (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
+    int kq = -1;                              // query slot in use
+    // release the current slot and acquire every later one through k_to, in order
+    auto acquire_q_through = [&](int k_to) -> bool {
+      while (kq < k_to) {
+        if (kq >= 0) mma_commit(&qempty[kq & 1]);
+        ++kq;
+        if (!mbar_wait(&qfull[kq & 1], (kq >> 1) & 1, abort_flag)) return false;
+      }
+      return true;
+    };
     int s = 0;
     uint32_t ph = 0, aph = 0;     // aph: phase bit of each accumulator
     bool ok = true;
-    for (int i = 0; i < n_local; ++i) {
-      if (unit != cur) {
-        if (cur != -1) mma_commit(&qempty[slot]);
-        cur = unit;
-        ++k;
-        slot = k & 1;
-        if (!(ok = mbar_wait(&qfull[slot], (k >> 1) & 1, abort_flag))) break;
+    for (int i = pp; i < n_local; i += 2) {
+      if (!(ok = acquire_q_through(unit - unit0))) break;
+      const int a = i % kNumAcc;
+      const int st = pp * S2 + s;
+      if (!(ok = mbar_wait(&tempty[a], ((aph >> a) & 1) ^ 1, abort_flag))) break;
+      if (!(ok = mbar_wait(&full[st], ph, abort_flag))) break;
+      tc_fence_after();
+      const uint64_t adesc = dhi | (((a_ring_u + st * lay.a_bytes) >> 4) & 0x3FFFu);
+      const uint64_t bdesc = dhi | (((q_slot_u + (kq & 1) * lay.img_bytes) >> 4) & 0x3FFFu);
+      const uint32_t d_tmem = tmem_base + a * kN;
+#pragma unroll
+      for (int ks = 0; ks < kKSteps; ++ks) {
+        constexpr uint32_t kA = (kTileM * 128) >> 4, kB = (kN * 128) >> 4;
+        mma<kFp8>(d_tmem, adesc + (ks >> 2) * kA + (ks & 3) * 2, bdesc + (ks >> 2) * kB + (ks & 3) * 2, idesc,
+                  ks > 0 ? 1u : 0u);
       }
-      if ((i & 1) == pp) {
-        const int a = i % kNumAcc;
-        const int st = pp * S2 + s;
-        if (!(ok = mbar_wait(&tempty[a], ((aph >> a) & 1) ^ 1, abort_flag))) break;
-        if (!(ok = mbar_wait(&full[st], ph, abort_flag))) break;
-        tc_fence_after();
-        const uint64_t adesc = dhi | (((a_ring_u + st * lay.a_bytes) >> 4) & 0x3FFFu);
-        const uint64_t bdesc = dhi | (((q_slot_u + slot * lay.img_bytes) >> 4) & 0x3FFFu);
-        const uint32_t d_tmem = tmem_base + a * kN;
-        for (int ks = 0; ks < lay.ksteps; ++ks) {
-          const uint32_t aoff = ((ks >> 2) * (kTileM * 128) + (ks & 3) * 32) >> 4;
-          const uint32_t boff = ((ks >> 2) * (kN * 128) + (ks & 3) * 32) >> 4;
-          mma<kFp8>(d_tmem, adesc + aoff, bdesc + boff, idesc, ks > 0 ? 1u : 0u);
-        }
-        mma_commit(&empty[st]);
-        mma_commit(&tfull[a]);
-        aph ^= 1u << a;
-        if (++s == S2) { s = 0; ph ^= 1; }
-      }
-      if (++tile == p.tiles_per_unit) { tile = 0; ++unit; }
+      mma_commit(&empty[st]);
+      mma_commit(&tfull[a]);
+      aph ^= 1u << a;
+      if (++s == S2) { s = 0; ph ^= 1; }
+      tile += 2;
+      if (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
+      if (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
     }
-    if (cur != -1 && ok) mma_commit(&qempty[slot]);
+    if (ok && acquire_q_through(k_last) && kq >= 0) mma_commit(&qempty[kq & 1]);
     // drain: all MMAs issued by this thread have completed
     mma_commit(&drain[pp]);
     volatile int no_abort = 0;
@@ -566,22 +583,37 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <bool kFp8, int kH>
+template <bool kFp8, int kH, int kKSteps>
 int launch_kernel(const CUtensorMap& map, const TcParams& p, const TcLayout& lay, int grid, cudaStream_t st) {
-  auto kern = score_tc_kernel<kFp8, kH>;
+  auto kern = score_tc_kernel<kFp8, kH, kKSteps>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.smem);
   kern<<<grid, TcShape<kFp8, kH>::kThreads, lay.smem, st>>>(map, p);
   return check_launch("score_tc");
 }
 
+template <bool kFp8, int kH>
+int launch_k(const CUtensorMap& map, const TcParams& p, const TcLayout& lay, int grid, cudaStream_t st) {
+  switch (lay.ksteps) {
+    case 4: return launch_kernel<kFp8, kH, 4>(map, p, lay, grid, st);
+    case 8: return launch_kernel<kFp8, kH, 8>(map, p, lay, grid, st);
+    case 12:
+      if constexpr (!kFp8) return launch_kernel<false, kH, 12>(map, p, lay, grid, st);
+      break;
+    case 16:
+      if constexpr (!kFp8) return launch_kernel<false, kH, 16>(map, p, lay, grid, st);
+      break;
+  }
+  return fail(LSA_ERR_UNSUPPORTED, "score_tc: %d MMA steps per tile", lay.ksteps);
+}
+
 template <bool kFp8>
 int launch_h(const CUtensorMap& map, const TcParams& p, const TcLayout& lay, int grid, cudaStream_t st) {
   switch (p.H) {
-    case 32: return launch_kernel<kFp8, 32>(map, p, lay, grid, st);
-    case 64: return launch_kernel<kFp8, 64>(map, p, lay, grid, st);
-    case 128: return launch_kernel<kFp8, 128>(map, p, lay, grid, st);
+    case 32: return launch_k<kFp8, 32>(map, p, lay, grid, st);
+    case 64: return launch_k<kFp8, 64>(map, p, lay, grid, st);
+    case 128: return launch_k<kFp8, 128>(map, p, lay, grid, st);
     case 256:
-      if constexpr (!kFp8) return launch_kernel<false, 256>(map, p, lay, grid, st);
+      if constexpr (!kFp8) return launch_k<false, 256>(map, p, lay, grid, st);
       break;
   }
   return fail(LSA_ERR_UNSUPPORTED, "score_tc: H=%d", p.H);
