@@ -52,6 +52,7 @@ def parse_args(argv=None):
                     help="sequences per GPU (default: the workload's B); smaller batches are for profiling")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-vote", action="store_true", help="skip the vote-label measurement")
     return ap.parse_args(argv)
 
 
@@ -411,6 +412,57 @@ def reference_arm(args):
     return 0
 
 
+def vote_measure(lsa, device, steps=5):
+    """Cross-layer vote labels + loss on the L=24 x P=64 x N=131072 workload: logits from the
+    generator, loss scores from the 512K workload's scorer (sequence 0, layer 0), one query
+    per position.  Returns the secondary bench object (device time of the lsa_vote_labels
+    call, HBM roofline on the 4 bytes per logit it must read)."""
+    v = W.VOTE_WORKLOADS["vote_labels_l24_p64_n131072"]
+    w2 = W.scaled(W.WORKLOADS["lsa_step_512k_b8_bf16"], B=1, L=1)
+    logits = torch.empty(v.L, v.P, v.N, dtype=torch.float32, device=device)
+    for p in range(v.P):
+        bs = W.vote_boost_set(v, p, device)
+        for l in range(v.L):
+            logits[l, p] = W.vote_logits(v, l, p, device, boost_set=bs)
+    bias, direction = W.load_params(w2.name)
+    Wd, Wu, Ww = (t[:1].contiguous() for t in W.all_layer_weights(W.WORKLOADS["lsa_step_512k_b8_bf16"], device))
+    K = W.keys(w2, 0, 0, direction[0, 0].double(), 0, w2.N, device)[0].reshape(1, 1, w2.N, w2.dI).contiguous()
+    hp = W.position_hidden(v, w2, device)
+    scores = torch.empty(v.P, v.N, dtype=torch.float32, device=device)
+    Nw2 = (w2.N + 31) // 32
+    mask = torch.empty(1, 1, Nw2, dtype=torch.int32, device=device)
+    ws = lsa.workspace(lsa.lsa_index_score_workspace_bytes(1, 1, w2.N, w2.D, w2.r, w2.H, w2.dI, 1, 1), device)
+    b1 = bias[:1].to(device)
+    for p in range(v.P):
+        lsa.lsa_index_score(1, 1, w2.N, w2.D, w2.r, w2.H, w2.dI, 1, hp[p:p + 1].reshape(1, 1, w2.D), Wd, Wu, Ww, b1,
+                            1, K, None, -1, None, None, None, None, mask, None, scores[p:p + 1], ws)
+    Nw = (v.N + 31) // 32
+    golden = torch.empty(v.P, Nw, dtype=torch.int32, device=device)
+    loss = torch.zeros(2, dtype=torch.float64, device=device)
+    vws = lsa.workspace(lsa.lsa_vote_labels_workspace_bytes(v.L, v.P, v.N), device)
+    run = lambda: lsa.lsa_vote_labels(v.L, v.P, v.N, logits, v.top_p, v.theta, golden, None, scores, v.gamma,
+                                      loss, vws)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        run()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    nbytes = logits.numel() * 4
+    hbm_peak, _ = measured_peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    out = {"workload": v.name, "ms": ms, "logits_per_s": logits.numel() / (ms * 1e-3),
+           "loss": [float(x) for x in loss.cpu()],
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                        "frac": achieved / hbm_peak, "bytes_per_launch": nbytes}}
+    del logits, K, scores
+    return out
+
+
 def our_arm(args):
     import lookahead_sparse_kv_score_b200 as lsa
     rank, world, local = dist_setup()
@@ -501,6 +553,11 @@ def our_arm(args):
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         base = cpu_baseline(inp, w)
+    vote = None
+    if rank == 0 and not args.no_vote:
+        del trig, cold
+        torch.cuda.empty_cache()
+        vote = vote_measure(lsa, device)
 
     if rank == 0:
         line = {
@@ -526,6 +583,7 @@ def our_arm(args):
                                 "bytes_per_step": fetched_rows * w.row_bytes, "rows_per_step": fetched_rows,
                                 "ms_per_step": gather_avg,
                                 "peak_kind": "measured here: pinned host->device cudaMemcpy, 1 GiB"},
+            "vote_labels": vote,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

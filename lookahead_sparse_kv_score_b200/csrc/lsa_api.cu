@@ -39,7 +39,7 @@ struct ScoreWs {
 static ScoreWs score_ws(int B, int L, int D, int r, int H, int dI, int wdt, int kdt) {
   ScoreWs o{};
   const size_t BL = static_cast<size_t>(B) * L;
-  const size_t SA = project_splits(D), SB = project_splits(r);
+  const size_t SA = project_splits(D), SB = project_splits_b(r);
   size_t off = 0;
   auto take = [&](size_t bytes) { const size_t at = off; off = align_up(off + bytes, 1024); return at; };
   o.partA = take(SA * BL * r * 4);

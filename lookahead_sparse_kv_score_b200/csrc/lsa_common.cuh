@@ -57,7 +57,8 @@ struct ProjectArgs {
   bool do_q, do_w;      // project the query / the head weights
 };
 int launch_project(const ProjectArgs& a, cudaStream_t s);
-int project_splits(int K);   // number of K-splits used for a reduction length K
+int project_splits(int K);     // reduction slices of h W_down / h W_w (length K = D)
+int project_splits_b(int K);   // reduction slices of c W_up (length K = r)
 
 // CUDA-core scoring of layers l0 .. l0+nL-1.
 struct ScoreArgs {

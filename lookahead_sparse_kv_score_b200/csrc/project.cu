@@ -5,11 +5,13 @@
 // low-rank query projections are trained.  For bf16 models c and q are rounded to
 // bf16 (nearest even) from an fp32 sum; w stays fp32.
 //
-// These are skinny products (B <= a few dozen rows against weight matrices of
-// millions of elements), bound by the weight bytes.  Each block owns 64 output
-// columns and a 256-long slice of the reduction dimension for up to 32 rows at a
-// time; the slices are summed in a fixed order by a second kernel, so results do not
-// depend on scheduling.
+// These are skinny products (B rows, a few dozen at most, against weight matrices of
+// millions of elements) bound by the weight bytes.  A block owns 32 rows x 256 output
+// columns of a slice of the reduction dimension: the weight rows stream through a
+// cp.async ring in shared memory, each thread holds a 4-row x 8-column tile in
+// registers (packed two-wide fp32 FMAs) and reads the four X values of its rows from a
+// staged, transposed X slice.  Slices are summed in a fixed order by a second kernel,
+// so the results do not depend on scheduling.
 #include <algorithm>
 
 #include "lsa_common.cuh"
@@ -17,68 +19,145 @@
 namespace lsa {
 namespace {
 
-constexpr int kCols = 64;      // output columns per block
-constexpr int kGroups = 4;     // reduction-dimension groups per block (256 threads)
-constexpr int kSplit = 256;    // reduction slice per block
-constexpr int kRows = 32;      // rows (sequences) per pass
-constexpr int kXStride = 36;   // padded row of the staged X slice (floats)
+constexpr int kTileCols = 256;     // output columns per block (32 threads x 8)
+constexpr int kTileRows = 32;      // rows per pass (8 row groups x 4)
+constexpr int kThreads = 256;
+constexpr int kXStride = 36;       // padded row of the transposed X slice (floats)
+constexpr int kSliceA = 256;       // reduction slice of h W_down / h W_w
+constexpr int kSliceB = 128;       // reduction slice of c W_up
 
 template <typename T> __device__ __forceinline__ float to_f(T v);
 template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-// part[s][li][b][m] = sum_{k in slice s} X[li][b][k] * W[l0+li][k][m]
-template <typename XT, typename WT>
-__global__ void __launch_bounds__(256)
-skinny_partial(const XT* __restrict__ X, const WT* __restrict__ W, int B, int K, int M, int l0,
-               float* __restrict__ part) {
-  __shared__ __align__(16) float xs[kSplit * kXStride];
-  const int tid = threadIdx.x;
-  const int c = tid % kCols, g = tid / kCols;
-  const int m = blockIdx.x * kCols + c;
+// acc += x * w for a pair of columns (two fp32 FMAs, round to nearest).
+__device__ __forceinline__ void fma2(float2& acc, float x, float2 w) {
+  unsigned long long a = *reinterpret_cast<unsigned long long*>(&acc);
+  const float2 xx = make_float2(x, x);
+  const unsigned long long xb = *reinterpret_cast<const unsigned long long*>(&xx);
+  const unsigned long long wb = *reinterpret_cast<const unsigned long long*>(&w);
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a) : "l"(xb), "l"(wb));
+  acc = *reinterpret_cast<float2*>(&a);
+}
+
+// 16-byte global -> shared copy, zero-filled when `valid` is false (nothing is read).
+__device__ __forceinline__ void cp16(void* dst, const void* src, bool valid) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(valid ? 16 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory"); }
+
+__device__ __forceinline__ void unpack8(const __nv_bfloat16* p, float2 (&w)[4]) {
+  const uint4 v = *reinterpret_cast<const uint4*>(p);
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = make_float2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xFFFF0000u));
+}
+__device__ __forceinline__ void unpack8(const float* p, float2 (&w)[4]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  w[0] = make_float2(a.x, a.y); w[1] = make_float2(a.z, a.w);
+  w[2] = make_float2(b.x, b.y); w[3] = make_float2(b.z, b.w);
+}
+
+constexpr int kStageRows = 8;      // weight rows per pipeline stage
+constexpr int kStages = 4;         // cp.async ring depth
+
+template <typename WT>
+constexpr size_t proj_smem(int slice) {
+  return static_cast<size_t>(slice) * kXStride * sizeof(float) +
+         static_cast<size_t>(kStages) * kStageRows * kTileCols * sizeof(WT);
+}
+
+// part[s][li][b][m] = sum_{k in slice s} X[li][b][k] * W[l0+li][k][m] for the columns of
+// W1 (m < M1) and, when blockIdx.x >= nb1, of W2 (written to part2 with M2 columns).
+// The weight rows of the slice stream through a kStages-deep cp.async ring of
+// kStageRows x 256 columns; X of the block's rows is staged once, transposed.
+template <typename XT, typename WT, int kSlice>
+__global__ void __launch_bounds__(kThreads)
+proj_partial(const XT* __restrict__ X, int B, int K, int l0,
+             const WT* __restrict__ W1, int M1, float* __restrict__ part1,
+             const WT* __restrict__ W2, int M2, float* __restrict__ part2) {
+  extern __shared__ __align__(16) uint8_t psm[];
+  float* xs = reinterpret_cast<float*>(psm);                                          // [kSlice][kXStride]
+  WT* ring = reinterpret_cast<WT*>(psm + static_cast<size_t>(kSlice) * kXStride * sizeof(float));
+  constexpr int kStageElems = kStageRows * kTileCols;                                  // per stage
+  constexpr int kVec = 16 / sizeof(WT);                                                // elements per copy
+  constexpr int kCopies = kStageElems / kVec / kThreads;                               // copies per thread
+  const int nb1 = (M1 + kTileCols - 1) / kTileCols;
+  const bool second = static_cast<int>(blockIdx.x) >= nb1;
+  const WT* W = second ? W2 : W1;
+  const int M = second ? M2 : M1;
+  float* part = second ? part2 : part1;
+  const int col0 = (second ? blockIdx.x - nb1 : blockIdx.x) * kTileCols;
+  const int tid = threadIdx.x, cg = tid & 31, rg = tid >> 5;
+  const int m = col0 + cg * 8;
   const int s = blockIdx.y, li = blockIdx.z, nL = gridDim.z;
-  const int k0 = s * kSplit, kn = min(kSplit, K - k0);
+  const int k0 = s * kSlice, kn = min(kSlice, K - k0);
+  const int nstages = (kn + kStageRows - 1) / kStageRows;
   const XT* Xl = X + static_cast<size_t>(li) * B * K;
-  const WT* Wl = W + static_cast<size_t>(l0 + li) * K * M;
-  for (int b0 = 0; b0 < B; b0 += kRows) {
-    const int nb = min(kRows, B - b0);
+  const WT* Wl = W + (static_cast<size_t>(l0 + li) * K + k0) * M;
+  auto issue = [&](int st) {
+    if (st < nstages) {
+      WT* dst = ring + (st % kStages) * kStageElems;
+#pragma unroll
+      for (int c = 0; c < kCopies; ++c) {
+        const int e = (c * kThreads + tid) * kVec;                 // element within the stage
+        const int kr = e / kTileCols, col = e % kTileCols;
+        const int k = st * kStageRows + kr;
+        const bool ok = k < kn && col0 + col < M;
+        cp16(dst + e, ok ? static_cast<const void*>(Wl + static_cast<size_t>(k) * M + col0 + col) : Wl, ok);
+      }
+    }
+    cp_commit();
+  };
+  for (int b0 = 0; b0 < B; b0 += kTileRows) {
+    const int nb = min(kTileRows, B - b0);
     __syncthreads();
-    for (int i = tid; i < kSplit * kRows; i += 256) {
-      const int kk = i % kSplit, bb = i / kSplit;
+    for (int st = 0; st < kStages - 1; ++st) issue(st);
+    for (int i = tid; i < kSlice * kTileRows; i += kThreads) {
+      const int kk = i % kSlice, bb = i / kSlice;
       float v = 0.f;
       if (kk < kn && bb < nb) v = to_f(Xl[static_cast<size_t>(b0 + bb) * K + k0 + kk]);
       xs[kk * kXStride + bb] = v;
     }
-    __syncthreads();
-    float acc[kRows];
+    const bool active = rg * 4 < nb && m < M;    // warp-uniform in rows; M is a multiple of 8
+    float2 acc[4][4];
 #pragma unroll
-    for (int bb = 0; bb < kRows; ++bb) acc[bb] = 0.f;
-    if (m < M) {
-      for (int kk = g; kk < kn; kk += kGroups) {
-        const float wv = to_f(Wl[static_cast<size_t>(k0 + kk) * M + m]);
-        const float4* xr = reinterpret_cast<const float4*>(xs + kk * kXStride);
+    for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int j = 0; j < kRows / 4; ++j) {
-          const float4 x4 = xr[j];
-          acc[4 * j + 0] = fmaf(x4.x, wv, acc[4 * j + 0]);
-          acc[4 * j + 1] = fmaf(x4.y, wv, acc[4 * j + 1]);
-          acc[4 * j + 2] = fmaf(x4.z, wv, acc[4 * j + 2]);
-          acc[4 * j + 3] = fmaf(x4.w, wv, acc[4 * j + 3]);
+      for (int c = 0; c < 4; ++c) acc[r][c] = make_float2(0.f, 0.f);
+    for (int st = 0; st < nstages; ++st) {
+      cp_wait<kStages - 2>();
+      __syncthreads();
+      issue(st + kStages - 1);
+      if (active) {
+        const WT* wst = ring + (st % kStages) * kStageElems + cg * 8;
+#pragma unroll
+        for (int kr = 0; kr < kStageRows; ++kr) {
+          const int k = st * kStageRows + kr;
+          float2 w[4];
+          unpack8(wst + kr * kTileCols, w);
+          const float4 x = *reinterpret_cast<const float4*>(xs + k * kXStride + rg * 4);
+          const float xr[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) fma2(acc[r][c], xr[r], w[c]);
         }
       }
     }
-    __syncthreads();
-    float* red = xs;   // [kGroups][kRows][kCols]
+    cp_wait<0>();
+    if (active) {
 #pragma unroll
-    for (int bb = 0; bb < kRows; ++bb) red[(g * kRows + bb) * kCols + c] = acc[bb];
-    __syncthreads();
-    for (int i = tid; i < kRows * kCols; i += 256) {
-      const int bb = i / kCols, cc = i % kCols;
-      const int mm = blockIdx.x * kCols + cc;
-      if (bb < nb && mm < M) {
-        float v = 0.f;
-        for (int gg = 0; gg < kGroups; ++gg) v += red[(gg * kRows + bb) * kCols + cc];
-        part[((static_cast<size_t>(s) * nL + li) * B + b0 + bb) * M + mm] = v;
+      for (int r = 0; r < 4; ++r) {
+        const int b = b0 + rg * 4 + r;
+        if (b - b0 >= nb) break;
+        float4* out = reinterpret_cast<float4*>(part + ((static_cast<size_t>(s) * nL + li) * B + b) * M + m);
+        out[0] = make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
+        out[1] = make_float4(acc[r][2].x, acc[r][2].y, acc[r][3].x, acc[r][3].y);
       }
     }
   }
@@ -102,43 +181,56 @@ __global__ void reduce_splits(const float* __restrict__ part, int S, size_t n, i
   }
 }
 
+unsigned grid_for(size_t n) { return static_cast<unsigned>(std::min<size_t>((n + 255) / 256, 148 * 16)); }
+
 template <typename WT>
 int project_typed(const ProjectArgs& a, cudaStream_t st) {
   const WT* h = static_cast<const WT*>(a.h) + static_cast<size_t>(a.l0) * a.B * a.D;
-  const int SA = project_splits(a.D), SB = project_splits(a.r);
+  const int SA = project_splits(a.D), SB = project_splits_b(a.r);
   const int rb = a.wdt == LSA_BF16;
   const size_t HD = static_cast<size_t>(a.H) * a.dI;
-  if (a.do_w) {   // w = h W_w
-    skinny_partial<WT, WT><<<dim3((a.H + kCols - 1) / kCols, SA, a.nL), 256, 0, st>>>(
-        h, static_cast<const WT*>(a.W_w), a.B, a.D, a.H, a.l0, a.partW);
+  int launches = 0;
+  // c = h W_down and w = h W_w in one launch (W_w's column blocks after W_down's)
+  const int nbd = a.do_q ? (a.r + kTileCols - 1) / kTileCols : 0;
+  const int nbw = a.do_w ? (a.H + kTileCols - 1) / kTileCols : 0;
+  constexpr size_t smA = proj_smem<WT>(kSliceA), smB = proj_smem<WT>(kSliceB);
+  cudaFuncSetAttribute(proj_partial<WT, WT, kSliceA>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA);
+  cudaFuncSetAttribute(proj_partial<float, WT, kSliceB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smB);
+  proj_partial<WT, WT, kSliceA><<<dim3(nbd + nbw, SA, a.nL), kThreads, smA, st>>>(
+      h, a.B, a.D, a.l0, static_cast<const WT*>(a.W_down), a.do_q ? a.r : 0, a.partA,
+      static_cast<const WT*>(a.W_w), a.H, a.partW);
+  ++launches;
+  if (a.do_w) {
     const size_t nw = static_cast<size_t>(a.nL) * a.B * a.H;
     const size_t woff = static_cast<size_t>(a.l0) * a.B * a.H;
-    reduce_splits<float><<<(unsigned)((nw + 255) / 256), 256, 0, st>>>(
-        a.partW, SA, nw, 0, a.w_ws + woff, a.w_out ? a.w_out + woff : nullptr, nullptr);
+    reduce_splits<float><<<grid_for(nw), 256, 0, st>>>(a.partW, SA, nw, 0, a.w_ws + woff,
+                                                        a.w_out ? a.w_out + woff : nullptr, nullptr);
+    ++launches;
   }
-  if (!a.do_q) return check_launch("project", a.do_w ? 2 : 0);
-  // c = h W_down (rounded to bf16 for bf16 models)
-  skinny_partial<WT, WT><<<dim3((a.r + kCols - 1) / kCols, SA, a.nL), 256, 0, st>>>(
-      h, static_cast<const WT*>(a.W_down), a.B, a.D, a.r, a.l0, a.partA);
-  const size_t nc = static_cast<size_t>(a.nL) * a.B * a.r;
-  reduce_splits<float><<<(unsigned)((nc + 255) / 256), 256, 0, st>>>(a.partA, SA, nc, rb, a.cbuf, nullptr, nullptr);
-  // q = c W_up in the storage type
-  skinny_partial<float, WT><<<dim3((unsigned)((HD + kCols - 1) / kCols), SB, a.nL), 256, 0, st>>>(
-      a.cbuf, static_cast<const WT*>(a.W_up), a.B, a.r, static_cast<int>(HD), a.l0, a.partB);
-  const size_t nq = static_cast<size_t>(a.nL) * a.B * HD;
-  const size_t qoff = static_cast<size_t>(a.l0) * a.B * HD;
-  unsigned gq = (unsigned)std::min<size_t>((nq + 255) / 256, 148 * 16);
-  reduce_splits<WT><<<gq, 256, 0, st>>>(a.partB, SB, nq, rb, nullptr,
-                                        static_cast<WT*>(a.q_ws) + qoff,
-                                        a.q_out ? static_cast<WT*>(a.q_out) + qoff : nullptr);
-  return check_launch("project", (a.do_w ? 2 : 0) + 4);
+  if (a.do_q) {
+    const size_t nc = static_cast<size_t>(a.nL) * a.B * a.r;
+    reduce_splits<float><<<grid_for(nc), 256, 0, st>>>(a.partA, SA, nc, rb, a.cbuf, nullptr, nullptr);
+    // q = c W_up in the storage type
+    proj_partial<float, WT, kSliceB><<<dim3(static_cast<unsigned>((HD + kTileCols - 1) / kTileCols), SB, a.nL),
+                                       kThreads, smB, st>>>(a.cbuf, a.B, a.r, a.l0, static_cast<const WT*>(a.W_up),
+                                                          static_cast<int>(HD), a.partB, nullptr, 0, nullptr);
+    const size_t nq = static_cast<size_t>(a.nL) * a.B * HD;
+    const size_t qoff = static_cast<size_t>(a.l0) * a.B * HD;
+    reduce_splits<WT><<<grid_for(nq), 256, 0, st>>>(a.partB, SB, nq, rb, nullptr, static_cast<WT*>(a.q_ws) + qoff,
+                                                    a.q_out ? static_cast<WT*>(a.q_out) + qoff : nullptr);
+    launches += 3;
+  }
+  return check_launch("project", launches);
 }
 
 }  // namespace
 
-int project_splits(int K) { return (K + kSplit - 1) / kSplit; }
+int project_splits(int K) { return (K + kSliceA - 1) / kSliceA; }
+int project_splits_b(int K) { return (K + kSliceB - 1) / kSliceB; }
 
 int launch_project(const ProjectArgs& a, cudaStream_t s) {
+  if ((a.r % 8) != 0 || (a.H % 8) != 0 || ((static_cast<size_t>(a.H) * a.dI) % 8) != 0)
+    return fail(LSA_ERR_UNSUPPORTED, "project: r, H and H*dI must be multiples of 8");
   if (a.wdt == LSA_BF16) return project_typed<__nv_bfloat16>(a, s);
   return project_typed<float>(a, s);
 }

@@ -67,32 +67,57 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tmp, int* t
 }
 
 // ------------------------------------------------------------------ compact
-__global__ void __launch_bounds__(1024)
+// Block (chunk, b) owns words [chunk*kCompactWords, ...) of sequence b.  Its output
+// base is the popcount of all earlier words of the sequence (re-read from L2, at most
+// a few tens of KB); its indices are staged in shared memory and written coalesced.
+constexpr int kCompactWords = 256;
+constexpr int kCompactThreads = 256;
+
+__global__ void __launch_bounds__(kCompactThreads)
 compact_kernel(const uint32_t* __restrict__ bits, int Nw, int cap, int32_t* __restrict__ idx,
                int32_t* __restrict__ count, int32_t* status) {
   __shared__ int warp_tmp[32];
   __shared__ int total;
-  const int b = blockIdx.x;
+  __shared__ int sred[kCompactThreads / 32];
+  __shared__ int32_t sidx[kCompactWords * 32];
+  const int b = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x;
   const uint32_t* row = bits + static_cast<size_t>(b) * Nw;
-  int32_t* out = idx + static_cast<size_t>(b) * cap;
-  int base = 0;
-  for (int w0 = 0; w0 < Nw; w0 += blockDim.x) {
-    const int wi = w0 + threadIdx.x;
-    uint32_t word = wi < Nw ? row[wi] : 0u;
-    const int c = __popc(word);
-    int pos = base + block_exclusive_scan(c, warp_tmp, &total);
-    while (word) {
-      const int bit = __ffs(word) - 1;
-      word &= word - 1;
-      if (pos < cap) out[pos] = wi * 32 + bit;
-      ++pos;
+  const int w0 = chunk * kCompactWords;
+  // base: set bits in words [0, w0)
+  int pc = 0;
+  const int nvec = w0 / 4;             // w0 is a multiple of 4; row is 16-byte aligned when Nw % 4 == 0
+  if ((Nw & 3) == 0) {
+    const uint4* r4 = reinterpret_cast<const uint4*>(row);
+    for (int i = tid; i < nvec; i += kCompactThreads) {
+      const uint4 v = __ldg(r4 + i);
+      pc += __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
     }
-    base += total;
-    __syncthreads();
+  } else {
+    for (int i = tid; i < w0; i += kCompactThreads) pc += __popc(__ldg(row + i));
   }
-  if (threadIdx.x == 0) {
-    count[b] = base;
-    if (base > cap) raise_status(status, LSA_ERR_CAPACITY);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) pc += __shfl_xor_sync(0xffffffffu, pc, o);
+  if ((tid & 31) == 0) sred[tid >> 5] = pc;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < kCompactThreads / 32; ++w) base += sred[w];
+  // own words
+  const int wi = w0 + tid;
+  uint32_t word = wi < Nw ? __ldg(row + wi) : 0u;
+  int pos = block_exclusive_scan(__popc(word), warp_tmp, &total);
+  while (word) {
+    const int bit = __ffs(word) - 1;
+    word &= word - 1;
+    sidx[pos++] = wi * 32 + bit;
+  }
+  __syncthreads();
+  const int n = total;
+  int32_t* out = idx + static_cast<size_t>(b) * cap;
+  for (int i = tid; i < n; i += kCompactThreads)
+    if (base + i < cap) out[base + i] = sidx[i];
+  if (chunk == static_cast<int>(gridDim.x) - 1 && tid == 0) {
+    count[b] = base + n;
+    if (base + n > cap) raise_status(status, LSA_ERR_CAPACITY);
   }
 }
 
@@ -104,14 +129,47 @@ __device__ __forceinline__ uint32_t order_key(float x) {
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kKeysPerBlock = 2048;
 
-// One block per sequence: keys, 4 radix passes of 8 bits for the k-th largest key,
-// then a stable pass that keeps every key above it and the lowest-index ties.
+// keys[b][j] = order_key(max over layers of logit[l][b][idx[b][j]]), j < min(count, cap).
+__global__ void __launch_bounds__(256)
+topk_keys_kernel(int B, int L, int N, const int32_t* __restrict__ idx, int cap, const int32_t* __restrict__ count,
+                 const float* __restrict__ logit, uint32_t* __restrict__ keys) {
+  const int b = blockIdx.y;
+  const int n = max(0, min(count[b], cap));
+  const int j0 = blockIdx.x * kKeysPerBlock;
+  if (j0 >= n) return;
+  const int32_t* ib = idx + static_cast<size_t>(b) * cap;
+  uint32_t* kb = keys + static_cast<size_t>(b) * cap;
+#pragma unroll 4
+  for (int j = j0 + threadIdx.x; j < min(n, j0 + kKeysPerBlock); j += blockDim.x) {
+    const int e = __ldg(ib + j);
+    float key = -INFINITY;
+    if (e >= 0 && e < N)
+      for (int l = 0; l < L; ++l) key = fmaxf(key, __ldg(logit + (static_cast<size_t>(l) * B + b) * N + e));
+    kb[j] = order_key(key);
+  }
+}
+
+// Four consecutive keys of candidates j .. j+3 (those at or past n read as 0, which no
+// selection counts: 0 is below every order_key of a float).
+__device__ __forceinline__ uint4 keys4(const uint32_t* kb, int j, int n, bool vec) {
+  if (vec && j + 3 < n) return __ldg(reinterpret_cast<const uint4*>(kb + j));
+  uint4 r;
+  r.x = j < n ? __ldg(kb + j) : 0u;
+  r.y = j + 1 < n ? __ldg(kb + j + 1) : 0u;
+  r.z = j + 2 < n ? __ldg(kb + j + 2) : 0u;
+  r.w = j + 3 < n ? __ldg(kb + j + 3) : 0u;
+  return r;
+}
+
+// One block per sequence: 4 radix passes of 8 bits for the k-th largest key T (count
+// of keys equal to T to keep: kk), then rounds of 4096 consecutive candidates (four per
+// thread) in which two block scans place every kept entry in ascending candidate
+// (= entry) order: all keys above T and the lowest-index ties.
 __global__ void __launch_bounds__(kTopkThreads)
-topk_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx, int cap,
-            const int32_t* __restrict__ count, const float* __restrict__ logit,
-            int32_t* __restrict__ topk, int32_t* __restrict__ topk_count,
-            uint32_t* __restrict__ keys_ws) {
+topk_select_kernel(int k, const int32_t* __restrict__ idx, int cap, const int32_t* __restrict__ count,
+                   const uint32_t* __restrict__ keys, int32_t* __restrict__ topk, int32_t* __restrict__ topk_count) {
   __shared__ int sub[kTopkWarps][256];
   __shared__ int hist[256];
   __shared__ int warp_tmp[32];
@@ -119,8 +177,7 @@ topk_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx, int cap
   __shared__ uint32_t s_prefix;
   __shared__ int s_kk;
   const int b = blockIdx.x, tid = threadIdx.x, warp = tid >> 5;
-  int n = count[b];
-  n = max(0, min(n, cap));
+  const int n = max(0, min(count[b], cap));
   const int32_t* ib = idx + static_cast<size_t>(b) * cap;
   int32_t* ob = topk + static_cast<size_t>(b) * k;
   if (n <= k) {
@@ -128,26 +185,21 @@ topk_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx, int cap
     if (tid == 0 && topk_count) topk_count[b] = n;
     return;
   }
-  uint32_t* kb = keys_ws + static_cast<size_t>(b) * cap;
+  const uint32_t* kb = keys + static_cast<size_t>(b) * cap;
+  const bool vec = (cap & 3) == 0;          // rows of the key array are 16-byte aligned
   uint32_t prefix = 0, himask = 0;
   int kk = k;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     for (int i = tid; i < kTopkWarps * 256; i += kTopkThreads) (&sub[0][0])[i] = 0;
     __syncthreads();
-    for (int j = tid; j < n; j += kTopkThreads) {
-      uint32_t u;
-      if (pass == 0) {
-        const int e = ib[j];
-        float key = -INFINITY;
-        if (e >= 0 && e < N)
-          for (int l = 0; l < L; ++l) key = fmaxf(key, logit[(static_cast<size_t>(l) * B + b) * N + e]);
-        u = order_key(key);
-        kb[j] = u;
-      } else {
-        u = kb[j];
-      }
-      if ((u & himask) == prefix) atomicAdd(&sub[warp][(u >> shift) & 255u], 1);
+#pragma unroll 2
+    for (int j = 4 * tid; j < n; j += 4 * kTopkThreads) {
+      const uint4 u4 = keys4(kb, j, n, vec);
+      const uint32_t u[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (j + e < n && (u[e] & himask) == prefix) atomicAdd(&sub[warp][(u[e] >> shift) & 255u], 1);
     }
     __syncthreads();
     if (tid < 256) {
@@ -171,22 +223,35 @@ topk_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx, int cap
     himask |= 255u << shift;
     __syncthreads();
   }
-  // prefix = k-th largest key T; kk = how many keys equal to T to keep (lowest j first)
   const uint32_t T = prefix;
   int gt_base = 0, eq_base = 0;
-  for (int j0 = 0; j0 < n; j0 += kTopkThreads) {
-    const int j = j0 + tid;
-    const uint32_t u = j < n ? kb[j] : 0u;
-    const int gt = (j < n && u > T) ? 1 : 0;
-    const int eq = (j < n && u == T) ? 1 : 0;
-    const int packed = gt | (eq << 16);
-    const int ex = block_exclusive_scan(packed, warp_tmp, &total);
-    const int gt_before = gt_base + (ex & 0xFFFF);
-    const int eq_before = eq_base + (ex >> 16);
-    if (gt || (eq && eq_before < kk)) ob[gt_before + min(eq_before, kk)] = ib[j];
-    gt_base += total & 0xFFFF;
-    eq_base += total >> 16;
-    __syncthreads();
+  for (int r0 = 0; r0 < n; r0 += 4 * kTopkThreads) {
+    const int j = r0 + 4 * tid;
+    const uint4 u4 = keys4(kb, j, n, vec);
+    const uint32_t u[4] = {u4.x, u4.y, u4.z, u4.w};
+    int gt = 0, eq = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      gt += j + e < n && u[e] > T;
+      eq += j + e < n && u[e] == T;
+    }
+    int gt_before = gt_base + block_exclusive_scan(gt, warp_tmp, &total);
+    const int gt_round = total;
+    int eq_before = eq_base + block_exclusive_scan(eq, warp_tmp, &total);
+    const int eq_round = total;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (j + e >= n) break;
+      if (u[e] > T) {
+        ob[gt_before + min(eq_before, kk)] = __ldg(ib + j + e);
+        ++gt_before;
+      } else if (u[e] == T) {
+        if (eq_before < kk) ob[gt_before + eq_before] = __ldg(ib + j + e);
+        ++eq_before;
+      }
+    }
+    gt_base += gt_round;
+    eq_base += eq_round;
   }
   if (tid == 0 && topk_count) topk_count[b] = k;
 }
@@ -204,7 +269,9 @@ int launch_union(int B, int Nw, const uint32_t* m, uint32_t* U, uint32_t* nw, cu
 int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32_t* count,
                    int32_t* status, cudaStream_t s) {
   if (B == 0) return LSA_OK;
-  compact_kernel<<<B, 1024, 0, s>>>(bits, (N + 31) / 32, cap, idx, count, status);
+  const int Nw = (N + 31) / 32;
+  const dim3 grid(std::max(1, (Nw + kCompactWords - 1) / kCompactWords), B);
+  compact_kernel<<<grid, kCompactThreads, 0, s>>>(bits, Nw, cap, idx, count, status);
   return check_launch("compact");
 }
 
@@ -212,8 +279,12 @@ int launch_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const i
                 const float* logit, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws,
                 cudaStream_t s) {
   if (B == 0) return LSA_OK;
-  topk_kernel<<<B, kTopkThreads, 0, s>>>(B, L, N, k, idx, cap, count, logit, topk, topk_count, keys_ws);
-  return check_launch("topk");
+  if (cap > 0) {
+    const dim3 g1((cap + kKeysPerBlock - 1) / kKeysPerBlock, B);
+    topk_keys_kernel<<<g1, 256, 0, s>>>(B, L, N, idx, cap, count, logit, keys_ws);
+  }
+  topk_select_kernel<<<B, kTopkThreads, 0, s>>>(k, idx, cap, count, keys_ws, topk, topk_count);
+  return check_launch("topk", cap > 0 ? 2 : 1);
 }
 
 }  // namespace lsa

@@ -147,7 +147,7 @@ class OracleCache:
         return dq @ np.abs(wv) + (np.maximum(Kd @ q.T, 0) + dq) @ self.w_allowed(l, b)
 
 
-FP32_DEPTH = 128   # longest chain of sequential fp32 additions in the projection kernels
+FP32_DEPTH = 300   # longest chain of sequential fp32 additions in the projection kernels (256 + 16 + margin)
 
 
 def bf16_ulp(x: np.ndarray) -> np.ndarray:
