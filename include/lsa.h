@@ -228,6 +228,7 @@ int lsa_gather_cold(int B, int N, size_t row_bytes, const void* cold_host,
  *     (equal pi: lower index first) whose preceding mass is < top_p.
  *     count[p][s] = #{l : s in S_{l,p}};  golden[p] bit s = count >= theta.
  *   logits [L][P][N] fp32, golden [P][Nw] uint32, counts [P][N] uint8 or NULL.
+ *   L <= 255 and P <= 65535, else LSA_ERR_UNSUPPORTED.
  *   scores [P][N] fp32 probabilities in (0,1) or NULL; when given, loss[0] = mean BCE
  *   and loss[1] = mean focal loss with exponent gamma over all P*N (device doubles).
  * workspace: lsa_vote_labels_workspace_bytes(L, P, N) bytes.

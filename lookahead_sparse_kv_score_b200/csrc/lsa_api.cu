@@ -285,6 +285,8 @@ int lsa_vote_labels(int L, int P, int N, const float* logits, float top_p, int t
                     void* workspace, size_t workspace_bytes, void* stream) {
   g_err[0] = 0;
   if (L < 0 || P < 0 || N < 0) return fail(LSA_ERR_INVALID_ARG, "vote_labels: negative size");
+  if (L > 255) return fail(LSA_ERR_UNSUPPORTED, "vote_labels: L = %d layers (at most 255: counts are bytes)", L);
+  if (P > 65535) return fail(LSA_ERR_UNSUPPORTED, "vote_labels: P = %d positions (at most 65535)", P);
   if (!(top_p > 0.f && top_p <= 1.f)) return fail(LSA_ERR_INVALID_ARG, "vote_labels: top_p must be in (0, 1]");
   if (static_cast<size_t>(P) * N == 0) return LSA_OK;
   if ((L > 0 && !logits) || !golden) return fail(LSA_ERR_INVALID_ARG, "vote_labels: null pointer");

@@ -6,29 +6,45 @@
 // golden label when at least theta = 3 of the L layers select it.  §2.3: the indexer
 // is trained with binary cross-entropy plus a focal loss.
 //
-// Nucleus of one row (layer l, position p) over N entries, without sorting:
-//   pi_s = e_s / Z with e_s = exp(x_s - max x) (fp32 exp, fp64 sums).  In descending
-//   order of x (equal x: lower index first) an entry is selected iff the mass before
-//   it is < top_p * Z.  Since pi is increasing in x, the boundary is a threshold key T
-//   on the order-preserving integer image of x: everything above T is selected, and of
-//   the c entries tied at T the first c_sel in index order, where
-//   c_sel = ceil((top_p * Z - mass above T) / e_T).  T is found by a radix select on
-//   the keys (four 8-bit digits, most significant first) whose histograms accumulate
-//   both counts and mass: each pass keeps the digit whose cumulative mass from the top
-//   first reaches the target.
+// Nucleus of one row (layer l, position p) over N entries, without sorting the row:
+//   pi_s = e_s / Z with e_s = exp(x_s - c) for a constant c near max x (fp32 exp, fp64
+//   sums).  In descending order of x (equal x: lower index first) an entry is selected
+//   iff the mass before it is < top_p * Z.  Since pi is increasing in x, the boundary
+//   is a threshold key T on the order-preserving integer image of x plus a cutoff index
+//   among the entries tied at T.  The kernel finds the crossing inside a short run of
+//   candidate entries located by a count-only histogram (window_nucleus below) and
+//   falls back to a mass-weighted radix select over the whole row (radix_nucleus) for
+//   rows the window does not resolve.
 #include <algorithm>
+#include <cmath>
+#include <type_traits>
 
 #include "lsa_common.cuh"
 
 namespace lsa {
 namespace {
 
-constexpr int kRowThreads = 512;
+#ifndef LSA_VOTE_THREADS
+#define LSA_VOTE_THREADS 512
+#endif
+constexpr int kRowThreads = LSA_VOTE_THREADS;
 constexpr int kRowWarps = kRowThreads / 32;
-constexpr int kBins = 256;
+constexpr int kBins = 256;            // radix digit bins of the whole-row select
+constexpr int kFineBins = 4096;       // linear bins of the candidate window
+constexpr int kListCap = 8192;        // candidates resolved exactly in shared memory
+constexpr float kHeadroom = 4.0f;     // window extent above the sampled maximum
+constexpr int kSubBins = 1024;      // second-level bins over the run
+constexpr int kHistInts = kFineBins + 32;   // bins plus a trash bin for entries outside the window
+constexpr int kFineSmem = kHistInts * 4 + kListCap * 8;
+constexpr int kRadixSmem = kRowWarps * kBins * 12;
+constexpr int kRowSmem = kFineSmem > kRadixSmem ? kFineSmem : kRadixSmem;
+static_assert(kFineBins % kRowThreads == 0, "bins per thread");
+static_assert(kSubBins % kRowThreads == 0, "sub-bins per thread");
+static_assert(kSubBins * 12 <= kHistInts * 4, "sub-bins reuse the histogram");
 
 __device__ __forceinline__ uint32_t order_key(float x) {
-  const uint32_t u = __float_as_uint(x);
+  uint32_t u = __float_as_uint(x);
+  if (u == 0x80000000u) u = 0u;       // -0 and +0 are the same logit
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 __device__ __forceinline__ float key_value(uint32_t k) {
@@ -43,216 +59,778 @@ __device__ __forceinline__ T block_reduce(T v, T* tmp, Op op) {
   if (lane == 0) tmp[warp] = v;
   __syncthreads();
   T r = tmp[0];
-  for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) r = op(r, tmp[w]);
+#pragma unroll 8
+  for (int w = 1; w < kRowWarps; ++w) r = op(r, tmp[w]);
   __syncthreads();
   return r;
 }
 
+// Exclusive prefix over threads (in thread order) of two fp64 values at once.
+__device__ __forceinline__ void block_scan2(double a, double b, double2* tmp, double& ea, double& eb) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double ia = a, ib = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double ta = __shfl_up_sync(0xffffffffu, ia, o), tb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) { ia += ta; ib += tb; }
+  }
+  double xa = __shfl_up_sync(0xffffffffu, ia, 1), xb = __shfl_up_sync(0xffffffffu, ib, 1);
+  if (lane == 0) { xa = 0.0; xb = 0.0; }
+  if (lane == 31) tmp[warp] = make_double2(ia, ib);
+  __syncthreads();
+  double wa = 0.0, wb = 0.0;
+  for (int w = 0; w < warp; ++w) { wa += tmp[w].x; wb += tmp[w].y; }
+  __syncthreads();
+  ea = wa + xa;
+  eb = wb + xb;
+}
+
+// Exclusive prefix over threads (in thread order) of two fp32 values at once.
+__device__ __forceinline__ void block_scan2f(float a, float b, float2* tmp, float& ea, float& eb) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float ia = a, ib = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float ta = __shfl_up_sync(0xffffffffu, ia, o), tb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) { ia += ta; ib += tb; }
+  }
+  float xa = __shfl_up_sync(0xffffffffu, ia, 1), xb = __shfl_up_sync(0xffffffffu, ib, 1);
+  if (lane == 0) { xa = 0.f; xb = 0.f; }
+  if (lane == 31) tmp[warp] = make_float2(ia, ib);
+  __syncthreads();
+  float wa = 0.f, wb = 0.f;
+  for (int w = 0; w < warp; ++w) { wa += tmp[w].x; wb += tmp[w].y; }
+  __syncthreads();
+  ea = wa + xa;
+  eb = wb + xb;
+}
+
+// Four consecutive logits starting at s (s % 4 == 0); entries at or beyond N read NaN
+// and are skipped by the callers' s + j < N checks.
+__device__ __forceinline__ float4 load4(const float* x, int s, int N, bool vec) {
+  if (vec && s + 3 < N) return __ldg(reinterpret_cast<const float4*>(x + s));
+  float4 v = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
+                         __int_as_float(0x7fc00000));
+  if (s < N) v.x = x[s];
+  if (s + 1 < N) v.y = x[s + 1];
+  if (s + 2 < N) v.z = x[s + 2];
+  if (s + 3 < N) v.w = x[s + 3];
+  return v;
+}
+
+// Calls f(value, index) for every logit of the row, four loads in flight per thread.
+template <typename F>
+__device__ __forceinline__ void row_for_each(const float* x, int N, bool vec, F&& f) {
+  const int G = (N + 3) >> 2;
+  int g = threadIdx.x;
+  auto run = [&](const float4& v, int s) {
+    f(v.x, s);
+    if (s + 1 < N) f(v.y, s + 1);
+    if (s + 2 < N) f(v.z, s + 2);
+    if (s + 3 < N) f(v.w, s + 3);
+  };
+  for (; g + 3 * kRowThreads < G; g += 4 * kRowThreads) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = load4(x, 4 * (g + u * kRowThreads), N, vec);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) run(v[u], 4 * (g + u * kRowThreads));
+  }
+  for (; g < G; g += kRowThreads) run(load4(x, 4 * g, N, vec), 4 * g);
+}
+
+// Linear bin of x in the window [a - kFineBins / inv_w, a]: floor(t) for
+// t = a inv_w - x inv_w (one fma), by an add of 2^23 rounded down (exact for
+// 0 <= t < 2^23); larger t, infinities and NaN give values >= kFineBins, x > a negative
+// values (or bin 0 within a rounding of a).
+__device__ __forceinline__ int fine_bin(float x, float a_inv_w, float inv_w) {
+  const float t = fmaf(-x, inv_w, a_inv_w);
+  return __float_as_int(__fadd_rd(t, 8388608.f)) - 0x4B000000;
+}
+
+// Ascending bitonic sort of n entries (n a power of two, >= 64).  Stages whose partner
+// distance is below 64 stay inside 64-entry blocks, one warp per block, with warp
+// barriers only.
+__device__ void bitonic_sort(unsigned long long* a, int n) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  auto local = [&](int kmin, int kmax) {
+    for (int blk = warp; blk < n / 64; blk += kRowWarps) {
+      unsigned long long* b = a + blk * 64;
+      const int base = blk * 64;
+      for (int k = kmin; k <= kmax; k <<= 1) {
+        for (int j = (k >> 1) < 32 ? (k >> 1) : 32; j > 0; j >>= 1) {
+          const int i = ((lane & ~(j - 1)) << 1) | (lane & (j - 1));
+          const unsigned long long u = b[i], v = b[i | j];
+          if ((u > v) == (((base + i) & k) == 0)) { b[i] = v; b[i | j] = u; }
+          __syncwarp();
+        }
+      }
+    }
+  };
+  local(2, 64);
+  __syncthreads();
+  for (int k = 128; k <= n; k <<= 1) {
+    for (int j = k >> 1; j >= 64; j >>= 1) {
+      for (int q = tid; q < n / 2; q += kRowThreads) {
+        const int i = ((q & ~(j - 1)) << 1) | (q & (j - 1));
+        const unsigned long long u = a[i], v = a[i | j];
+        if ((u > v) == ((i & k) == 0)) { a[i] = v; a[i | j] = u; }
+      }
+      __syncthreads();
+    }
+    local(k, k);
+    __syncthreads();
+  }
+}
+
+struct RowShared {
+  float ftmp[32];
+  double dtmp[32];
+  int itmp[32];
+  double2 d2tmp[32];
+  float2 f2tmp[32];
+  double bin_mass[kBins];
+  int bin_cnt[kBins];
+  double above, target;
+  int sel, cnt, cut, tie_base, ilo, ihi, count, jstar, sstar;
+  int nsel;
+  double before;               // mass before the crossing sub-bin
+  unsigned long long last;     // the last selected entry of the run
+  unsigned long long sub[32];  // the crossing sub-bin's entries
+};
+
+// Nucleus threshold of one row by a radix select over all N keys (four 8-bit digits,
+// most significant first) whose histograms carry counts and mass.  Used when the
+// candidate window does not apply: top_p = 1, non-finite logits, or more than
+// kListCap entries in the window's crossing bins (heavily tied rows).  Returns
+// (T, cut): an entry is selected iff key > T, or key == T and index <= cut.
+__device__ int2 radix_nucleus(const float* x, int N, float m, float top_p, uint8_t* dsm, RowShared& sh) {
+  double* hmass = reinterpret_cast<double*>(dsm);                          // [warps][256]
+  int* hcnt = reinterpret_cast<int*>(hmass + kRowWarps * kBins);           // [warps][256]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t prefix = 0, hmask = 0;
+  double above = 0.0, target = 0.0;
+  int cnt_final = 0;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = lane; i < kBins; i += 32) {
+      hmass[warp * kBins + i] = 0.0;
+      hcnt[warp * kBins + i] = 0;
+    }
+    __syncwarp();
+    for (int s = tid; s < N; s += kRowThreads) {
+      const float xv = x[s];
+      const uint32_t u = order_key(xv);
+      if ((u & hmask) == prefix) {
+        const int bin = (u >> shift) & (kBins - 1);
+        atomicAdd(&hcnt[warp * kBins + bin], 1);
+        atomicAdd(&hmass[warp * kBins + bin], static_cast<double>(__expf(xv - m)));
+      }
+    }
+    __syncthreads();
+    if (tid < kBins) {
+      double ms = 0.0;
+      int c = 0;
+      for (int w = 0; w < kRowWarps; ++w) {
+        ms += hmass[w * kBins + tid];
+        c += hcnt[w * kBins + tid];
+      }
+      sh.bin_mass[tid] = ms;
+      sh.bin_cnt[tid] = c;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // Lane j owns bins 255-8j .. 248-8j (descending).  The selected bin is the first,
+      // in descending order, at which base + cumulative mass reaches the target; if
+      // rounding keeps the total below the target (top_p close to 1), the lowest
+      // non-empty bin is taken (every entry above it is selected).
+      double loc = 0.0;
+      int nonempty = 0;
+      for (int i = 0; i < 8; ++i) {
+        const int b = kBins - 1 - (8 * lane + i);
+        loc += sh.bin_mass[b];
+        nonempty |= sh.bin_cnt[b] > 0;
+      }
+      double total = loc;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+      double incl = loc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const double excl = incl - loc;
+      const double tgt = pass == 0 ? static_cast<double>(top_p) * total : sh.target;
+      const double base = pass == 0 ? 0.0 : sh.above;
+      const unsigned reach = __ballot_sync(0xffffffffu, nonempty && base + incl >= tgt);
+      const unsigned ne = __ballot_sync(0xffffffffu, nonempty);
+      const int owner = reach ? __ffs(reach) - 1 : 31 - __clz(ne ? ne : 1u);
+      if (lane == owner) {
+        double cum = base + excl;
+        int sel = -1;
+        for (int i = 0; i < 8; ++i) {
+          const int b = kBins - 1 - (8 * lane + i);
+          if (sh.bin_cnt[b] == 0) continue;
+          if (reach && cum + sh.bin_mass[b] >= tgt) { sel = b; break; }
+          sel = b;                       // no reach: ends at the lowest non-empty bin
+          cum += sh.bin_mass[b];
+        }
+        if (!reach) cum -= sh.bin_mass[sel];   // mass strictly above the selected bin
+        sh.sel = sel;
+        sh.above = cum;
+        sh.cnt = sh.bin_cnt[sel];
+        if (pass == 0) sh.target = tgt;
+      }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(sh.sel) << shift;
+    hmask |= 255u << shift;
+    above = sh.above;
+    target = sh.target;
+    cnt_final = sh.cnt;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;
+  // number of entries tied at T to select, in index order
+  const double eT = static_cast<double>(__expf(key_value(T) - m));
+  long long want = eT > 0.0 ? static_cast<long long>(ceil((target - above) / eT)) : cnt_final;
+  want = want < 1 ? 1 : (want > cnt_final ? cnt_final : want);
+  // cutoff index: the want-th tie in index order (all ties when want == cnt_final)
+  int cut = N;
+  if (want < cnt_final) {
+    if (tid == 0) { sh.cut = N; sh.tie_base = 0; }
+    __syncthreads();
+    for (int s0 = 0; s0 < N; s0 += kRowThreads) {
+      const int s = s0 + tid;
+      const bool tie = s < N && order_key(x[s]) == T;
+      const unsigned b = __ballot_sync(0xffffffffu, tie);
+      if (lane == 0) hcnt[warp] = __popc(b);
+      __syncthreads();
+      int before = sh.tie_base;
+      for (int w = 0; w < warp; ++w) before += hcnt[w];
+      before += __popc(b & ((1u << lane) - 1));
+      if (tie && before + 1 == want) sh.cut = s;
+      __syncthreads();
+      if (tid == 0) {
+        int tot = 0;
+        for (int w = 0; w < kRowWarps; ++w) tot += hcnt[w];
+        sh.tie_base += tot;
+      }
+      __syncthreads();
+      if (sh.cut < N) break;
+    }
+    cut = sh.cut;
+    __syncthreads();
+  }
+  return make_int2(static_cast<int>(T), cut);
+}
+
+// Crossing inside a gathered run of C entries (list: ~key << 32 | index) by a full
+// sort: the run sorted by (key descending, index ascending), its mass scanned in that
+// order; the first entry whose mass before reaches the target is the first one not
+// selected.  The selected entries are or-ed into the row's words.
+__device__ bool sorted_run_crossing(unsigned long long* list, int C, double above, double target, float m0,
+                                    RowShared& sh, uint32_t* out, int2& res) {
+  const int tid = threadIdx.x;
+  int P2 = 64;
+  while (P2 < C) P2 <<= 1;
+  for (int i = C + tid; i < P2; i += kRowThreads) list[i] = ~0ull;
+  __syncthreads();
+  bitonic_sort(list, P2);
+  const int chunk = (C + kRowThreads - 1) / kRowThreads;
+  const int j0 = tid * chunk < C ? tid * chunk : C, j1 = j0 + chunk < C ? j0 + chunk : C;
+  double loc = 0.0;
+  for (int j = j0; j < j1; ++j) loc += static_cast<double>(__expf(key_value(~static_cast<uint32_t>(list[j] >> 32)) - m0));
+  double ex, ex2;
+  block_scan2(loc, 0.0, sh.d2tmp, ex, ex2);
+  if (tid == 0) sh.jstar = C + 1;     // C + 1: the crossing lies below the run
+  __syncthreads();
+  {
+    double run = ex;
+    for (int j = j0; j < j1; ++j) {
+      if (above + run >= target) { atomicMin(&sh.jstar, j); break; }
+      run += static_cast<double>(__expf(key_value(~static_cast<uint32_t>(list[j] >> 32)) - m0));
+    }
+    // every entry of the run selected, the first one below it not
+    if (j1 == C && j0 < j1 && above + run >= target) atomicMin(&sh.jstar, C);
+  }
+  __syncthreads();
+  const int js = sh.jstar;
+  if (js == 0 || js > C) return false;
+  for (int j = tid; j < js; j += kRowThreads) {
+    const uint32_t idx = static_cast<uint32_t>(list[j] & 0xffffffffu);
+    atomicOr(&out[idx >> 5], 1u << (idx & 31));
+  }
+  const unsigned long long last = list[js - 1];
+  res = make_int2(static_cast<int>(~static_cast<uint32_t>(last >> 32)), static_cast<int>(last & 0xffffffffu));
+  __syncthreads();
+  return true;
+}
+
+// Nucleus of one row from a candidate window.  Every entry outside the window
+// [m - R, m], R = ln(N / (1 - top_p)) + 1, lies below the threshold: their total mass
+// is below N e^-R < (1 - top_p) <= (1 - top_p) Z (Z >= 1 counts the maximum itself),
+// so the entries inside already hold more than top_p Z.  The window is cut into
+// kFineBins linear bins and only counts are histogrammed; with each bin's exponentials
+// bounded by its edges, the crossing bin lies in a short run [ilo, ihi] of bins.  A
+// second pass sums the exact mass above the run, writes the row's selection words
+// (entries above the run set, the run's entries clear) and gathers the run's entries,
+// which are sorted by (key descending, index ascending) and scanned for the crossing;
+// the selected part of the run is then or-ed into the words.  Returns false when the
+// run does not resolve the row (the words are then rewritten by the caller).
+__device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, float R, uint8_t* dsm,
+                              RowShared& sh, uint32_t* out, int2& res) {
+  int* hist = reinterpret_cast<int*>(dsm);
+  unsigned long long* list = reinterpret_cast<unsigned long long*>(dsm + kHistInts * 4);
+  const int tid = threadIdx.x, lane = tid & 31;
+  constexpr int kPer = kFineBins / kRowThreads;
+  const int G = (N + 3) >> 2;
+  const int Gf = vec ? (N >> 2) : 0;   // float4 groups read without checks
+  // anchor: the maximum of the first 4 * kRowThreads logits, plus headroom
+  float m0;
+  {
+    const float4 v = load4(x, 4 * tid, N, vec);
+    float mv = -INFINITY;
+    if (4 * tid < N) mv = v.x;
+    if (4 * tid + 1 < N) mv = fmaxf(mv, v.y);
+    if (4 * tid + 2 < N) mv = fmaxf(mv, v.z);
+    if (4 * tid + 3 < N) mv = fmaxf(mv, v.w);
+    m0 = block_reduce(mv, sh.ftmp, [](float a, float b) { return fmaxf(a, b); });
+  }
+  if (!isfinite(m0)) return false;
+  const float inv_w = static_cast<float>(kFineBins) / (R + kHeadroom);
+  float m = -INFINITY;
+  double Z = 0.0;
+  float a = 0.f;
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    a = attempt == 0 ? m0 + kHeadroom : m;
+    for (int i = tid; i < kHistInts; i += kRowThreads) hist[i] = 0;
+    __syncthreads();
+    float mloc = -INFINITY;
+    double zloc = 0.0;
+    // Entries above a (only when the row gets re-anchored) and NaN spoil Z, which is
+    // then discarded; entries outside the window land in the trash bin.
+    // a inv_w rounded up: every x <= a then gets t >= 0, bin 0 included
+    const float ainv = __fmul_ru(a, inv_w);
+    auto body = [&](auto full, const float4& v, int s) {
+      constexpr bool kFull = decltype(full)::value;
+      const float xs[4] = {v.x, v.y, v.z, v.w};
+      float ez = 0.f;              // at most four terms <= e^4 before the fp64 sum
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (kFull || s + j < N) {
+          mloc = fmaxf(mloc, xs[j]);
+          ez += __expf(xs[j] - m0);
+          const unsigned b = static_cast<unsigned>(fine_bin(xs[j], ainv, inv_w));
+          atomicAdd(&hist[b < static_cast<unsigned>(kFineBins) ? b : kFineBins], 1);
+        }
+      }
+      zloc += static_cast<double>(ez);
+    };
+    int g0 = tid;
+    for (; g0 + 3 * kRowThreads < Gf; g0 += 4 * kRowThreads) {
+      float4 v4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v4[u] = __ldg(reinterpret_cast<const float4*>(x) + g0 + u * kRowThreads);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) body(std::true_type{}, v4[u], 4 * (g0 + u * kRowThreads));
+    }
+    for (; g0 < G; g0 += 4 * kRowThreads) {
+      float4 v4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v4[u] = load4(x, 4 * (g0 + u * kRowThreads), N, vec);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) body(std::false_type{}, v4[u], 4 * (g0 + u * kRowThreads));
+    }
+    m = block_reduce(mloc, sh.ftmp, [](float p, float q) { return fmaxf(p, q); });
+    Z = block_reduce(zloc, sh.dtmp, [](double p, double q) { return p + q; });
+    if (!isfinite(m)) return false;
+    if (m <= a) break;
+    if (attempt == 1) return false;
+    m0 = m - kHeadroom;           // a maximum above the headroom: re-anchor at it
+  }
+  if (!(Z > 0.0) || !isfinite(Z)) return false;
+  const double target = static_cast<double>(top_p) * Z;
+  // Bounds of each bin's mass from its edges: half a bin of slack for rounding in
+  // fine_bin, 2^-10 relative for the fp32 exponentials and these fp32 sums (whose own
+  // rounding stays below 3e-6 relative).  Only the run's extent depends on them: the
+  // crossing found inside it is checked exactly below.
+  const float w = 1.f / inv_w;
+  const float A = static_cast<float>(static_cast<double>(a) - static_cast<double>(m0));
+  const float targetf = static_cast<float>(target);
+  const int b0 = tid * kPer;
+  int cnt[kPer];
+  float lo[kPer], hi[kPer], slo = 0.f, shi = 0.f;
+  {
+    const float r = expf(-w);
+    float ehi = expf(A - (b0 - 0.5f) * w) * (1.f + 1.f / 1024.f);
+    float elo = expf(A - (b0 + 1.5f) * w) * (1.f - 1.f / 1024.f);
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      cnt[i] = hist[b0 + i];
+      hi[i] = cnt[i] * ehi;
+      lo[i] = cnt[i] * elo;
+      shi += hi[i];
+      slo += lo[i];
+      ehi *= r;
+      elo *= r;
+    }
+  }
+  float chi, clo;
+  block_scan2f(shi, slo, sh.f2tmp, chi, clo);
+  if (tid == 0) { sh.ilo = kFineBins; sh.ihi = kFineBins - 1; }
+  __syncthreads();
+  {
+    int ilo = kFineBins, ihi = kFineBins;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      chi += hi[i];
+      clo += lo[i];
+      if (ilo == kFineBins && cnt[i] > 0 && chi >= targetf) ilo = b0 + i;
+      if (ihi == kFineBins && cnt[i] > 0 && clo >= targetf) ihi = b0 + i;
+    }
+    if (ilo < kFineBins) atomicMin(&sh.ilo, ilo);
+    if (ihi < kFineBins) atomicMin(&sh.ihi, ihi);
+  }
+  __syncthreads();
+  const int ilo = sh.ilo, ihi = sh.ihi;
+  if (ilo >= kFineBins || ihi < ilo) return false;
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) c += (b0 + i >= ilo && b0 + i <= ihi) ? cnt[i] : 0;
+  const int Cbins = block_reduce(c, sh.itmp, [](int p, int q) { return p + q; });
+  if (Cbins > kListCap || Cbins == 0) return false;
+  // Exact mass above the run, the row's words, the run's entries.  The pass splits the
+  // row at two thresholds in x placed at the run's bin edges; any split monotone in x
+  // serves, since the crossing found among the gathered entries is checked exactly
+  // against the mass above them.
+  const float xu = a - static_cast<float>(ilo) * w;        // above the run: x > xu
+  const float xl = a - static_cast<float>(ihi + 1) * w;    // in the run: xl < x <= xu
+  if (tid == 0) sh.count = 0;
+  __syncthreads();
+  double aloc = 0.0;
+  {
+    const int Nw = (N + 31) >> 5;
+    const int Gr = (G + 31) & ~31;      // whole warps per iteration
+    auto body = [&](auto full, const float4& v, int s) {
+      constexpr bool kFull = decltype(full)::value;
+      const float xs[4] = {v.x, v.y, v.z, v.w};
+      uint32_t nib = 0, inm = 0;
+      float ea = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (kFull || s + j < N) {
+          const bool up = xs[j] > xu;
+          const float e = __expf(xs[j] - m0);
+          ea += up ? e : 0.f;
+          nib |= static_cast<uint32_t>(up) << j;
+          inm |= static_cast<uint32_t>(!up && xs[j] > xl) << j;
+        }
+      }
+      aloc += static_cast<double>(ea);
+      uint32_t word = nib << (4 * (lane & 7));
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      word |= __shfl_xor_sync(0xffffffffu, word, 2);
+      word |= __shfl_xor_sync(0xffffffffu, word, 4);
+      if ((lane & 7) == 0 && (kFull || s < Nw * 32)) out[s >> 5] = word;
+      if (inm) {
+        int pos = atomicAdd(&sh.count, __popc(inm));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if ((inm >> j) & 1u) {
+            if (pos < kListCap)
+              list[pos] = (static_cast<unsigned long long>(~order_key(xs[j])) << 32) | static_cast<uint32_t>(s + j);
+            ++pos;
+          }
+        }
+      }
+    };
+    int g0 = tid;
+    // whole warps whose four groups are all full
+    for (; (g0 - lane) + 31 + 3 * kRowThreads < Gf; g0 += 4 * kRowThreads) {
+      float4 v4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v4[u] = __ldg(reinterpret_cast<const float4*>(x) + g0 + u * kRowThreads);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) body(std::true_type{}, v4[u], 4 * (g0 + u * kRowThreads));
+    }
+    for (; g0 < Gr; g0 += 4 * kRowThreads) {
+      float4 v4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v4[u] = load4(x, 4 * (g0 + u * kRowThreads), N, vec);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) body(std::false_type{}, v4[u], 4 * (g0 + u * kRowThreads));
+    }
+  }
+  const double above = block_reduce(aloc, sh.dtmp, [](double p, double q) { return p + q; });
+  const int C = sh.count;
+  if (!(above < target) || C == 0 || C > kListCap) return false;
+  // Second level: the run's entries in kSubBins sub-bins by x (monotone, so every entry
+  // of a sub-bin precedes every entry of a later one), with counts and fp64 mass.  The
+  // crossing sub-bin is the first whose cumulative mass reaches the target; its few
+  // entries are ranked by (key descending, index ascending) in one warp.
+  int* scnt = hist;
+  double* smass = reinterpret_cast<double*>(dsm + kSubBins * 4);
+  const float inv_ws = static_cast<float>(kSubBins) / fmaxf(xu - xl, 1e-30f);
+  auto sub_bin = [&](unsigned long long ent) {
+    const float xv = key_value(~static_cast<uint32_t>(ent >> 32));
+    const int sb = __float_as_int(__fadd_rd((xu - xv) * inv_ws, 8388608.f)) - 0x4B000000;
+    return sb < 0 ? 0 : (sb >= kSubBins ? kSubBins - 1 : sb);
+  };
+  for (int i = tid; i < kSubBins; i += kRowThreads) { scnt[i] = 0; smass[i] = 0.0; }
+  if (tid == 0) { sh.sstar = kSubBins; sh.nsel = 0; }
+  __syncthreads();
+  for (int j = tid; j < C; j += kRowThreads) {
+    const unsigned long long ent = list[j];
+    const int sb = sub_bin(ent);
+    atomicAdd(&scnt[sb], 1);
+    atomicAdd(&smass[sb], static_cast<double>(__expf(key_value(~static_cast<uint32_t>(ent >> 32)) - m0)));
+  }
+  __syncthreads();
+  constexpr int kSubPer = kSubBins / kRowThreads;
+  const int s0 = tid * kSubPer;
+  double ms[kSubPer], sloc = 0.0;
+#pragma unroll
+  for (int i = 0; i < kSubPer; ++i) { ms[i] = smass[s0 + i]; sloc += ms[i]; }
+  double sex, sex2;
+  block_scan2(sloc, 0.0, sh.d2tmp, sex, sex2);
+  {
+    double cum = above + sex;
+#pragma unroll
+    for (int i = 0; i < kSubPer; ++i) {
+      if (cum + ms[i] >= target) { atomicMin(&sh.sstar, s0 + i); break; }
+      cum += ms[i];
+    }
+  }
+  __syncthreads();
+  const int S = sh.sstar;
+  if (S >= kSubBins) return false;    // the crossing lies below the run
+  if (tid == S / kSubPer) {           // only the owner of S holds the sum before it
+    double cum = above + sex;
+    for (int i = 0; i < S - s0; ++i) cum += ms[i];
+    sh.before = cum;
+  }
+  const int nS = scnt[S];
+  if (nS > 32) return sorted_run_crossing(list, C, above, target, m0, sh, out, res);   // dense: sort the run
+  for (int j = tid; j < C; j += kRowThreads) {
+    const unsigned long long ent = list[j];
+    if (sub_bin(ent) == S) {
+      const int at = atomicAdd(&sh.nsel, 1);
+      if (at < 32) sh.sub[at] = ent;
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    const unsigned long long mine = lane < nS ? sh.sub[lane] : ~0ull;
+    const double em =
+        lane < nS ? static_cast<double>(__expf(key_value(~static_cast<uint32_t>(mine >> 32)) - m0)) : 0.0;
+    double mb = 0.0;                  // mass of the sub-bin's entries before this one
+    for (int o = 0; o < nS; ++o) {
+      const unsigned long long other = __shfl_sync(0xffffffffu, mine, o);
+      const double eo = __shfl_sync(0xffffffffu, em, o);
+      if (other < mine) mb += eo;
+    }
+    const bool sel = lane < nS && sh.before + mb < target;
+    unsigned long long lastv = sel ? mine : 0ull;   // the largest selected, in sorted order
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long t = __shfl_xor_sync(0xffffffffu, lastv, o);
+      lastv = t > lastv ? t : lastv;
+    }
+    if (lane == 0) sh.last = lastv;
+  }
+  __syncthreads();
+  const unsigned long long last = sh.last;
+  if (last == 0ull) return false;
+  // the selected part of the run: earlier sub-bins, and the crossing sub-bin's entries
+  // up to the last selected one
+  for (int j = tid; j < C; j += kRowThreads) {
+    const unsigned long long ent = list[j];
+    const int sb = sub_bin(ent);
+    if (sb < S || (sb == S && ent <= last)) {
+      const uint32_t idx = static_cast<uint32_t>(ent & 0xffffffffu);
+      atomicOr(&out[idx >> 5], 1u << (idx & 31));
+    }
+  }
+  res = make_int2(static_cast<int>(~static_cast<uint32_t>(last >> 32)), static_cast<int>(last & 0xffffffffu));
+  __syncthreads();
+  return true;
+}
+
 // One row per iteration of the block.  selbits [L*P][Nw]; rowparam [L*P] = (T, cutoff index).
-__global__ void __launch_bounds__(kRowThreads, 2)
-vote_rows_kernel(const float* __restrict__ logits, int rows, int N, float top_p,
+__global__ void __launch_bounds__(kRowThreads, kRowThreads >= 1024 ? 1 : 2)
+vote_rows_kernel(const float* __restrict__ logits, int rows, int N, float top_p, float R,
                  uint32_t* __restrict__ selbits, int2* __restrict__ rowparam) {
   extern __shared__ __align__(16) uint8_t vsm[];
-  double* hmass = reinterpret_cast<double*>(vsm);                          // [warps][256]
-  int* hcnt = reinterpret_cast<int*>(hmass + kRowWarps * kBins);           // [warps][256]
-  __shared__ float ftmp[kRowWarps];
-  __shared__ double dtmp[kRowWarps];
-  __shared__ double s_bin_mass[kBins];
-  __shared__ int s_bin_cnt[kBins];
-  __shared__ int s_sel, s_cnt;
-  __shared__ double s_above, s_target;
-  __shared__ int s_cut;
-  __shared__ int s_tie_base;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ RowShared sh;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int Nw = (N + 31) / 32;
   for (int row = blockIdx.x; row < rows; row += gridDim.x) {
     const float* x = logits + static_cast<size_t>(row) * N;
-    // ---- max
-    float m = -INFINITY;
-    for (int s = tid; s < N; s += kRowThreads) m = fmaxf(m, x[s]);
-    m = block_reduce(m, ftmp, [](float a, float b) { return fmaxf(a, b); });
-    // ---- radix select on the keys with mass histograms
-    uint32_t prefix = 0, hmask = 0;
-    double above = 0.0, target = 0.0;
-    int cnt_final = 0;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      for (int i = lane; i < kBins; i += 32) {
-        hmass[warp * kBins + i] = 0.0;
-        hcnt[warp * kBins + i] = 0;
-      }
-      __syncwarp();
-      for (int s = tid; s < N; s += kRowThreads) {
-        const float xv = x[s];
-        const uint32_t u = order_key(xv);
-        if ((u & hmask) == prefix) {
-          const int bin = (u >> shift) & (kBins - 1);
-          atomicAdd(&hcnt[warp * kBins + bin], 1);
-          atomicAdd(&hmass[warp * kBins + bin], static_cast<double>(__expf(xv - m)));
-        }
-      }
-      __syncthreads();
-      if (tid < kBins) {
-        double ms = 0.0;
-        int c = 0;
-        for (int w = 0; w < kRowWarps; ++w) {
-          ms += hmass[w * kBins + tid];
-          c += hcnt[w * kBins + tid];
-        }
-        s_bin_mass[tid] = ms;
-        s_bin_cnt[tid] = c;
-      }
-      __syncthreads();
-      if (warp == 0) {
-        // Lane j owns bins 255-8j .. 248-8j (descending).  The selected bin is the first,
-        // in descending order, at which base + cumulative mass reaches the target; if
-        // rounding keeps the total below the target (top_p close to 1), the lowest
-        // non-empty bin is taken (every entry above it is selected).
-        double loc = 0.0;
-        int nonempty = 0;
-        for (int i = 0; i < 8; ++i) {
-          const int b = kBins - 1 - (8 * lane + i);
-          loc += s_bin_mass[b];
-          nonempty |= s_bin_cnt[b] > 0;
-        }
-        double total = loc;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
-        double incl = loc;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const double t = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += t;
-        }
-        const double excl = incl - loc;
-        const double tgt = pass == 0 ? static_cast<double>(top_p) * total : s_target;
-        const double base = pass == 0 ? 0.0 : s_above;
-        const unsigned reach = __ballot_sync(0xffffffffu, nonempty && base + incl >= tgt);
-        const unsigned ne = __ballot_sync(0xffffffffu, nonempty);
-        const int owner = reach ? __ffs(reach) - 1 : 31 - __clz(ne ? ne : 1u);
-        if (lane == owner) {
-          double cum = base + excl;
-          int sel = -1;
-          for (int i = 0; i < 8; ++i) {
-            const int b = kBins - 1 - (8 * lane + i);
-            if (s_bin_cnt[b] == 0) continue;
-            if (reach && cum + s_bin_mass[b] >= tgt) { sel = b; break; }
-            sel = b;                       // no reach: ends at the lowest non-empty bin
-            if (!reach) { cum += s_bin_mass[b]; continue; }
-            cum += s_bin_mass[b];
-          }
-          if (!reach) cum -= s_bin_mass[sel];   // mass strictly above the selected bin
-          s_sel = sel;
-          s_above = cum;
-          s_cnt = s_bin_cnt[sel];
-          if (pass == 0) s_target = tgt;
-        }
-      }
-      __syncthreads();
-      prefix |= static_cast<uint32_t>(s_sel) << shift;
-      hmask |= 255u << shift;
-      above = s_above;
-      target = s_target;
-      cnt_final = s_cnt;
-      __syncthreads();
-    }
-    const uint32_t T = prefix;
-    // number of entries tied at T to select, in index order
-    const double eT = static_cast<double>(__expf(key_value(T) - m));
-    long long want = eT > 0.0 ? static_cast<long long>(ceil((target - above) / eT)) : cnt_final;
-    want = want < 1 ? 1 : (want > cnt_final ? cnt_final : want);
-    // cutoff index: the want-th tie in index order (all ties when want == cnt_final)
-    int cut = N;
-    if (want < cnt_final) {
-      if (tid == 0) { s_cut = N; s_tie_base = 0; }
-      __syncthreads();
-      for (int s0 = 0; s0 < N; s0 += kRowThreads) {
-        const int s = s0 + tid;
-        const bool tie = s < N && order_key(x[s]) == T;
-        const unsigned b = __ballot_sync(0xffffffffu, tie);
-        if (lane == 0) hcnt[warp] = __popc(b);
-        __syncthreads();
-        int before = s_tie_base;
-        for (int w = 0; w < warp; ++w) before += hcnt[w];
-        before += __popc(b & ((1u << lane) - 1));
-        if (tie && before + 1 == want) s_cut = s;
-        __syncthreads();
-        if (tid == 0) {
-          int tot = 0;
-          for (int w = 0; w < kRowWarps; ++w) tot += hcnt[w];
-          s_tie_base += tot;
-        }
-        __syncthreads();
-        if (s_cut < N) break;
-      }
-      cut = s_cut;
-      __syncthreads();
-    }
-    if (tid == 0) rowparam[row] = make_int2(static_cast<int>(T), cut);
-    // ---- selection bits of the row
+    const bool vec = (N % 4 == 0) && (reinterpret_cast<uintptr_t>(x) % 16 == 0);
     uint32_t* out = selbits + static_cast<size_t>(row) * Nw;
-    for (int s = tid; s < Nw * 32; s += kRowThreads) {
-      bool sel = false;
-      if (s < N) {
-        const uint32_t u = order_key(x[s]);
-        sel = u > T || (u == T && s <= cut);
+    int2 tc;
+    const bool ok = top_p < 1.f && window_nucleus(x, N, vec, top_p, R, vsm, sh, out, tc);
+    if (tid == 0 && ok) rowparam[row] = tc;
+    if (ok) continue;   // window_nucleus ends on a block barrier
+    float mv = -INFINITY;
+    for (int s = tid; s < N; s += kRowThreads) mv = fmaxf(mv, x[s]);
+    const float m = block_reduce(mv, sh.ftmp, [](float p, float q) { return fmaxf(p, q); });
+    tc = radix_nucleus(x, N, m, top_p, vsm, sh);
+    if (tid == 0) rowparam[row] = tc;
+    const uint32_t T = static_cast<uint32_t>(tc.x);
+    const int cut = tc.y;
+    // selection bits: lanes 8k .. 8k+7 hold the 32 entries of one word
+    const int Gr = (Nw * 8 + 31) & ~31;
+    for (int g0 = tid; g0 < Gr; g0 += 4 * kRowThreads) {
+      float4 v4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v4[u] = load4(x, 4 * (g0 + u * kRowThreads), N, vec);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int s = 4 * (g0 + u * kRowThreads);
+        const float xs[4] = {v4[u].x, v4[u].y, v4[u].z, v4[u].w};
+        uint32_t nib = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (s + j < N) {
+            const uint32_t k = order_key(xs[j]);
+            nib |= static_cast<uint32_t>(k > T || (k == T && s + j <= cut)) << j;
+          }
+        }
+        uint32_t word = nib << (4 * (lane & 7));
+        word |= __shfl_xor_sync(0xffffffffu, word, 1);
+        word |= __shfl_xor_sync(0xffffffffu, word, 2);
+        word |= __shfl_xor_sync(0xffffffffu, word, 4);
+        if ((lane & 7) == 0 && s < Nw * 32) out[s >> 5] = word;
       }
-      const unsigned bits = __ballot_sync(0xffffffffu, sel);
-      if (lane == 0) out[s >> 5] = bits;
     }
     __syncthreads();
   }
 }
 
-// Per (position, word): count over layers, golden bits (count >= theta), counts.
+// Per (position, word): the 32 entries' layer counts as a bit-sliced counter (plane k
+// holds bit k of every count), golden bits (count >= theta) and optional byte counts.
+template <int kPlanes>
 __global__ void vote_count_kernel(const uint32_t* __restrict__ selbits, int L, int P, int N, int theta,
                                   uint32_t* __restrict__ golden, uint8_t* __restrict__ counts) {
   const int Nw = (N + 31) / 32;
   const int p = blockIdx.y;
   const int w = blockIdx.x * blockDim.x + threadIdx.x;
   if (w >= Nw) return;
-  uint8_t cnt[32];
+  uint32_t pl[kPlanes];
 #pragma unroll
-  for (int b = 0; b < 32; ++b) cnt[b] = 0;
-  for (int l = 0; l < L; ++l) {
-    const uint32_t bits = selbits[(static_cast<size_t>(l) * P + p) * Nw + w];
+  for (int k = 0; k < kPlanes; ++k) pl[k] = 0u;
+  const uint32_t* src = selbits + static_cast<size_t>(p) * Nw + w;
+  const size_t stride = static_cast<size_t>(P) * Nw;
+  int l = 0;
+  for (; l + 4 <= L; l += 4) {
+    uint32_t b[4];
 #pragma unroll
-    for (int b = 0; b < 32; ++b) cnt[b] += (bits >> b) & 1u;
+    for (int u = 0; u < 4; ++u) b[u] = __ldg(src + (l + u) * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      uint32_t carry = b[u];
+#pragma unroll
+      for (int k = 0; k < kPlanes; ++k) {
+        const uint32_t t = pl[k] & carry;
+        pl[k] ^= carry;
+        carry = t;
+      }
+    }
   }
-  uint32_t g = 0;
+  for (; l < L; ++l) {
+    uint32_t carry = __ldg(src + l * stride);
 #pragma unroll
-  for (int b = 0; b < 32; ++b) g |= static_cast<uint32_t>(cnt[b] >= theta) << b;
-  if (w * 32 + 32 > N) g &= (N - w * 32 >= 32) ? 0xffffffffu : ((1u << (N - w * 32)) - 1u);
+    for (int k = 0; k < kPlanes; ++k) {
+      const uint32_t t = pl[k] & carry;
+      pl[k] ^= carry;
+      carry = t;
+    }
+  }
+  // count >= theta  <=>  no borrow out of count - theta (0 < theta < 2^kPlanes)
+  uint32_t g;
+  if (theta <= 0) {
+    g = 0xffffffffu;
+  } else if (theta >= (1 << kPlanes)) {
+    g = 0u;
+  } else {
+    uint32_t borrow = 0u;
+#pragma unroll
+    for (int k = 0; k < kPlanes; ++k)
+      borrow = ((theta >> k) & 1) ? (~pl[k] | borrow) : (~pl[k] & borrow);
+    g = ~borrow;
+  }
+  const int valid = N - w * 32;
+  if (valid < 32) g &= (1u << valid) - 1u;
   golden[static_cast<size_t>(p) * Nw + w] = g;
   if (counts) {
+    uint32_t packed[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint32_t v = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int bit = 4 * q + j;
+        uint32_t c = 0;
+#pragma unroll
+        for (int k = 0; k < kPlanes; ++k) c |= ((pl[k] >> bit) & 1u) << k;
+        v |= c << (8 * j);
+      }
+      packed[q] = v;
+    }
     uint8_t* c = counts + static_cast<size_t>(p) * N + static_cast<size_t>(w) * 32;
-    for (int b = 0; b < 32 && w * 32 + b < N; ++b) c[b] = cnt[b];
+    if (valid >= 32 && (reinterpret_cast<uintptr_t>(c) & 15) == 0) {
+      reinterpret_cast<uint4*>(c)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      reinterpret_cast<uint4*>(c)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+    } else {
+      for (int b = 0; b < 32 && b < valid; ++b) c[b] = static_cast<uint8_t>(packed[b >> 2] >> (8 * (b & 3)));
+    }
   }
 }
 
-// Sums of the BCE and focal terms over all P*N entries (fp64), then means.
+// Sums of the BCE and focal terms over all P*N entries, then means.  Per-entry terms
+// in fp32 (logf / log1pf, exact squares for gamma = 2), sums in fp64.
+__device__ __forceinline__ float focal_pow(float q, float gamma) {
+  return gamma == 2.f ? q * q : (gamma == 1.f ? q : (gamma == 0.f ? 1.f : powf(q, gamma)));
+}
+
 __global__ void vote_loss_kernel(const float* __restrict__ scores, const uint32_t* __restrict__ golden, int P,
                                  int N, float gamma, double* __restrict__ acc) {
   __shared__ double tmp[2][32];
   const int Nw = (N + 31) / 32;
-  const size_t total = static_cast<size_t>(P) * N;
-  const double eps = 1.0 / 1048576.0;   // 2^-20: probabilities clamped to [eps, 1 - eps]
+  const int p = blockIdx.y;
+  const float eps = 1.f / 1048576.f;   // 2^-20: probabilities clamped to [eps, 1 - eps]
+  const float* sc = scores + static_cast<size_t>(p) * N;
+  const uint32_t* gw = golden + static_cast<size_t>(p) * Nw;
   double bce = 0.0, fl = 0.0;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const size_t p = i / N, s = i - p * N;
-    const bool y = (golden[p * Nw + (s >> 5)] >> (s & 31)) & 1u;
-    double pr = static_cast<double>(scores[i]);
-    pr = pr < eps ? eps : (pr > 1.0 - eps ? 1.0 - eps : pr);
+  auto term = [&](float pr, bool y) {
+    pr = fminf(fmaxf(pr, eps), 1.f - eps);
     if (y) {
-      const double lp = log(pr);
-      bce -= lp;
-      fl -= pow(1.0 - pr, static_cast<double>(gamma)) * lp;
+      const float lp = logf(pr);
+      bce -= static_cast<double>(lp);
+      fl -= static_cast<double>(focal_pow(1.f - pr, gamma) * lp);
     } else {
-      const double lq = log1p(-pr);
-      bce -= lq;
-      fl -= pow(pr, static_cast<double>(gamma)) * lq;
+      const float lq = log1pf(-pr);
+      bce -= static_cast<double>(lq);
+      fl -= static_cast<double>(focal_pow(pr, gamma) * lq);
     }
+  };
+  const int stride = gridDim.x * blockDim.x;
+  if ((N & 3) == 0 && (reinterpret_cast<uintptr_t>(sc) & 15) == 0) {
+    const int G = N >> 2;
+    for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < G; g += stride) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(sc) + g);
+      const uint32_t bits = __ldg(gw + (g >> 3)) >> (4 * (g & 7));
+      term(v.x, bits & 1u);
+      term(v.y, (bits >> 1) & 1u);
+      term(v.z, (bits >> 2) & 1u);
+      term(v.w, (bits >> 3) & 1u);
+    }
+  } else {
+    for (int s = blockIdx.x * blockDim.x + threadIdx.x; s < N; s += stride)
+      term(__ldg(sc + s), (__ldg(gw + (s >> 5)) >> (s & 31)) & 1u);
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -281,24 +859,34 @@ int launch_vote(const VoteArgs& a, cudaStream_t st) {
   const int rows = a.L * a.P;
   const int Nw = (a.N + 31) / 32;
   int rc = LSA_OK;
-  if (rows > 0) {
-    const size_t smem = static_cast<size_t>(kRowWarps) * kBins * (sizeof(double) + sizeof(int));
-    cudaFuncSetAttribute(vote_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (rows > 0 && a.N > 0) {
+    const int smem = kRowSmem;
+    cudaFuncSetAttribute(vote_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int grid = std::min(rows, 2 * sms);
-    vote_rows_kernel<<<grid, kRowThreads, smem, st>>>(a.logits, rows, a.N, a.top_p, a.selbits,
+    int per_sm = 1;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, vote_rows_kernel, kRowThreads, smem);
+    per_sm = per_sm < 1 ? 1 : per_sm;
+    const int grid = std::min(rows, per_sm * sms);
+    // window half-width ln(N / (1 - top_p)) + 1 (unused when top_p = 1)
+    const float R = a.top_p < 1.f ? static_cast<float>(std::log(static_cast<double>(a.N) / (1.0 - a.top_p)) + 1.0)
+                                  : 0.f;
+    vote_rows_kernel<<<grid, kRowThreads, smem, st>>>(a.logits, rows, a.N, a.top_p, R, a.selbits,
                                                       reinterpret_cast<int2*>(a.rowparam));
     if ((rc = check_launch("vote_labels/rows")) != LSA_OK) return rc;
   }
-  vote_count_kernel<<<dim3((Nw + 255) / 256, a.P), 256, 0, st>>>(a.selbits, a.L, a.P, a.N, a.theta, a.golden,
-                                                                 a.counts);
+  const dim3 cgrid((Nw + 255) / 256, a.P);
+  if (a.L <= 31)
+    vote_count_kernel<5><<<cgrid, 256, 0, st>>>(a.selbits, a.L, a.P, a.N, a.theta, a.golden, a.counts);
+  else
+    vote_count_kernel<8><<<cgrid, 256, 0, st>>>(a.selbits, a.L, a.P, a.N, a.theta, a.golden, a.counts);
   if ((rc = check_launch("vote_labels/count")) != LSA_OK) return rc;
   if (a.scores) {
     cudaMemsetAsync(a.lossacc, 0, 2 * sizeof(double), st);
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    vote_loss_kernel<<<2 * sms, 256, 0, st>>>(a.scores, a.golden, a.P, a.N, a.gamma, a.lossacc);
+    const int per_row = std::max(1, std::min((a.N + 1023) / 1024, (4 * sms + a.P - 1) / a.P));
+    vote_loss_kernel<<<dim3(per_row, a.P), 256, 0, st>>>(a.scores, a.golden, a.P, a.N, a.gamma, a.lossacc);
     vote_loss_finalize<<<1, 1, 0, st>>>(a.lossacc, static_cast<double>(a.P) * a.N, a.loss);
     if ((rc = check_launch("vote_labels/loss", 2)) != LSA_OK) return rc;
   }

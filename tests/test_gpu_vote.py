@@ -94,6 +94,38 @@ def test_vote_top_p_range(top_p):
     check_vote(x, top_p, 2, gg, gc)
 
 
+@pytest.mark.parametrize("top_p", [0.1, 0.6, 0.95])
+def test_vote_full_length_rows(top_p):
+    """Rows of 2^17 logits: the candidate run spans from a few entries (top_p = 0.1) to a
+    few thousand (top_p = 0.95)."""
+    g = np.random.default_rng(int(top_p * 100))
+    x = g.standard_normal((3, 2, 2 ** 17)).astype(np.float32)
+    x[:, 1] *= 3.0
+    gg, gc, _ = run_vote(x, top_p, 2)
+    check_vote(x, top_p, 2, gg, gc)
+
+
+def test_vote_dense_ties_full_length():
+    """Logits on a 0.01 grid: hundreds of entries share the crossing value, so the
+    crossing is resolved by sorting the whole run."""
+    g = np.random.default_rng(5)
+    x = np.round(g.standard_normal((3, 2, 2 ** 17)), 2).astype(np.float32)
+    gg, gc, _ = run_vote(x, 0.6, 2)
+    check_vote(x, 0.6, 2, gg, gc)
+
+
+def test_vote_ragged_lengths_and_outliers():
+    """N not a multiple of 4 (scalar loads), a late maximum far above the first block of
+    logits (re-anchoring), and -inf entries."""
+    g = np.random.default_rng(9)
+    x = g.standard_normal((3, 2, 50001)).astype(np.float32)
+    x[0, 0, 45000] = 30.0
+    x[1, 1, 40000:40010] = 12.0
+    x[2, :, ::7] = -np.inf
+    gg, gc, _ = run_vote(x, 0.6, 1)
+    check_vote(x, 0.6, 1, gg, gc)
+
+
 def test_vote_all_equal_logits_exact_nucleus():
     N = 2 ** 17
     x = np.zeros((3, 2, N), dtype=np.float32)
