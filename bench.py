@@ -160,8 +160,10 @@ class Trigger:
         self.ws_score = lsa.workspace(lsa.lsa_index_score_workspace_bytes(B, L, N, w.D, w.r, w.H, w.dI,
                                                                           self.wdt, self.kdt), device)
         self.ws_topk = lsa.workspace(lsa.lsa_topk_workspace_bytes(B, N), device)
-        self.main = torch.cuda.Stream(device)
-        self.side = torch.cuda.Stream(device)
+        # The selection runs at a higher priority than the gathers beside it, so that the
+        # SMs a retiring gather block frees go to the selection first.
+        self.main = torch.cuda.Stream(device, priority=-1)
+        self.side = torch.cuda.Stream(device, priority=0)
         self.timing = []     # per step: [(score_start, score_end, gather_start, gather_end) per layer]
 
     def run(self, record=False):
@@ -172,7 +174,9 @@ class Trigger:
         lsa, w, inp = self.lsa, self.w, self.inp
         B, L, N = w.B, w.L, w.N
         m, sd = self.main, self.side
-        e = [torch.cuda.Event(enable_timing=record) for _ in range(2 + 2 * L)]
+        e = [torch.cuda.Event(enable_timing=record) for _ in range(4 + 2 * L)]
+        if record:
+            e[2 + 2 * L].record(m)
         lsa.lsa_index_project(B, L, w.D, w.r, w.H, w.dI, self.wdt, inp["h"], inp["Wd"], inp["Wu"], inp["Ww"], -1,
                               self.q, self.wv, self.ws_proj, stream=m)
         if record:
@@ -199,6 +203,8 @@ class Trigger:
         lsa.lsa_compact(B, N, self.U, N, self.idx_U, self.cnt_U, self.status, stream=m)
         lsa.lsa_topk(B, L, N, w.k, self.idx_U, N, self.cnt_U, self.logit, self.topk, self.topk_cnt, self.ws_topk,
                      stream=m)
+        if record:
+            e[3 + 2 * L].record(m)
         done = torch.cuda.Event()
         done.record(sd)
         m.wait_event(done)
@@ -206,11 +212,13 @@ class Trigger:
             self.timing.append(e)
 
     def kernel_times_ms(self):
-        """(score launch per step, gather launches per step) in ms."""
+        """Per step, in ms: the score launch; the gather launches; the main stream from
+        the projection through the top-k (the gathers run beside it on the side stream)."""
         L = self.w.L
         score = [e[0].elapsed_time(e[1]) for e in self.timing]
         gather = [sum(e[2 + 2 * l].elapsed_time(e[3 + 2 * l]) for l in range(L)) for e in self.timing]
-        return score, gather
+        select = [e[2 + 2 * L].elapsed_time(e[3 + 2 * L]) for e in self.timing]
+        return score, gather, select
 
 
 # ----------------------------------------------------------------------------- measurements
@@ -507,7 +515,8 @@ def our_arm(args):
         raise SystemExit(f"device status {status} ({lsa.status_string(status)}) during the timed region")
 
     units, ms, value = whole_job(w.B * w.L * w.N * args.steps, ms_local, dist, device)
-    score_ms, gather_ms = trig.kernel_times_ms()
+    score_ms, gather_ms, select_ms = trig.kernel_times_ms()
+    _, sel_ms, sel_value = whole_job(w.B * w.L * w.N * args.steps, sum(select_ms), dist, device)
     score_avg = statistics.mean(score_ms)
     gather_avg = statistics.mean(gather_ms)
     fetched_rows = int(trig.cnt_new.sum().item())          # rows moved by the last step
@@ -583,6 +592,9 @@ def our_arm(args):
                                 "bytes_per_step": fetched_rows * w.row_bytes, "rows_per_step": fetched_rows,
                                 "ms_per_step": gather_avg,
                                 "peak_kind": "measured here: pinned host->device cudaMemcpy, 1 GiB"},
+            "select_path": {"value": sel_value, "unit": UNIT, "ms_per_step": sel_ms / args.steps,
+                            "covers": "projection, scoring, union, compaction and top-k on the main stream of "
+                                      "each timed step, with that step's gathers running on the side stream"},
             "vote_labels": vote,
         }
         print(json.dumps(line), flush=True)

@@ -7,10 +7,14 @@
 // inside the fetched subset once it is in GPU memory).
 #include <algorithm>
 
+#include <cooperative_groups.h>
+
 #include "lsa_common.cuh"
 
 namespace lsa {
 namespace {
+
+namespace cg = cooperative_groups;
 
 // ------------------------------------------------------------------ union
 __global__ void union_kernel(size_t nwords, const uint32_t* __restrict__ m, uint32_t* __restrict__ U,
@@ -129,131 +133,169 @@ __device__ __forceinline__ uint32_t order_key(float x) {
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kKeysPerBlock = 2048;
+constexpr int kTopkSmemKeys = 49152;   // keys of one CTA's candidate slice held in shared memory
+constexpr int kSubHists = 16;          // digit sub-histograms, one per pair of warps
 
-// keys[b][j] = order_key(max over layers of logit[l][b][idx[b][j]]), j < min(count, cap).
-__global__ void __launch_bounds__(256)
-topk_keys_kernel(int B, int L, int N, const int32_t* __restrict__ idx, int cap, const int32_t* __restrict__ count,
-                 const float* __restrict__ logit, uint32_t* __restrict__ keys) {
-  const int b = blockIdx.y;
+struct TopkShared {
+  int sub[kSubHists][256];
+  int hist[2][256];   // this CTA's digit histogram by pass parity, read by the whole cluster
+  int tot[256];
+  int warp_tmp[32];
+  int total;
+  int cnt[2];         // this CTA's counts of keys above T and equal to T, read by the cluster
+  int gbase, ebase;
+  uint32_t prefix;
+  int kk;
+};
+
+// One thread-block cluster per sequence; CTA `rank` owns the contiguous candidate slice
+// [rank m, (rank + 1) m), m = ceil(n / cluster size).  Its keys
+//   key_j = order_key(max over layers of logit[l][b][idx[b][j]])
+// go to shared memory (to the key workspace when the slice exceeds kTopkSmemKeys).  Four
+// radix passes of 8 bits find the k-th largest key T and the number kk of keys equal to
+// T to keep; each pass adds the CTAs' digit histograms through distributed shared
+// memory.  The kept entries, all keys above T and the kk lowest-index ties, are written
+// in ascending candidate (= entry) order: each CTA's offsets come from the counts of the
+// CTAs before it, and inside a CTA from block scans over rounds of 4096 candidates.
+__global__ void __launch_bounds__(kTopkThreads, 1)
+topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx, int cap,
+                    const int32_t* __restrict__ count, const float* __restrict__ logit,
+                    uint32_t* __restrict__ keys_ws, int32_t* __restrict__ topk, int32_t* __restrict__ topk_count) {
+  extern __shared__ uint32_t skeys[];
+  __shared__ TopkShared sh;
+  cg::cluster_group cl = cg::this_cluster();
+  const int cs = static_cast<int>(cl.num_blocks());
+  const int rank = static_cast<int>(cl.block_rank());
+  const int b = blockIdx.x / cs;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = max(0, min(count[b], cap));
-  const int j0 = blockIdx.x * kKeysPerBlock;
-  if (j0 >= n) return;
   const int32_t* ib = idx + static_cast<size_t>(b) * cap;
-  uint32_t* kb = keys + static_cast<size_t>(b) * cap;
+  int32_t* ob = topk + static_cast<size_t>(b) * k;
+  if (n <= k) {                      // the same for every CTA of the cluster: no barrier follows
+    if (rank == 0) {
+      for (int j = tid; j < k; j += kTopkThreads) ob[j] = j < n ? ib[j] : -1;
+      if (tid == 0 && topk_count) topk_count[b] = n;
+    }
+    return;
+  }
+  const int m = (n + cs - 1) / cs;
+  const int j0 = min(n, rank * m), mloc = min(n, j0 + m) - j0;
+  uint32_t* kb = m <= kTopkSmemKeys ? skeys : keys_ws + static_cast<size_t>(b) * cap + j0;
 #pragma unroll 4
-  for (int j = j0 + threadIdx.x; j < min(n, j0 + kKeysPerBlock); j += blockDim.x) {
-    const int e = __ldg(ib + j);
+  for (int j = tid; j < mloc; j += kTopkThreads) {
+    const int e = __ldg(ib + j0 + j);
     float key = -INFINITY;
     if (e >= 0 && e < N)
       for (int l = 0; l < L; ++l) key = fmaxf(key, __ldg(logit + (static_cast<size_t>(l) * B + b) * N + e));
     kb[j] = order_key(key);
   }
-}
-
-// Four consecutive keys of candidates j .. j+3 (those at or past n read as 0, which no
-// selection counts: 0 is below every order_key of a float).
-__device__ __forceinline__ uint4 keys4(const uint32_t* kb, int j, int n, bool vec) {
-  if (vec && j + 3 < n) return __ldg(reinterpret_cast<const uint4*>(kb + j));
-  uint4 r;
-  r.x = j < n ? __ldg(kb + j) : 0u;
-  r.y = j + 1 < n ? __ldg(kb + j + 1) : 0u;
-  r.z = j + 2 < n ? __ldg(kb + j + 2) : 0u;
-  r.w = j + 3 < n ? __ldg(kb + j + 3) : 0u;
-  return r;
-}
-
-// One block per sequence: 4 radix passes of 8 bits for the k-th largest key T (count
-// of keys equal to T to keep: kk), then rounds of 4096 consecutive candidates (four per
-// thread) in which two block scans place every kept entry in ascending candidate
-// (= entry) order: all keys above T and the lowest-index ties.
-__global__ void __launch_bounds__(kTopkThreads)
-topk_select_kernel(int k, const int32_t* __restrict__ idx, int cap, const int32_t* __restrict__ count,
-                   const uint32_t* __restrict__ keys, int32_t* __restrict__ topk, int32_t* __restrict__ topk_count) {
-  __shared__ int sub[kTopkWarps][256];
-  __shared__ int hist[256];
-  __shared__ int warp_tmp[32];
-  __shared__ int total;
-  __shared__ uint32_t s_prefix;
-  __shared__ int s_kk;
-  const int b = blockIdx.x, tid = threadIdx.x, warp = tid >> 5;
-  const int n = max(0, min(count[b], cap));
-  const int32_t* ib = idx + static_cast<size_t>(b) * cap;
-  int32_t* ob = topk + static_cast<size_t>(b) * k;
-  if (n <= k) {
-    for (int j = tid; j < k; j += kTopkThreads) ob[j] = j < n ? ib[j] : -1;
-    if (tid == 0 && topk_count) topk_count[b] = n;
-    return;
-  }
-  const uint32_t* kb = keys + static_cast<size_t>(b) * cap;
-  const bool vec = (cap & 3) == 0;          // rows of the key array are 16-byte aligned
+  __syncthreads();
   uint32_t prefix = 0, himask = 0;
   int kk = k;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int i = tid; i < kTopkWarps * 256; i += kTopkThreads) (&sub[0][0])[i] = 0;
+    for (int i = tid; i < kSubHists * 256; i += kTopkThreads) (&sh.sub[0][0])[i] = 0;
     __syncthreads();
-#pragma unroll 2
-    for (int j = 4 * tid; j < n; j += 4 * kTopkThreads) {
-      const uint4 u4 = keys4(kb, j, n, vec);
-      const uint32_t u[4] = {u4.x, u4.y, u4.z, u4.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (j + e < n && (u[e] & himask) == prefix) atomicAdd(&sub[warp][(u[e] >> shift) & 255u], 1);
+    for (int j = tid; j < mloc; j += kTopkThreads) {
+      const uint32_t u = kb[j];
+      if ((u & himask) == prefix) atomicAdd(&sh.sub[warp >> 1][(u >> shift) & 255u], 1);
     }
     __syncthreads();
     if (tid < 256) {
       int h = 0;
-      for (int w = 0; w < kTopkWarps; ++w) h += sub[w][tid];
-      hist[tid] = h;
+#pragma unroll
+      for (int w = 0; w < kSubHists; ++w) h += sh.sub[w][tid];
+      sh.hist[pass & 1][tid] = h;
+    }
+    // After this barrier every CTA's histogram of the pass is complete.  A CTA rewrites
+    // hist[pass & 1] two passes later, after the next barrier, which no CTA passes
+    // before it has finished reading this pass's histograms.
+    cl.sync();
+    if (tid < 256) {
+      int t = 0;
+      for (int r = 0; r < cs; ++r) t += cl.map_shared_rank(&sh.hist[pass & 1][0], r)[tid];
+      sh.tot[tid] = t;
     }
     __syncthreads();
     if (tid == 0) {
       int cum = 0, sel = 0;
       for (int d = 255; d >= 0; --d) {
-        if (cum + hist[d] >= kk) { sel = d; break; }
-        cum += hist[d];
+        if (cum + sh.tot[d] >= kk) { sel = d; break; }
+        cum += sh.tot[d];
       }
-      s_kk = kk - cum;
-      s_prefix = prefix | (static_cast<uint32_t>(sel) << shift);
+      sh.kk = kk - cum;
+      sh.prefix = prefix | (static_cast<uint32_t>(sel) << shift);
     }
     __syncthreads();
-    kk = s_kk;
-    prefix = s_prefix;
+    kk = sh.kk;
+    prefix = sh.prefix;
     himask |= 255u << shift;
-    __syncthreads();
   }
   const uint32_t T = prefix;
-  int gt_base = 0, eq_base = 0;
-  for (int r0 = 0; r0 < n; r0 += 4 * kTopkThreads) {
+  {
+    int gt = 0, eq = 0;
+    for (int j = tid; j < mloc; j += kTopkThreads) {
+      const uint32_t u = kb[j];
+      gt += u > T;
+      eq += u == T;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      gt += __shfl_xor_sync(0xffffffffu, gt, o);
+      eq += __shfl_xor_sync(0xffffffffu, eq, o);
+    }
+    if (lane == 0) { sh.sub[0][warp] = gt; sh.sub[1][warp] = eq; }
+    __syncthreads();
+    if (tid == 0) {
+      int g = 0, q = 0;
+      for (int w = 0; w < kTopkWarps; ++w) { g += sh.sub[0][w]; q += sh.sub[1][w]; }
+      sh.cnt[0] = g;
+      sh.cnt[1] = q;
+    }
+    cl.sync();
+    if (tid == 0) {
+      int g = 0, q = 0;
+      for (int r = 0; r < rank; ++r) {
+        const int* rc = cl.map_shared_rank(&sh.cnt[0], r);
+        g += rc[0];
+        q += rc[1];
+      }
+      sh.gbase = g;
+      sh.ebase = q;
+    }
+    cl.sync();   // no CTA leaves while another may still read its shared memory
+  }
+  int gt_base = sh.gbase, eq_base = sh.ebase;
+  for (int r0 = 0; r0 < mloc; r0 += 4 * kTopkThreads) {
     const int j = r0 + 4 * tid;
-    const uint4 u4 = keys4(kb, j, n, vec);
-    const uint32_t u[4] = {u4.x, u4.y, u4.z, u4.w};
+    uint32_t u[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) u[e] = j + e < mloc ? kb[j + e] : 0u;
     int gt = 0, eq = 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      gt += j + e < n && u[e] > T;
-      eq += j + e < n && u[e] == T;
+      gt += j + e < mloc && u[e] > T;
+      eq += j + e < mloc && u[e] == T;
     }
-    int gt_before = gt_base + block_exclusive_scan(gt, warp_tmp, &total);
-    const int gt_round = total;
-    int eq_before = eq_base + block_exclusive_scan(eq, warp_tmp, &total);
-    const int eq_round = total;
+    int gt_before = gt_base + block_exclusive_scan(gt, sh.warp_tmp, &sh.total);
+    const int gt_round = sh.total;
+    int eq_before = eq_base + block_exclusive_scan(eq, sh.warp_tmp, &sh.total);
+    const int eq_round = sh.total;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      if (j + e >= n) break;
+      if (j + e >= mloc) break;
       if (u[e] > T) {
-        ob[gt_before + min(eq_before, kk)] = __ldg(ib + j + e);
+        ob[gt_before + min(eq_before, kk)] = __ldg(ib + j0 + j + e);
         ++gt_before;
       } else if (u[e] == T) {
-        if (eq_before < kk) ob[gt_before + eq_before] = __ldg(ib + j + e);
+        if (eq_before < kk) ob[gt_before + eq_before] = __ldg(ib + j0 + j + e);
         ++eq_before;
       }
     }
     gt_base += gt_round;
     eq_base += eq_round;
   }
-  if (tid == 0 && topk_count) topk_count[b] = k;
+  if (rank == 0 && tid == 0 && topk_count) topk_count[b] = k;
 }
 
 }  // namespace
@@ -279,12 +321,33 @@ int launch_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const i
                 const float* logit, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws,
                 cudaStream_t s) {
   if (B == 0) return LSA_OK;
-  if (cap > 0) {
-    const dim3 g1((cap + kKeysPerBlock - 1) / kKeysPerBlock, B);
-    topk_keys_kernel<<<g1, 256, 0, s>>>(B, L, N, idx, cap, count, logit, keys_ws);
+  const int smem = kTopkSmemKeys * 4;
+  cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // CTAs per sequence: as many as keep B x cs within one wave, at most 8 (portable)
+  int cs = 8;
+  while (cs > 1 && B * cs > sms) cs >>= 1;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  cfg.blockDim = dim3(kTopkThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  for (;; cs >>= 1) {
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(B * cs);
+    if (cs == 1) break;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, topk_cluster_kernel, &cfg) == cudaSuccess && clusters > 0) break;
+    cudaGetLastError();
   }
-  topk_select_kernel<<<B, kTopkThreads, 0, s>>>(k, idx, cap, count, keys_ws, topk, topk_count);
-  return check_launch("topk", cap > 0 ? 2 : 1);
+  cudaLaunchKernelEx(&cfg, topk_cluster_kernel, B, L, N, k, idx, cap, count, logit, keys_ws, topk, topk_count);
+  return check_launch("topk");
 }
 
 }  // namespace lsa

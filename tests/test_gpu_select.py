@@ -108,6 +108,38 @@ def test_topk_exact_with_ties(k):
         assert np.all(topk[b, len(e): k] == -1)
 
 
+def check_topk(idx_list, logits, k, topk, tc):
+    for b in range(len(idx_list)):
+        key = logits[:, b, :].astype(np.float64).max(axis=0)
+        e = O.topk_in_fetched(idx_list[b], key, k)
+        assert tc[b] == len(e)
+        assert np.array_equal(topk[b, : len(e)], e), b
+        assert np.all(topk[b, len(e): k] == -1)
+
+
+def test_topk_many_sequences_keys_beyond_shared_memory():
+    """150 sequences (one CTA each on a 148-SM part); 60,000 candidates exceed one CTA's
+    shared-memory key slice, so those keys live in the workspace."""
+    g = np.random.default_rng(21)
+    L, B, N, k = 2, 150, 60000, 2048
+    logits = np.round(g.standard_normal((L, B, N)) * 3, 1).astype(np.float32)   # ties at the k-th key
+    sizes = [N if b % 3 == 0 else (50000 if b % 3 == 1 else int(g.integers(0, 5000))) for b in range(B)]
+    idx_list = [np.arange(N) if n == N else np.sort(g.choice(N, size=n, replace=False)) for n in sizes]
+    topk, tc = run_topk(idx_list, logits, k, N)
+    check_topk(idx_list, logits, k, topk, tc)
+
+
+def test_topk_long_sequences_cluster_slices():
+    """Two sequences split over a cluster of CTAs: 300,000 candidates (keys in shared
+    memory) and 450,000 (slices beyond shared memory)."""
+    g = np.random.default_rng(22)
+    L, B, N, k = 3, 2, 500000, 2048
+    logits = np.round(g.standard_normal((L, B, N)) * 4, 2).astype(np.float32)
+    idx_list = [np.sort(g.choice(N, size=300000, replace=False)), np.sort(g.choice(N, size=450000, replace=False))]
+    topk, tc = run_topk(idx_list, logits, k, N)
+    check_topk(idx_list, logits, k, topk, tc)
+
+
 def test_topk_negative_keys_and_all_equal():
     L, B, N = 1, 2, 3000
     logits = np.full((L, B, N), -2.5, dtype=np.float32)
@@ -144,6 +176,31 @@ def test_gather_bytes_exact_and_range_status():
     lsa.lsa_gather_cold(B, N, R, cold, idx, cnt, cap, hot, st)
     torch.cuda.synchronize()
     assert int(st) == lsa.LSA_ERR_RANGE
+
+
+def test_gather_many_unbalanced_sequences():
+    """70 sequences with fetch counts from 0 to the whole pool (rows of 64 bytes): the
+    blocks share one flat range of rows, including empty and capped sequences."""
+    g = np.random.default_rng(3)
+    B, N, R = 70, 3000, 64
+    cold = torch.from_numpy(g.integers(0, 256, size=(B, N, R), dtype=np.uint8)).pin_memory()
+    sizes = [0 if b % 7 == 0 else (N if b % 11 == 0 else int(g.integers(1, 400))) for b in range(B)]
+    lists = [np.sort(g.choice(N, size=n, replace=False)) for n in sizes]
+    cap = N
+    idx = torch.zeros(B, cap, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(B, dtype=torch.int32, device="cuda")
+    for b, x in enumerate(lists):
+        idx[b, : len(x)] = torch.from_numpy(x.astype(np.int32))
+        cnt[b] = len(x)
+    hot = torch.zeros(B, cap, R, dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lsa.lsa_gather_cold(B, N, R, cold, idx, cnt, cap, hot, st)
+    torch.cuda.synchronize()
+    assert int(st) == 0
+    hc = hot.cpu().numpy()
+    for b, x in enumerate(lists):
+        assert np.array_equal(hc[b, : len(x)], O.gather_rows(cold[b].numpy(), x)), b
+        assert not hc[b, len(x):].any()
 
 
 def test_gather_rejects_pageable_memory():
