@@ -204,6 +204,69 @@ def gather_rows(cold, idx) -> np.ndarray:
     return np.asarray(cold)[np.asarray(idx, dtype=np.int64)]
 
 
+# ----------------------------------------------------------------------------- hot pool
+
+
+class HotPool:
+    """Residency of fetched rows across triggers, for one sequence.
+
+    [SUMMARY] §2.1 and [REVIEW] 二: the indexer runs every tau decode steps and keeps
+    only the KV blocks it predicts as needed in GPU memory, fetching them from the CPU
+    cold pool.  The pages do not say what happens to rows fetched by an earlier trigger;
+    the reading taken here: a row stays in its hot-pool slot until its slot is needed
+    for a row the current trigger wants and the pool has no free slot, so only rows
+    not yet resident cross the host link.
+
+    State: slot_of[e] (-1 if entry e is not resident), entry_of[s] (-1 if slot s is
+    free), stamp[s] (the last trigger whose fetch set contained slot s's entry; 0 for
+    a slot never used).  One update with fetch set U at trigger t >= 1:
+      1. every resident entry of U gets stamp t (its slot is kept);
+      2. need = entries of U not resident, ascending;
+      3. if |U| > slots the update fails (nothing moves, stamps of step 1 stay);
+      4. the candidate slots are those not kept, in order of (stamp, slot): free slots
+         first, then the least recently needed; the first |need| of them are taken;
+      5. the i-th entry of need goes to the i-th taken slot in ascending slot order,
+         evicting the entry that slot held; its row is copied from the cold pool.
+    """
+
+    def __init__(self, N: int, slots: int):
+        self.N, self.slots = N, slots
+        self.slot_of = [-1] * N
+        self.entry_of = [-1] * slots
+        self.stamp = [0] * slots
+
+    def update(self, U, t: int, cold=None, hot=None):
+        """U: iterable of entry indices (the trigger's fetch set).  Returns the list of
+        (entry, slot) moves in entry order, or None when |U| exceeds the pool."""
+        assert t >= 1
+        U = sorted(set(int(e) for e in U))
+        inU = set(U)
+        kept = set()
+        for e in U:
+            s = self.slot_of[e]
+            if s >= 0:
+                self.stamp[s] = t
+                kept.add(s)
+        need = [e for e in U if self.slot_of[e] < 0]
+        if len(U) > self.slots:
+            return None
+        cand = sorted((self.stamp[s], s) for s in range(self.slots) if s not in kept)
+        taken = sorted(s for _, s in cand[: len(need)])
+        moves = []
+        for e, s in zip(need, taken):
+            old = self.entry_of[s]
+            assert old < 0 or old not in inU
+            if old >= 0:
+                self.slot_of[old] = -1
+            self.entry_of[s] = e
+            self.slot_of[e] = s
+            self.stamp[s] = t
+            if cold is not None:
+                hot[s] = cold[e]
+            moves.append((e, s))
+        return moves
+
+
 # ----------------------------------------------------------------------------- labels
 
 
