@@ -220,6 +220,45 @@ int lsa_gather_cold(int B, int N, size_t row_bytes, const void* cold_host,
                     int32_t* status, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * Hot-pool residency across triggers ([SUMMARY] §2.1 and [REVIEW] 二: every tau decode
+ * steps the indexer predicts which compressed KV blocks will be needed, and only those
+ * are kept in GPU memory, fetched from the CPU cold pool).  The pages do not say what
+ * becomes of a row fetched by an earlier trigger; here it stays in its slot until a
+ * later trigger needs the slot, so only rows not yet resident cross the host link.
+ *
+ * State (device, caller-allocated, lsa_hot_pool_state_bytes; 256-byte aligned), four
+ * arrays at the offsets lsa_hot_pool_layout returns:
+ *   slot_of  [B][N] int32      slot holding entry e, or -1
+ *   entry_of [B][slots] int32  entry held by slot s, or -1 (free)
+ *   stamp    [B][slots] uint32 last trigger whose fetch set held the slot's entry (0: never)
+ *   resident [B][ceil(N/32)] uint32 bits, bit e set iff slot_of[e] >= 0
+ * lsa_hot_pool_reset empties the pool (no kernel: four memsets on the stream).
+ *
+ * lsa_hot_pool_update, for trigger index `trigger` (>= 1, increasing across calls) and
+ * fetch set U [B][ceil(N/32)] (bits past N ignored), per sequence b:
+ *   1. resident entries of U keep their slots; their stamp becomes `trigger`;
+ *   2. if |U| > slots nothing moves and *status is raised to LSA_ERR_CAPACITY;
+ *   3. else the missing entries of U (ascending) take the free or least recently
+ *      needed slots: slots not kept, ordered by (stamp, slot index), the first as many
+ *      as needed, paired in ascending slot order; each evicts the entry it held;
+ *   4. hot[b][slot][0..row_bytes) = cold[b][entry][0..row_bytes) for each move.
+ *   moved [B] (device, or NULL): rows moved per sequence.
+ *   cold  HOST pointer [B][N][row_bytes], page-locked and mapped (as lsa_gather_cold);
+ *   hot   device [B][slots][row_bytes]; slots >= 1; row_bytes a positive multiple of 16.
+ *   workspace: lsa_hot_pool_workspace_bytes(B, N, slots) bytes, 256-byte aligned.
+ * Six launches; asynchronous on `stream`; calls on one state must not overlap.
+ * ---------------------------------------------------------------------------------- */
+size_t lsa_hot_pool_state_bytes(int B, int N, int slots);
+size_t lsa_hot_pool_workspace_bytes(int B, int N, int slots);
+/* offsets[0..3] = byte offsets of slot_of, entry_of, stamp, resident in the state */
+int lsa_hot_pool_layout(int B, int N, int slots, size_t offsets[4]);
+int lsa_hot_pool_reset(int B, int N, int slots, void* state, void* stream);
+int lsa_hot_pool_update(int B, int N, int slots, size_t row_bytes, uint32_t trigger,
+                        const uint32_t* U, const void* cold_host, void* hot, void* state,
+                        int32_t* moved, int32_t* status,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * lsa_vote_labels -- cross-layer majority-vote golden labels and their loss
  * ([SUMMARY] §2.2: softmax over the indexer logits, per-layer nucleus top-p, an entry
  * is golden when at least theta of the L layers select it; §2.3 / [REVIEW] 二: BCE

@@ -9,6 +9,8 @@ raises LsaError.  Shapes and layouts are documented in include/lsa.h.
 """
 from __future__ import annotations
 
+import ctypes
+
 import torch
 
 from . import _abi
@@ -135,6 +137,35 @@ def lsa_topk_noalloc(B, L, N, k, idx, cap, count, logit, topk, topk_count, strea
 def lsa_gather_cold(B, N, row_bytes, cold_host, idx, count, cap, hot, status=None, stream=None):
     _check(lib().lsa_gather_cold(B, N, row_bytes, _p(cold_host), _p(idx), _p(count), cap, _p(hot),
                                  _p(status), _stream(stream)), "lsa_gather_cold")
+
+
+# ----------------------------------------------------------------------------- hot pool
+
+def lsa_hot_pool_state_bytes(B, N, slots) -> int:
+    return int(lib().lsa_hot_pool_state_bytes(B, N, slots))
+
+
+def lsa_hot_pool_workspace_bytes(B, N, slots) -> int:
+    return int(lib().lsa_hot_pool_workspace_bytes(B, N, slots))
+
+
+def lsa_hot_pool_layout(B, N, slots):
+    """Byte offsets of (slot_of, entry_of, stamp, resident) inside the state."""
+    off = (ctypes.c_size_t * 4)()
+    _check(lib().lsa_hot_pool_layout(B, N, slots, off), "lsa_hot_pool_layout")
+    return tuple(int(x) for x in off)
+
+
+def lsa_hot_pool_reset(B, N, slots, state, stream=None):
+    _check(lib().lsa_hot_pool_reset(B, N, slots, _p(state), _stream(stream)), "lsa_hot_pool_reset")
+
+
+def lsa_hot_pool_update(B, N, slots, row_bytes, trigger, U, cold_host, hot, state, moved, status,
+                        workspace, stream=None):
+    _check(lib().lsa_hot_pool_update(B, N, slots, row_bytes, trigger, _p(U), _p(cold_host), _p(hot), _p(state),
+                                     _p(moved), _p(status), _p(workspace),
+                                     0 if workspace is None else workspace.numel(), _stream(stream)),
+           "lsa_hot_pool_update")
 
 
 # ----------------------------------------------------------------------------- labels

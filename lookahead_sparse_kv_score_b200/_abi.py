@@ -34,6 +34,12 @@ SIGNATURES = {
                                  c_void_p, c_void_p]),
     "lsa_gather_cold": (c_int, [c_int, c_int, c_size_t, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
                                 c_void_p, c_void_p]),
+    "lsa_hot_pool_state_bytes": (c_size_t, [c_int, c_int, c_int]),
+    "lsa_hot_pool_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
+    "lsa_hot_pool_layout": (c_int, [c_int, c_int, c_int, ctypes.POINTER(c_size_t)]),
+    "lsa_hot_pool_reset": (c_int, [c_int, c_int, c_int, c_void_p, c_void_p]),
+    "lsa_hot_pool_update": (c_int, [c_int, c_int, c_int, c_size_t, ctypes.c_uint32, c_void_p, c_void_p, c_void_p,
+                                    c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "lsa_vote_labels_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
     "lsa_vote_labels": (c_int, [c_int, c_int, c_int, c_void_p, c_float, c_int, c_void_p, c_void_p,
                                 c_void_p, c_float, c_void_p, c_void_p, c_size_t, c_void_p]),

@@ -272,6 +272,77 @@ int lsa_gather_cold(int B, int N, size_t row_bytes, const void* cold_host,
                        static_cast<cudaStream_t>(stream));
 }
 
+static int hot_sizes_ok(int B, int N, int slots) { return B >= 0 && N >= 0 && slots >= 0; }
+
+size_t lsa_hot_pool_state_bytes(int B, int N, int slots) {
+  return hot_sizes_ok(B, N, slots) ? hot_layout(B, N, slots).state_bytes : 0;
+}
+
+size_t lsa_hot_pool_workspace_bytes(int B, int N, int slots) {
+  return hot_sizes_ok(B, N, slots) ? hot_layout(B, N, slots).ws_bytes : 0;
+}
+
+int lsa_hot_pool_layout(int B, int N, int slots, size_t offsets[4]) {
+  g_err[0] = 0;
+  if (!hot_sizes_ok(B, N, slots)) return fail(LSA_ERR_INVALID_ARG, "hot_pool_layout: negative size");
+  if (!offsets) return fail(LSA_ERR_INVALID_ARG, "hot_pool_layout: null pointer");
+  const HotLayout l = hot_layout(B, N, slots);
+  offsets[0] = l.slot_of;
+  offsets[1] = l.entry_of;
+  offsets[2] = l.stamp;
+  offsets[3] = l.resident;
+  return LSA_OK;
+}
+
+int lsa_hot_pool_reset(int B, int N, int slots, void* state, void* stream) {
+  g_err[0] = 0;
+  if (!hot_sizes_ok(B, N, slots)) return fail(LSA_ERR_INVALID_ARG, "hot_pool_reset: negative size");
+  if (!state) return fail(LSA_ERR_INVALID_ARG, "hot_pool_reset: null pointer");
+  if (!aligned(state, 256)) return fail(LSA_ERR_INVALID_ARG, "hot_pool_reset: state must be 256-byte aligned");
+  const HotLayout l = hot_layout(B, N, slots);
+  uint8_t* st = static_cast<uint8_t*>(state);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t Nw = (static_cast<size_t>(N) + 31) / 32;
+  if (cudaMemsetAsync(st + l.slot_of, 0xff, static_cast<size_t>(B) * N * 4, s) != cudaSuccess ||
+      cudaMemsetAsync(st + l.entry_of, 0xff, static_cast<size_t>(B) * slots * 4, s) != cudaSuccess ||
+      cudaMemsetAsync(st + l.stamp, 0, static_cast<size_t>(B) * slots * 4, s) != cudaSuccess ||
+      cudaMemsetAsync(st + l.resident, 0, static_cast<size_t>(B) * Nw * 4, s) != cudaSuccess) {
+    const cudaError_t e = cudaGetLastError();
+    return fail(LSA_ERR_CUDA, "hot_pool_reset: %s", cudaGetErrorString(e));
+  }
+  return LSA_OK;
+}
+
+int lsa_hot_pool_update(int B, int N, int slots, size_t row_bytes, uint32_t trigger,
+                        const uint32_t* U, const void* cold_host, void* hot, void* state,
+                        int32_t* moved, int32_t* status,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  if (!hot_sizes_ok(B, N, slots)) return fail(LSA_ERR_INVALID_ARG, "hot_pool_update: negative size");
+  if (row_bytes == 0 || row_bytes % 16 != 0)
+    return fail(LSA_ERR_INVALID_ARG, "hot_pool_update: row_bytes %zu is not a positive multiple of 16", row_bytes);
+  if (trigger == 0 || trigger == 0xffffffffu)
+    return fail(LSA_ERR_INVALID_ARG, "hot_pool_update: trigger must be in [1, 2^32 - 2]");
+  if (slots < 1) return fail(LSA_ERR_INVALID_ARG, "hot_pool_update: slots must be >= 1");
+  if (B == 0 || N == 0) return LSA_OK;
+  if (!U || !cold_host || !state || !hot)
+    return fail(LSA_ERR_INVALID_ARG, "hot_pool_update: null pointer");
+  if (!aligned(state, 256) || !aligned(U, 16) || !aligned(cold_host, 16) || (hot && !aligned(hot, 16)))
+    return fail(LSA_ERR_INVALID_ARG, "hot_pool_update: misaligned pointer (state 256 B, others 16 B)");
+  const HotLayout l = hot_layout(B, N, slots);
+  if (!workspace || workspace_bytes < l.ws_bytes || !aligned(workspace, 256))
+    return fail(LSA_ERR_NOMEM, "hot_pool_update: workspace %zu bytes (need %zu, 256-byte aligned)", workspace_bytes,
+                l.ws_bytes);
+  cudaPointerAttributes attr{};
+  if (cudaPointerGetAttributes(&attr, cold_host) != cudaSuccess || attr.type != cudaMemoryTypeHost ||
+      attr.devicePointer == nullptr) {
+    cudaGetLastError();
+    return fail(LSA_ERR_INVALID_ARG, "hot_pool_update: cold pool is not page-locked, mapped host memory");
+  }
+  return launch_hot_update(B, N, slots, row_bytes, trigger, U, attr.devicePointer, hot, state, moved, status,
+                           workspace, static_cast<cudaStream_t>(stream));
+}
+
 size_t lsa_vote_labels_workspace_bytes(int L, int P, int N) {
   if (L < 0 || P < 0 || N < 0) return 0;
   const size_t Nw = (static_cast<size_t>(N) + 31) / 32;

@@ -92,6 +92,22 @@ int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, in
 int launch_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
                 const float* logit, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws,
                 cudaStream_t s);
+// Direct-key selection: per sequence b, the kdev[b] largest of keys[b][0..n) (ties to the
+// lower index) in ascending index order, or none with LSA_ERR_CAPACITY when kdev[b]
+// exceeds n - kept[b].  out [B][n], out_count [B].
+int launch_select_keys(int B, int n, const uint32_t* keys, const int32_t* kdev, const int32_t* kept,
+                       int32_t* status, int32_t* out, int32_t* out_count, uint32_t* keys_ws, cudaStream_t s);
+
+// Hot-pool residency: byte offsets of the state arrays and of the update's workspace.
+struct HotLayout {
+  size_t slot_of, entry_of, stamp, resident, state_bytes;
+  size_t need_bits, keys, need, need_count, kept_count, taken, moved, select_ws, ws_bytes;
+};
+HotLayout hot_layout(int B, int N, int slots);
+int launch_hot_update(int B, int N, int slots, size_t row_bytes, uint32_t t, const uint32_t* U,
+                      const void* cold_dev, void* hot, void* state, int32_t* moved, int32_t* status,
+                      void* ws, cudaStream_t s);
+
 int launch_gather(int B, int N, size_t row_bytes, const void* cold_dev, const int32_t* idx,
                   const int32_t* count, int cap, void* hot, int32_t* status, cudaStream_t s);
 

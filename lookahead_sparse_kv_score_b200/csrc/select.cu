@@ -148,10 +148,15 @@ struct TopkShared {
   int kk;
 };
 
+// Candidates and keys come in one of two ways.  Fetched-set mode: candidate j is entry
+// idx[b][j] (j < count[b]) with key order_key(max over layers of logit[l][b][entry]),
+// and k is the same for every sequence.  Direct mode (dkeys != nullptr): candidate j is
+// j itself for j < cap, its key is dkeys[b][j], and sequence b keeps kdev[b] of them,
+// or none (raising LSA_ERR_CAPACITY) when kdev[b] exceeds cap - kept[b]; the output row
+// stride is then cap.
+//
 // One thread-block cluster per sequence; CTA `rank` owns the contiguous candidate slice
-// [rank m, (rank + 1) m), m = ceil(n / cluster size).  Its keys
-//   key_j = order_key(max over layers of logit[l][b][idx[b][j]])
-// go to shared memory (to the key workspace when the slice exceeds kTopkSmemKeys).  Four
+// [rank m, (rank + 1) m), m = ceil(n / cluster size).  Its keys go to shared memory (to the key workspace when the slice exceeds kTopkSmemKeys).  Four
 // radix passes of 8 bits find the k-th largest key T and the number kk of keys equal to
 // T to keep; each pass adds the CTAs' digit histograms through distributed shared
 // memory.  The kept entries, all keys above T and the kk lowest-index ties, are written
@@ -160,6 +165,8 @@ struct TopkShared {
 __global__ void __launch_bounds__(kTopkThreads, 1)
 topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx, int cap,
                     const int32_t* __restrict__ count, const float* __restrict__ logit,
+                    const uint32_t* __restrict__ dkeys, const int32_t* __restrict__ kdev,
+                    const int32_t* __restrict__ kept, int32_t* status,
                     uint32_t* __restrict__ keys_ws, int32_t* __restrict__ topk, int32_t* __restrict__ topk_count) {
   extern __shared__ uint32_t skeys[];
   __shared__ TopkShared sh;
@@ -168,36 +175,53 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
   const int rank = static_cast<int>(cl.block_rank());
   const int b = blockIdx.x / cs;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int n = max(0, min(count[b], cap));
-  const int32_t* ib = idx + static_cast<size_t>(b) * cap;
-  int32_t* ob = topk + static_cast<size_t>(b) * k;
-  if (n <= k) {                      // the same for every CTA of the cluster: no barrier follows
+  const bool direct = dkeys != nullptr;
+  int n, kb;                         // candidates and keys to keep for this sequence
+  if (direct) {
+    n = cap;
+    kb = max(0, kdev[b]);
+    if (kb > cap - kept[b]) {
+      if (rank == 0 && tid == 0) raise_status(status, LSA_ERR_CAPACITY);
+      kb = 0;
+    }
+  } else {
+    n = max(0, min(count[b], cap));
+    kb = k;
+  }
+  const int32_t* ib = direct ? nullptr : idx + static_cast<size_t>(b) * cap;
+  int32_t* ob = topk + static_cast<size_t>(b) * (direct ? cap : k);
+  if (n <= kb || kb == 0) {          // the same for every CTA of the cluster: no barrier follows
     if (rank == 0) {
-      for (int j = tid; j < k; j += kTopkThreads) ob[j] = j < n ? ib[j] : -1;
-      if (tid == 0 && topk_count) topk_count[b] = n;
+      const int m = min(n, kb);
+      for (int j = tid; j < (direct ? m : k); j += kTopkThreads) ob[j] = j < m ? (direct ? j : ib[j]) : -1;
+      if (tid == 0 && topk_count) topk_count[b] = m;
     }
     return;
   }
   const int m = (n + cs - 1) / cs;
   const int j0 = min(n, rank * m), mloc = min(n, j0 + m) - j0;
-  uint32_t* kb = m <= kTopkSmemKeys ? skeys : keys_ws + static_cast<size_t>(b) * cap + j0;
+  uint32_t* key = m <= kTopkSmemKeys ? skeys : keys_ws + static_cast<size_t>(b) * cap + j0;
+  if (direct) {
+    for (int j = tid; j < mloc; j += kTopkThreads) key[j] = __ldg(dkeys + static_cast<size_t>(b) * cap + j0 + j);
+  } else {
 #pragma unroll 4
-  for (int j = tid; j < mloc; j += kTopkThreads) {
-    const int e = __ldg(ib + j0 + j);
-    float key = -INFINITY;
-    if (e >= 0 && e < N)
-      for (int l = 0; l < L; ++l) key = fmaxf(key, __ldg(logit + (static_cast<size_t>(l) * B + b) * N + e));
-    kb[j] = order_key(key);
+    for (int j = tid; j < mloc; j += kTopkThreads) {
+      const int e = __ldg(ib + j0 + j);
+      float z = -INFINITY;
+      if (e >= 0 && e < N)
+        for (int l = 0; l < L; ++l) z = fmaxf(z, __ldg(logit + (static_cast<size_t>(l) * B + b) * N + e));
+      key[j] = order_key(z);
+    }
   }
   __syncthreads();
   uint32_t prefix = 0, himask = 0;
-  int kk = k;
+  int kk = kb;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     for (int i = tid; i < kSubHists * 256; i += kTopkThreads) (&sh.sub[0][0])[i] = 0;
     __syncthreads();
     for (int j = tid; j < mloc; j += kTopkThreads) {
-      const uint32_t u = kb[j];
+      const uint32_t u = key[j];
       if ((u & himask) == prefix) atomicAdd(&sh.sub[warp >> 1][(u >> shift) & 255u], 1);
     }
     __syncthreads();
@@ -235,7 +259,7 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
   {
     int gt = 0, eq = 0;
     for (int j = tid; j < mloc; j += kTopkThreads) {
-      const uint32_t u = kb[j];
+      const uint32_t u = key[j];
       gt += u > T;
       eq += u == T;
     }
@@ -270,7 +294,7 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
     const int j = r0 + 4 * tid;
     uint32_t u[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) u[e] = j + e < mloc ? kb[j + e] : 0u;
+    for (int e = 0; e < 4; ++e) u[e] = j + e < mloc ? key[j + e] : 0u;
     int gt = 0, eq = 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -284,18 +308,19 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       if (j + e >= mloc) break;
+      const int c = j0 + j + e;
       if (u[e] > T) {
-        ob[gt_before + min(eq_before, kk)] = __ldg(ib + j0 + j + e);
+        ob[gt_before + min(eq_before, kk)] = direct ? c : __ldg(ib + c);
         ++gt_before;
       } else if (u[e] == T) {
-        if (eq_before < kk) ob[gt_before + eq_before] = __ldg(ib + j0 + j + e);
+        if (eq_before < kk) ob[gt_before + eq_before] = direct ? c : __ldg(ib + c);
         ++eq_before;
       }
     }
     gt_base += gt_round;
     eq_base += eq_round;
   }
-  if (rank == 0 && tid == 0 && topk_count) topk_count[b] = k;
+  if (rank == 0 && tid == 0 && topk_count) topk_count[b] = kb;
 }
 
 }  // namespace
@@ -317,10 +342,11 @@ int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, in
   return check_launch("compact");
 }
 
-int launch_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
-                const float* logit, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws,
-                cudaStream_t s) {
-  if (B == 0) return LSA_OK;
+namespace {
+
+int launch_topk_cluster(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
+                        const float* logit, const uint32_t* dkeys, const int32_t* kdev, const int32_t* kept,
+                        int32_t* status, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws, cudaStream_t s) {
   const int smem = kTopkSmemKeys * 4;
   cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   int sms = 148, dev = 0;
@@ -346,8 +372,26 @@ int launch_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const i
     if (cudaOccupancyMaxActiveClusters(&clusters, topk_cluster_kernel, &cfg) == cudaSuccess && clusters > 0) break;
     cudaGetLastError();
   }
-  cudaLaunchKernelEx(&cfg, topk_cluster_kernel, B, L, N, k, idx, cap, count, logit, keys_ws, topk, topk_count);
+  cudaLaunchKernelEx(&cfg, topk_cluster_kernel, B, L, N, k, idx, cap, count, logit, dkeys, kdev, kept, status,
+                     keys_ws, topk, topk_count);
   return check_launch("topk");
+}
+
+}  // namespace
+
+int launch_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
+                const float* logit, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws,
+                cudaStream_t s) {
+  if (B == 0) return LSA_OK;
+  return launch_topk_cluster(B, L, N, k, idx, cap, count, logit, nullptr, nullptr, nullptr, nullptr, topk,
+                             topk_count, keys_ws, s);
+}
+
+int launch_select_keys(int B, int n, const uint32_t* keys, const int32_t* kdev, const int32_t* kept,
+                       int32_t* status, int32_t* out, int32_t* out_count, uint32_t* keys_ws, cudaStream_t s) {
+  if (B == 0) return LSA_OK;
+  return launch_topk_cluster(B, 0, n, 0, nullptr, n, nullptr, nullptr, keys, kdev, kept, status, out, out_count,
+                             keys_ws, s);
 }
 
 }  // namespace lsa

@@ -66,6 +66,24 @@ def test_host_side_argument_errors(lib):
     rc = lib.lsa_index_score(*args, 0, 256, 256, 256, 256, 256, 0, 256, None, 0,
                              None, None, None, None, 256, None, None, None, None, 0, None)
     assert rc == lsa.LSA_ERR_NOMEM                  # no workspace
+    upd = lib.lsa_hot_pool_update
+    assert upd(1, 64, 8, 1152, 0, 256, 256, 256, 256, None, None, 256, 1 << 20, None) == lsa.LSA_ERR_INVALID_ARG
+    assert b"trigger" in lib.lsa_last_error()
+    assert upd(1, 64, 0, 1152, 1, 256, 256, 256, 256, None, None, 256, 1 << 20, None) == lsa.LSA_ERR_INVALID_ARG
+    assert upd(1, 64, 8, 24, 1, 256, 256, 256, 256, None, None, 256, 1 << 20, None) == lsa.LSA_ERR_INVALID_ARG
+    assert upd(1, 64, 8, 1152, 1, None, 256, 256, 256, None, None, 256, 1 << 20, None) == lsa.LSA_ERR_INVALID_ARG
+    assert upd(1, 64, 8, 1152, 1, 256, 256, 256, 264, None, None, 256, 1 << 20, None) == lsa.LSA_ERR_INVALID_ARG
+    assert upd(1, 64, 8, 1152, 1, 256, 256, 256, 256, None, None, 256, 16, None) == lsa.LSA_ERR_NOMEM
+    assert lib.lsa_hot_pool_reset(1, 64, 8, None, None) == lsa.LSA_ERR_INVALID_ARG
+
+
+def test_hot_pool_layout():
+    B, N, slots = 3, 1000, 40
+    off = lsa.lsa_hot_pool_layout(B, N, slots)
+    assert off[0] == 0 and all(o % 256 == 0 for o in off)
+    assert off[1] >= B * N * 4 and off[2] >= off[1] + B * slots * 4 and off[3] >= off[2] + B * slots * 4
+    assert lsa.lsa_hot_pool_state_bytes(B, N, slots) >= off[3] + B * ((N + 31) // 32) * 4
+    assert lsa.lsa_hot_pool_workspace_bytes(B, N, slots) > 0
 
 
 def test_workspace_queries(lib):
