@@ -53,6 +53,7 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-vote", action="store_true", help="skip the vote-label measurement")
+    ap.add_argument("--no-hot-pool", action="store_true", help="skip the residency measurement")
     return ap.parse_args(argv)
 
 
@@ -420,6 +421,65 @@ def reference_arm(args):
     return 0
 
 
+def hot_pool_measure(lsa, trig, device, triggers=8, rho=0.9):
+    """Residency across triggers on the benchmark workload: `triggers` consecutive
+    triggers whose hidden states drift (h_t = rho h_{t-1} + sqrt(1 - rho^2) eps_t).  Each
+    trigger projects, scores all layers, unions them, compacts the union and ranks it on
+    the main stream, while lsa_hot_pool_update on the side stream moves only the rows of
+    the union not yet resident.  The first trigger fills an empty pool; the figures
+    are the mean over the later ones (device time, CUDA events around each trigger)."""
+    w, inp = trig.w, trig.inp
+    B, L, N = w.B, w.L, w.N
+    slots = N               # a sequence's union can reach most of N here; no update may fail
+    hs = [W.drifted_hidden_states(w, t, rho, device).transpose(0, 1).contiguous() for t in range(1, triggers + 1)]
+    hot = torch.empty(B, slots, w.row_bytes, dtype=torch.uint8, device=device)
+    state = lsa.workspace(lsa.lsa_hot_pool_state_bytes(B, N, slots), device)
+    ws = lsa.workspace(lsa.lsa_hot_pool_workspace_bytes(B, N, slots), device)
+    moved = torch.zeros(B, dtype=torch.int32, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    m, sd = trig.main, trig.side
+    lsa.lsa_hot_pool_reset(B, N, slots, state, stream=m)
+    torch.cuda.synchronize()
+    ms, moved_rows, fetch_rows = [], [], []
+    for t, h in enumerate(hs, start=1):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(m)
+        lsa.lsa_index_project(B, L, w.D, w.r, w.H, w.dI, trig.wdt, h, inp["Wd"], inp["Wu"], inp["Ww"], -1,
+                              trig.q, trig.wv, trig.ws_proj, stream=m)
+        lsa.lsa_index_score(B, L, N, w.D, w.r, w.H, w.dI, trig.wdt, None, None, None, None, inp["bias"],
+                            trig.kdt, inp["K"], inp["kscale"], -1, trig.q, trig.wv, None, None,
+                            trig.mask, trig.logit, None, trig.ws_score, status=status, stream=m)
+        with torch.cuda.stream(m):
+            trig.U.zero_()
+        for l in range(L):
+            lsa.lsa_select_union(B, trig.Nw, trig.mask[l], trig.U, None, stream=m)
+        ready = torch.cuda.Event()
+        ready.record(m)
+        sd.wait_event(ready)
+        lsa.lsa_hot_pool_update(B, N, slots, w.row_bytes, t, trig.U, trig.cold, hot, state, moved, status, ws,
+                                stream=sd)
+        lsa.lsa_compact(B, N, trig.U, N, trig.idx_U, trig.cnt_U, status, stream=m)
+        lsa.lsa_topk(B, L, N, w.k, trig.idx_U, N, trig.cnt_U, trig.logit, trig.topk, trig.topk_cnt, trig.ws_topk,
+                     stream=m)
+        done = torch.cuda.Event()
+        done.record(sd)
+        m.wait_event(done)
+        e1.record(m)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+        moved_rows.append(int(moved.sum().item()))
+        fetch_rows.append(int(trig.cnt_U.sum().item()))
+    st = int(status.item())
+    later = slice(1, None)
+    mean = lambda xs: statistics.mean(xs[later])
+    return {"workload": f"{w.name}, {triggers} triggers, hidden-state drift rho={rho} between triggers",
+            "slots_per_sequence": slots, "status": st,
+            "value": B * L * N / (mean(ms) * 1e-3), "unit": UNIT, "ms_per_trigger": mean(ms),
+            "first_trigger_ms": ms[0], "fetch_rows_per_trigger": mean(fetch_rows),
+            "moved_rows_per_trigger": mean(moved_rows), "first_trigger_moved_rows": moved_rows[0],
+            "host_link_bytes_per_trigger": mean(moved_rows) * w.row_bytes}
+
+
 def vote_measure(lsa, device, steps=5):
     """Cross-layer vote labels + loss on the L=24 x P=64 x N=131072 workload: logits from the
     generator, loss scores from the 512K workload's scorer (sequence 0, layer 0), one query
@@ -562,6 +622,9 @@ def our_arm(args):
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         base = cpu_baseline(inp, w)
+    hot_pool = None
+    if rank == 0 and not args.no_hot_pool:
+        hot_pool = hot_pool_measure(lsa, trig, device)
     vote = None
     if rank == 0 and not args.no_vote:
         del trig, cold
@@ -595,6 +658,7 @@ def our_arm(args):
             "select_path": {"value": sel_value, "unit": UNIT, "ms_per_step": sel_ms / args.steps,
                             "covers": "projection, scoring, union, compaction and top-k on the main stream of "
                                       "each timed step, with that step's gathers running on the side stream"},
+            "hot_pool": hot_pool,
             "vote_labels": vote,
         }
         print(json.dumps(line), flush=True)

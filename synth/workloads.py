@@ -38,6 +38,7 @@ from . import rng
 # Stream identifiers (any fixed small integers will do; they only separate streams).
 _S_H, _S_WDOWN, _S_WUP, _S_WW, _S_FRAC, _S_PLANT, _S_KNOISE, _S_COLD = range(1, 9)
 _S_VOTE_X, _S_VOTE_BOOST_SET, _S_VOTE_BOOST_LAYERS, _S_VOTE_NLAYERS, _S_POS_H = range(20, 25)
+_S_DRIFT = 30
 
 E4M3_MAX = 448.0
 
@@ -144,6 +145,23 @@ def hidden_states(w: ScoreWorkload, device="cpu") -> torch.Tensor:
             key = rng.stream_key(w.seed, _S_H, b, l)
             out[b, l] = _to_storage(rng.normal(key, rng.arange(w.D, device=device)), w.wdtype)
     return out
+
+
+def drifted_hidden_states(w: ScoreWorkload, t: int, rho: float, device="cpu") -> torch.Tensor:
+    """h [B][L][D] at trigger t >= 1 of a sequence of triggers whose hidden states follow
+    an AR(1) walk: h_1 = hidden_states(w), h_t = rho h_{t-1} + sqrt(1 - rho^2) eps_t with
+    eps_t ~ N(0, 1) from its own stream (fp64, stored in w.wdtype)."""
+    h = torch.empty(w.B, w.L, w.D, dtype=torch.float64, device=device)
+    for b in range(w.B):
+        for l in range(w.L):
+            h[b, l] = rng.normal(rng.stream_key(w.seed, _S_H, b, l), rng.arange(w.D, device=device))
+    c = math.sqrt(max(0.0, 1.0 - rho * rho))
+    for step in range(2, t + 1):
+        for b in range(w.B):
+            for l in range(w.L):
+                eps = rng.normal(rng.stream_key(w.seed, _S_DRIFT, b, l, step), rng.arange(w.D, device=device))
+                h[b, l] = rho * h[b, l] + c * eps
+    return _to_storage(h, w.wdtype)
 
 
 def layer_weights(w: ScoreWorkload, l: int, device="cpu"):
