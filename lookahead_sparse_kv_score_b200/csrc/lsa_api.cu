@@ -185,6 +185,7 @@ int lsa_index_score(int B, int L, int N, int D, int r, int H, int dI,
     pa.w_out = w_out;
     pa.do_q = need_q;
     pa.do_w = need_w;
+    pa.status = status;
     rc = launch_project(pa, st);
     if (rc != LSA_OK) return rc;
   }

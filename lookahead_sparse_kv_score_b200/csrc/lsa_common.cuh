@@ -55,8 +55,18 @@ struct ProjectArgs {
   void* q_out;
   float* w_out;
   bool do_q, do_w;      // project the query / the head weights
+  int32_t* status;      // device status word or null (a tensor-core pipeline wait that gave up)
 };
 int launch_project(const ProjectArgs& a, cudaStream_t s);
+// Tensor-core projection (bf16 weights, B <= 256) and the reductions it shares with the
+// CUDA-core version.
+struct ProjectTcBufs {
+  __nv_bfloat16* c_bf16;   // [nL][B][r]: c rounded to bf16, the input of q = c W_up
+};
+bool project_tc_supported(const ProjectArgs& a);
+int launch_project_tc(const ProjectArgs& a, const ProjectTcBufs& t, cudaStream_t s);
+int launch_project_reductions(const ProjectArgs& a, int S, const ProjectTcBufs& t, cudaStream_t s);
+int launch_project_q_reduction(const ProjectArgs& a, int S, cudaStream_t s);
 int project_splits(int K);     // reduction slices of h W_down / h W_w (length K = D)
 int project_splits_b(int K);   // reduction slices of c W_up (length K = r)
 

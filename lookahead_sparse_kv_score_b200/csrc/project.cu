@@ -228,10 +228,43 @@ int project_typed(const ProjectArgs& a, cudaStream_t st) {
 int project_splits(int K) { return (K + kSliceA - 1) / kSliceA; }
 int project_splits_b(int K) { return (K + kSliceB - 1) / kSliceB; }
 
+// Fixed-order sums of S slices for the tensor-core path: w (fp32) and c (rounded to bf16,
+// stored as bf16 for q = c W_up).
+int launch_project_reductions(const ProjectArgs& a, int S, const ProjectTcBufs& t, cudaStream_t st) {
+  int launches = 0;
+  if (a.do_w) {
+    const size_t nw = static_cast<size_t>(a.nL) * a.B * a.H;
+    const size_t woff = static_cast<size_t>(a.l0) * a.B * a.H;
+    reduce_splits<float><<<grid_for(nw), 256, 0, st>>>(a.partW, S, nw, 0, a.w_ws + woff,
+                                                        a.w_out ? a.w_out + woff : nullptr, nullptr);
+    ++launches;
+  }
+  if (a.do_q) {
+    const size_t nc = static_cast<size_t>(a.nL) * a.B * a.r;
+    reduce_splits<__nv_bfloat16><<<grid_for(nc), 256, 0, st>>>(a.partA, S, nc, 1, nullptr, t.c_bf16, nullptr);
+    ++launches;
+  }
+  return check_launch("project/reduce", launches);
+}
+
+int launch_project_q_reduction(const ProjectArgs& a, int S, cudaStream_t st) {
+  const size_t HD = static_cast<size_t>(a.H) * a.dI;
+  const size_t nq = static_cast<size_t>(a.nL) * a.B * HD;
+  const size_t qoff = static_cast<size_t>(a.l0) * a.B * HD;
+  reduce_splits<__nv_bfloat16><<<grid_for(nq), 256, 0, st>>>(
+      a.partB, S, nq, 1, nullptr, static_cast<__nv_bfloat16*>(a.q_ws) + qoff,
+      a.q_out ? static_cast<__nv_bfloat16*>(a.q_out) + qoff : nullptr);
+  return check_launch("project/reduce q");
+}
+
 int launch_project(const ProjectArgs& a, cudaStream_t s) {
   if ((a.r % 8) != 0 || (a.H % 8) != 0 || ((static_cast<size_t>(a.H) * a.dI) % 8) != 0)
     return fail(LSA_ERR_UNSUPPORTED, "project: r, H and H*dI must be multiples of 8");
-  if (a.wdt == LSA_BF16) return project_typed<__nv_bfloat16>(a, s);
+  if (a.wdt == LSA_BF16) {
+    if (project_tc_supported(a))
+      return launch_project_tc(a, ProjectTcBufs{reinterpret_cast<__nv_bfloat16*>(a.cbuf)}, s);
+    return project_typed<__nv_bfloat16>(a, s);
+  }
   return project_typed<float>(a, s);
 }
 

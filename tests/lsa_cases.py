@@ -147,7 +147,12 @@ class OracleCache:
         return dq @ np.abs(wv) + (np.maximum(Kd @ q.T, 0) + dq) @ self.w_allowed(l, b)
 
 
-FP32_DEPTH = 300   # longest chain of sequential fp32 additions in the projection kernels (256 + 16 + margin)
+# Longest chain of fp32 additions behind one projected element, in units of 2^-24 relative
+# error each.  CUDA cores: 256-element slices and 16 slice sums.  Tensor cores: a
+# 512-element slice accumulated by tcgen05.mma, whose addition order and rounding mode
+# are unspecified, counted as 512 additions of error up to 2^-23 each, then 8 fp32 slice
+# sums; with margin.
+FP32_DEPTH = 1100
 
 
 def bf16_ulp(x: np.ndarray) -> np.ndarray:
