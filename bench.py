@@ -38,7 +38,8 @@ METRIC = "LSA entries scored+selected/sec at 1M ctx (B=32, 3 layers); % of roofl
 UNIT = "entry-layer scorings/s"
 DEFAULT_WORKLOAD = "lsa_step_1m_b32_fp8"
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "score_tc_fp8_1m_b32_traffic.txt")
-SCORE_SRC = os.path.join(ROOT, "lookahead_sparse_kv_score_b200", "csrc", "score_tc.cu")
+# the score kernel's source: the kernel file and the tcgen05 / TMA wrappers it includes
+SCORE_SRC = [os.path.join(ROOT, "lookahead_sparse_kv_score_b200", "csrc", f) for f in ("score_tc.cu", "tc_ptx.cuh")]
 
 
 def parse_args(argv=None):
@@ -300,6 +301,13 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def score_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in SCORE_SRC:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()
+
+
 def traffic_per_launch():
     """DRAM bytes per score launch from the committed ncu summary, if it was taken on
     the current kernel source (else None)."""
@@ -310,7 +318,7 @@ def traffic_per_launch():
         if ":" in line:
             k, v = line.split(":", 1)
             kv[k.strip()] = v.strip()
-    sha = hashlib.sha256(open(SCORE_SRC, "rb").read()).hexdigest()
+    sha = score_source_sha()
     if kv.get("source_sha256") != sha:
         return None
     try:
