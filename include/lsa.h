@@ -259,6 +259,19 @@ int lsa_hot_pool_update(int B, int N, int slots, size_t row_bytes, uint32_t trig
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * lsa_check_bounded_wait -- self-check of the pipeline waits (no counterpart on the pages).
+ * Every wait inside the tensor-core kernels is bounded: when a pipeline stage does not
+ * arrive within its limit (2 s) the kernel drains what it issued, frees its tensor
+ * memory, raises the status word to LSA_ERR_TIMEOUT and returns.  This call launches one
+ * kernel whose wait, the same bounded wait shortened to limit_us (1 .. 2,000,000), is on
+ * a barrier that nothing arrives at: *status (device) becomes LSA_ERR_TIMEOUT after about
+ * limit_us and the context stays usable.
+ * Environment: LSA_FAULT=launch makes every call report a failed launch (LSA_ERR_CUDA),
+ * for testing callers' error paths; it is read once per process.
+ * ---------------------------------------------------------------------------------- */
+int lsa_check_bounded_wait(uint32_t limit_us, int32_t* status, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * lsa_vote_labels -- cross-layer majority-vote golden labels and their loss
  * ([SUMMARY] §2.2: softmax over the indexer logits, per-layer nucleus top-p, an entry
  * is golden when at least theta of the L layers select it; §2.3 / [REVIEW] 二: BCE

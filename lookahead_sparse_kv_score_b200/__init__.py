@@ -168,6 +168,12 @@ def lsa_hot_pool_update(B, N, slots, row_bytes, trigger, U, cold_host, hot, stat
            "lsa_hot_pool_update")
 
 
+# ----------------------------------------------------------------------------- self-check
+
+def lsa_check_bounded_wait(limit_us, status, stream=None):
+    _check(lib().lsa_check_bounded_wait(limit_us, _p(status), _stream(stream)), "lsa_check_bounded_wait")
+
+
 # ----------------------------------------------------------------------------- labels
 
 def lsa_vote_labels_workspace_bytes(L, P, N) -> int:

@@ -6,6 +6,9 @@
 #include <algorithm>
 #include <atomic>
 
+#include <cstdlib>
+#include <cstring>
+
 #include "lsa_common.cuh"
 
 namespace lsa {
@@ -21,9 +24,20 @@ int fail(int code, const char* fmt, ...) {
   return code;
 }
 
+// Host-side fault injection for the error-path tests: with LSA_FAULT=launch in the
+// environment every launch check reports a failed launch (read once per process).
+static bool injected_launch_fault() {
+  static const bool on = [] {
+    const char* v = std::getenv("LSA_FAULT");
+    return v != nullptr && std::strcmp(v, "launch") == 0;
+  }();
+  return on;
+}
+
 int check_launch(const char* what, int kernels) {
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  if (injected_launch_fault()) return fail(LSA_ERR_CUDA, "%s: injected launch failure (LSA_FAULT=launch)", what);
   g_launches.fetch_add(static_cast<unsigned long long>(kernels), std::memory_order_relaxed);
   return LSA_OK;
 }
@@ -342,6 +356,15 @@ int lsa_hot_pool_update(int B, int N, int slots, size_t row_bytes, uint32_t trig
   }
   return launch_hot_update(B, N, slots, row_bytes, trigger, U, attr.devicePointer, hot, state, moved, status,
                            workspace, static_cast<cudaStream_t>(stream));
+}
+
+int lsa_check_bounded_wait(uint32_t limit_us, int32_t* status, void* stream) {
+  g_err[0] = 0;
+  if (!status) return fail(LSA_ERR_INVALID_ARG, "check_bounded_wait: null status");
+  if (limit_us == 0 || limit_us > 2000000u)
+    return fail(LSA_ERR_INVALID_ARG, "check_bounded_wait: limit %u us outside [1, 2000000]", limit_us);
+  return launch_wait_check(static_cast<unsigned long long>(limit_us) * 1000ull, status,
+                           static_cast<cudaStream_t>(stream));
 }
 
 size_t lsa_vote_labels_workspace_bytes(int L, int P, int N) {

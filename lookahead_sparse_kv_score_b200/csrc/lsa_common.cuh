@@ -102,6 +102,10 @@ int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, in
 int launch_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
                 const float* logit, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws,
                 cudaStream_t s);
+// One kernel whose bounded wait on an mbarrier nothing arrives at gives up after
+// limit_ns and raises *status to LSA_ERR_TIMEOUT.
+int launch_wait_check(unsigned long long limit_ns, int32_t* status, cudaStream_t s);
+
 // Direct-key selection: per sequence b, the kdev[b] largest of keys[b][0..n) (ties to the
 // lower index) in ascending index order, or none with LSA_ERR_CAPACITY when kdev[b]
 // exceeds n - kept[b].  out [B][n], out_count [B].
