@@ -538,8 +538,53 @@ def vote_measure(lsa, device, steps=5):
            "loss": [float(x) for x in loss.cpu()],
            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                         "frac": achieved / hbm_peak, "bytes_per_launch": nbytes}}
+    out["train_step"] = train_measure(lsa, device, hp, Wd, Wu, Ww, K, float(b1[0].item()), golden, v.gamma,
+                                      [float(x) for x in loss.cpu()], steps)
     del logits, K, scores
     return out
+
+
+def train_measure(lsa, device, hp, Wd, Wu, Ww, K, bias, golden, gamma, vote_loss, steps=5):
+    """One indexer training step (lsa_index_train_step) on the vote workload's P = 64
+    positions against sequence 0's N = 131,072 layer-0 keys of the 512K workload, with
+    the vote's golden bits as labels: projection, fused forward + backward on the tensor
+    cores, projection gradients.  The loss it reports must equal the vote call's loss
+    (same scorer, same labels).  Roofline: the forward and backward key products,
+    4 P H dI N flops, against the measured dense bf16 peak."""
+    P, D = hp.shape
+    r, HD = Wu.shape[1], Wu.shape[2]
+    H = Ww.shape[2]
+    dI = HD // H
+    N = K.shape[2]
+    loss = torch.zeros(2, dtype=torch.float64, device=device)
+    dbias = torch.zeros(1, dtype=torch.float64, device=device)
+    dWd = torch.empty(D, r, device=device)
+    dWu = torch.empty(r, HD, device=device)
+    dWw = torch.empty(D, H, device=device)
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    ws = lsa.workspace(lsa.lsa_index_train_step_workspace_bytes(P, N, D, r, H, dI), device)
+    Kf = K.reshape(N, dI)
+    run = lambda: lsa.lsa_index_train_step(P, N, D, r, H, dI, 1, hp, Wd[0], Wu[0], Ww[0], bias, 1, Kf, None, golden,
+                                           gamma, None, None, None, loss, dWd, dWu, dWw, dbias, ws, status=st)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        run()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    flops = 4.0 * P * H * dI * N
+    peak = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))).get("bf16_tflops") \
+        if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 1590.0
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"workload": f"train_step_l0_p{P}_n{N} (H={H}, dI={dI}, D={D}, r={r}, vote labels)", "ms": ms,
+            "status": int(st.item()), "loss": [float(x) for x in loss.cpu()], "vote_loss": vote_loss,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "flops_per_step": flops,
+                         "peak_kind": "measured dense bf16 (burst)"}}
 
 
 def our_arm(args):

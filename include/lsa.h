@@ -259,6 +259,36 @@ int lsa_hot_pool_update(int B, int N, int slots, size_t row_bytes, uint32_t trig
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * lsa_index_train_step -- loss and gradients of one indexer training step ([SUMMARY]
+ * §2.3: K_IComp frozen, only the query-side projections trained, BCE combined with a
+ * focal loss; §2.2: vote labels).  For P query positions of one indexer layer against N
+ * frozen keys:
+ *   c = h W_down, q = c W_up (both rounded to bf16), w = h W_w;
+ *   z_ps = sum_h w_ph ReLU(q_ph . k_s) + bias;  prob = sigmoid(z) clamped to [2^-20, 1 - 2^-20];
+ *   J = mean BCE(prob, y) + mean focal(prob, y; gamma) over all P*N pairs;
+ *   outputs: loss[0] = mean BCE, loss[1] = mean focal (device doubles, or NULL);
+ *   dW_down [D][r], dW_up [r][H*dI], dW_w [D][H] fp32 = dJ/dW; *dbias = dJ/dbias (device
+ *   double, or NULL).  The bf16 roundings pass gradients straight through; where the
+ *   probability clamp is active the derivative is zero.
+ *   h [P][D], W_down [D][r], W_up [r][H*dI], W_w [D][H]: bf16 (wdt = LSA_BF16).
+ *   K [N][dI] bf16 (kdt = LSA_BF16, kscale NULL); labels [P][ceil(N/32)] bits.
+ *   c_in [P][r] bf16, q_in [P][H][dI] bf16, w_in [P][H] fp32: all three (the forward
+ *   projection, e.g. from lsa_index_project) or none (then projected here; P <= 256).
+ *   Supported: H in {32, 64, 128}, dI in {64, 128}, P a multiple of 128/H; else
+ *   LSA_ERR_UNSUPPORTED.  workspace: lsa_index_train_step_workspace_bytes bytes.
+ *   The product of the keys with the positions' queries (forward) and with the gated
+ *   gradients (backward) runs on the tensor cores; a stalled pipeline ends as
+ *   LSA_ERR_TIMEOUT in *status.
+ * ---------------------------------------------------------------------------------- */
+size_t lsa_index_train_step_workspace_bytes(int P, int N, int D, int r, int H, int dI);
+int lsa_index_train_step(int P, int N, int D, int r, int H, int dI, int wdt,
+                         const void* h, const void* W_down, const void* W_up, const void* W_w, float bias,
+                         int kdt, const void* K, const float* kscale, const uint32_t* labels, float gamma,
+                         const void* c_in, const void* q_in, const float* w_in,
+                         double* loss, float* dW_down, float* dW_up, float* dW_w, double* dbias,
+                         int32_t* status, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * lsa_check_bounded_wait -- self-check of the pipeline waits (no counterpart on the pages).
  * Every wait inside the tensor-core kernels is bounded: when a pipeline stage does not
  * arrive within its limit (2 s) the kernel drains what it issued, frees its tensor

@@ -168,6 +168,21 @@ def lsa_hot_pool_update(B, N, slots, row_bytes, trigger, U, cold_host, hot, stat
            "lsa_hot_pool_update")
 
 
+# ----------------------------------------------------------------------------- training step
+
+def lsa_index_train_step_workspace_bytes(P, N, D, r, H, dI) -> int:
+    return int(lib().lsa_index_train_step_workspace_bytes(P, N, D, r, H, dI))
+
+
+def lsa_index_train_step(P, N, D, r, H, dI, wdt, h, W_down, W_up, W_w, bias, kdt, K, kscale, labels, gamma,
+                         c_in, q_in, w_in, loss, dW_down, dW_up, dW_w, dbias, workspace, status=None, stream=None):
+    _check(lib().lsa_index_train_step(P, N, D, r, H, dI, wdt, _p(h), _p(W_down), _p(W_up), _p(W_w), float(bias), kdt,
+                                      _p(K), _p(kscale), _p(labels), float(gamma), _p(c_in), _p(q_in), _p(w_in),
+                                      _p(loss), _p(dW_down), _p(dW_up), _p(dW_w), _p(dbias), _p(status),
+                                      _p(workspace), 0 if workspace is None else workspace.numel(),
+                                      _stream(stream)), "lsa_index_train_step")
+
+
 # ----------------------------------------------------------------------------- self-check
 
 def lsa_check_bounded_wait(limit_us, status, stream=None):

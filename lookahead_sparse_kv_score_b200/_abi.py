@@ -41,6 +41,11 @@ SIGNATURES = {
     "lsa_hot_pool_update": (c_int, [c_int, c_int, c_int, c_size_t, ctypes.c_uint32, c_void_p, c_void_p, c_void_p,
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "lsa_check_bounded_wait": (c_int, [ctypes.c_uint32, c_void_p, c_void_p]),
+    "lsa_index_train_step_workspace_bytes": (c_size_t, [c_int] * 6),
+    "lsa_index_train_step": (c_int, [c_int] * 7 + [c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_int,
+                                                    c_void_p, c_void_p, c_void_p, c_float, c_void_p, c_void_p,
+                                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                    c_void_p, c_void_p, c_size_t, c_void_p]),
     "lsa_vote_labels_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
     "lsa_vote_labels": (c_int, [c_int, c_int, c_int, c_void_p, c_float, c_int, c_void_p, c_void_p,
                                 c_void_p, c_float, c_void_p, c_void_p, c_size_t, c_void_p]),

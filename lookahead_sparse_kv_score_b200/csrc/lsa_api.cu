@@ -358,6 +358,77 @@ int lsa_hot_pool_update(int B, int N, int slots, size_t row_bytes, uint32_t trig
                            workspace, static_cast<cudaStream_t>(stream));
 }
 
+// Workspace of lsa_index_train_step: the projection's regions (as lsa_index_score with
+// B = P, L = 1), then the training regions.
+static size_t train_ws_bytes(int P, int N, int D, int r, int H, int dI, int wdt, size_t* proj_bytes) {
+  const ScoreWs pw = score_ws(P, 1, D, r, H, dI, wdt, LSA_BF16);
+  const size_t pb = align_up(pw.qimg, 1024);      // regions up to (not including) the query images
+  if (proj_bytes) *proj_bytes = pb;
+  return pb + train_layout(P, N, D, r, H, dI).total;
+}
+
+size_t lsa_index_train_step_workspace_bytes(int P, int N, int D, int r, int H, int dI) {
+  if (P <= 0 || N < 0 || D <= 0 || r <= 0 || H <= 0 || dI <= 0) return 0;
+  return train_ws_bytes(P, N, D, r, H, dI, LSA_BF16, nullptr);
+}
+
+int lsa_index_train_step(int P, int N, int D, int r, int H, int dI, int wdt,
+                         const void* h, const void* W_down, const void* W_up, const void* W_w, float bias,
+                         int kdt, const void* K, const float* kscale, const uint32_t* labels, float gamma,
+                         const void* c_in, const void* q_in, const float* w_in,
+                         double* loss, float* dW_down, float* dW_up, float* dW_w, double* dbias,
+                         int32_t* status, void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  if (P <= 0 || N < 0 || D <= 0 || r <= 0 || H <= 0 || dI <= 0)
+    return fail(LSA_ERR_INVALID_ARG, "index_train_step: bad size");
+  if (!train_supported(P, H, dI, wdt, kdt) || kscale != nullptr || D % 8 != 0 || r % 8 != 0)
+    return fail(LSA_ERR_UNSUPPORTED,
+                "index_train_step: needs bf16 weights and keys, H in {32, 64, 128}, dI in {64, 128}, P a multiple "
+                "of 128/H, D and r multiples of 8");
+  const bool given = c_in || q_in || w_in;
+  if (given && !(c_in && q_in && w_in))
+    return fail(LSA_ERR_INVALID_ARG, "index_train_step: give all of c_in, q_in, w_in or none");
+  if (!given && P > 256) return fail(LSA_ERR_UNSUPPORTED, "index_train_step: projecting P > 256 positions");
+  if (!h || !W_up || !K || !labels || !dW_down || !dW_up || !dW_w || (!given && (!W_down || !W_w)))
+    return fail(LSA_ERR_INVALID_ARG, "index_train_step: null pointer");
+  const void* ptrs[] = {h, W_down, W_up, W_w, K, labels, c_in, q_in, w_in, dW_down, dW_up, dW_w};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return fail(LSA_ERR_INVALID_ARG, "index_train_step: pointer %p not 16-byte aligned", p);
+  size_t pb = 0;
+  const size_t need = train_ws_bytes(P, N, D, r, H, dI, wdt, &pb);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+    return fail(LSA_ERR_NOMEM, "index_train_step: workspace %zu bytes (need %zu)", workspace_bytes, need);
+  if (N == 0) return LSA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  const ScoreWs pw = score_ws(P, 1, D, r, H, dI, wdt, LSA_BF16);
+  TrainArgs ta{};
+  ta.P = P; ta.N = N; ta.D = D; ta.r = r; ta.H = H; ta.dI = dI;
+  ta.h = h; ta.W_up = W_up; ta.K = K; ta.bias = bias; ta.gamma = gamma; ta.labels = labels;
+  ta.loss = loss; ta.dbias = dbias; ta.dW_down = dW_down; ta.dW_up = dW_up; ta.dW_w = dW_w;
+  ta.status = status; ta.ws = base + pb;
+  if (given) {
+    ta.c = c_in; ta.q = q_in; ta.w = w_in;
+  } else {
+    ProjectArgs pa{};
+    pa.B = P; pa.L = 1; pa.D = D; pa.r = r; pa.H = H; pa.dI = dI; pa.wdt = wdt; pa.l0 = 0; pa.nL = 1;
+    pa.h = h; pa.W_down = W_down; pa.W_up = W_up; pa.W_w = W_w;
+    pa.partA = reinterpret_cast<float*>(base + pw.partA);
+    pa.partW = reinterpret_cast<float*>(base + pw.partW);
+    pa.partB = reinterpret_cast<float*>(base + pw.partB);
+    pa.cbuf = reinterpret_cast<float*>(base + pw.cbuf);
+    pa.q_ws = base + pw.q;
+    pa.w_ws = reinterpret_cast<float*>(base + pw.w);
+    pa.do_q = pa.do_w = true;
+    pa.status = status;
+    if (!project_tc_supported(pa)) return fail(LSA_ERR_UNSUPPORTED, "index_train_step: projection shape");
+    const int rc = launch_project(pa, st);      // leaves c (bf16) in cbuf, q and w in the workspace
+    if (rc != LSA_OK) return rc;
+    ta.c = base + pw.cbuf; ta.q = base + pw.q; ta.w = reinterpret_cast<const float*>(base + pw.w);
+  }
+  return launch_train(ta, st);
+}
+
 int lsa_check_bounded_wait(uint32_t limit_us, int32_t* status, void* stream) {
   g_err[0] = 0;
   if (!status) return fail(LSA_ERR_INVALID_ARG, "check_bounded_wait: null status");

@@ -102,6 +102,26 @@ int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, in
 int launch_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
                 const float* logit, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws,
                 cudaStream_t s);
+// One indexer training step (bf16 weights and keys): loss sums, db and the gradients of
+// W_down, W_up, W_w from P positions' c [P][r], q [P][H][dI] (bf16) and w [P][H].
+struct TrainArgs {
+  int P, N, D, r, H, dI;
+  const void *h, *c, *q, *W_up, *K;
+  const float* w;
+  float bias, gamma;
+  const uint32_t* labels;
+  double *loss, *dbias;
+  float *dW_down, *dW_up, *dW_w;
+  int32_t* status;
+  void* ws;
+};
+struct TrainLayout {
+  size_t qimg, upart, dq, dw, dc, dcpart, dq16, acc, total;
+};
+bool train_supported(int P, int H, int dI, int wdt, int kdt);
+TrainLayout train_layout(int P, int N, int D, int r, int H, int dI);
+int launch_train(const TrainArgs& a, cudaStream_t s);
+
 // One kernel whose bounded wait on an mbarrier nothing arrives at gives up after
 // limit_ns and raises *status to LSA_ERR_TIMEOUT.
 int launch_wait_check(unsigned long long limit_ns, int32_t* status, cudaStream_t s);

@@ -1,0 +1,561 @@
+// One indexer training step on the tensor cores: loss and gradients of the query side
+// against frozen compressed keys.
+//
+// Technical summary of FlashMemory-DeepSeek-V4 (gist.science), §2.3: K_IComp is frozen,
+// only the low-rank query projections are trained, the objective is BCE combined with a
+// focal loss; §2.2: the labels are the cross-layer majority-vote bits.  For P query
+// positions of one indexer layer:
+//   a_phs = q_ph . k_s,  z_ps = sum_h w_ph ReLU(a_phs) + b,  J = mean BCE + mean FL,
+//   g_ps = dJ/dz_ps,  U_ph = sum_s g_ps 1[a_phs > 0] k_s,
+//   dq_ph = w_ph U_ph,  dw_ph = q_ph . U_ph,  db = sum g,
+//   dW_up = c^T dq,  dc = dq W_up^T,  dW_down = h^T dc,  dW_w = h^T dw.
+//
+// train_tc_kernel fuses the forward scores, the loss terms, g and U.  A CTA owns a group
+// of 128 / H positions (128 (position, head) rows) and a chunk of key tiles of 128
+// entries.  Per tile: tcgen05.mma A = the key tile (K-major), B = the group's query
+// image -> F [entries x (p, h)] in TMEM; the epilogue warps (one thread per entry) read
+// F, form z, the loss terms and g, and write G' = g 1[a > 0] as bf16 hi and lo parts
+// (hi + lo carries g to ~2^-17) into shared memory as an MN-major operand; then
+// tcgen05.mma A = G' (MN-major, (p, h) x entries), B = the same key tile read MN-major
+// -> U [(p, h) x dI] accumulated in TMEM over the chunk.  Partial U per chunk, the loss
+// sums and db go to global memory; small CUDA-core kernels finish dq, dw and the
+// projection gradients.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "lsa_common.cuh"
+#include "tc_ptx.cuh"
+
+namespace lsa {
+namespace {
+
+using namespace tc;
+
+constexpr int kTE = 128;          // entries per key tile
+constexpr int kTR = 128;          // (position, head) rows per group
+// warp 0 producer, warp 1 MMA, warps 4 .. 4 + 4 Pg - 1 epilogue (one per TMEM lane quarter
+// and position of the group)
+template <int kH>
+constexpr int train_threads() { return 128 + 128 * (kTR / kH); }
+constexpr int kTStages = 2;
+constexpr int kTChunks = 4;       // entry chunks per group
+
+struct TrainParams {
+  int P, N, H, dI, Pg, chunks, ntiles;
+  const uint8_t* qimg;            // [groups][kTR x dI bf16], K-major, 128-byte swizzle
+  const float* w;                 // [P][H]
+  float bias, gamma;
+  const uint32_t* labels;         // [P][Nw]
+  float* Upart;                   // [chunks][P*H][dI]
+  double* acc;                    // [3]: sum BCE, sum FL, sum g
+  int32_t* status;
+};
+
+__device__ __forceinline__ uint64_t desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// fp32 accumulate, bf16 operands, M = 128; transposes select MN-major operands.
+__host__ __device__ constexpr uint32_t t_idesc(int n, bool ta, bool tb) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((ta ? 1u : 0u) << 15) | ((tb ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ bool wait_timed(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_timer() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+__device__ __forceinline__ void ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+        "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+        "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(a));
+  const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(b));
+  return lo | (hi << 16);
+}
+
+// dJ/dz of BCE + focal (gamma) for one pair, before the 1/n of the means (zero where
+// the probability clamp [2^-20, 1 - 2^-20] is active); also the pair's BCE and FL terms.
+// Everything is taken from z: the clamp is |z| > ln(2^20 - 1), p = sigmoid(z) and
+// 1 - p = sigmoid(-z) are each computed directly, ln p = -log1p(e^-z) and
+// ln(1 - p) = -log1p(e^z), so nothing near saturation rests on 1 - p in fp32.
+__device__ __forceinline__ float pair_grad(float z, bool y, float gamma, double& bce, double& fl) {
+  const float eps = 1.f / 1048576.f;
+  const float zc = 13.862942f;                 // ln(2^20 - 1): sigmoid(zc) = 1 - 2^-20
+  const bool clamped = z > zc || z < -zc;
+  float pc, qc, lp, lq;
+  if (z > zc) {
+    pc = 1.f - eps; qc = eps; lp = log1pf(-eps); lq = logf(eps);
+  } else if (z < -zc) {
+    pc = eps; qc = 1.f - eps; lp = logf(eps); lq = log1pf(-eps);
+  } else {
+    const float en = expf(-z), ep = expf(z);
+    pc = 1.f / (1.f + en);
+    qc = 1.f / (1.f + ep);
+    lp = -log1pf(en);
+    lq = -log1pf(ep);
+  }
+  const float fw = gamma == 2.f ? (y ? qc * qc : pc * pc) : (y ? powf(qc, gamma) : powf(pc, gamma));
+  float d;
+  if (y) {
+    bce -= lp;
+    fl -= static_cast<double>(fw * lp);
+    d = -qc + gamma * pc * fw * lp - fw * qc;                 // (p - 1) + g p (1-p)^g ln p - (1-p)^(g+1)
+  } else {
+    bce -= lq;
+    fl -= static_cast<double>(fw * lq);
+    d = pc + fw * pc - gamma * fw * qc * lq;                  // p + p^(g+1) - g p^g (1-p) ln(1-p)
+  }
+  return clamped ? 0.f : d;
+}
+
+template <int kH, int kDI>
+__global__ void __launch_bounds__(train_threads<kH>(), 1)
+train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
+  constexpr int kPg = kTR / kH;                        // positions per group
+  constexpr int kBoxes = kDI / 64;                     // 64-element key columns per tile row
+  constexpr int kBoxBytes = kTE * 128;                 // one box: 128 entries x 128 bytes
+  constexpr int kKeyBytes = kBoxes * kBoxBytes;
+  constexpr int kQBytes = kTR * kDI * 2;
+  constexpr int kGBytes = kTR * kTE * 2;               // one of G'hi / G'lo
+  constexpr int kGHalf = kGBytes / 2;                  // 64 (p, h) columns x 128 entry rows
+  extern __shared__ __align__(1024) uint8_t smraw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  uint8_t* keys = sm;
+  uint8_t* qs = keys + kTStages * kKeyBytes;
+  uint8_t* ghi = qs + kQBytes;
+  uint8_t* glo = ghi + kGBytes;
+  float* ws = reinterpret_cast<float*>(glo + kGBytes);                 // [kTR] head weights of the group
+  uint64_t* full = reinterpret_cast<uint64_t*>(ws + kTR);
+  uint64_t* empty = full + kTStages;
+  uint64_t* f_full = empty + kTStages;
+  uint64_t* f_free = f_full + 1;
+  uint64_t* g_full = f_free + 1;
+  uint64_t* g_free = g_full + 1;
+  uint64_t* u_done = g_free + 1;
+  uint64_t* q_bar = u_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int group = blockIdx.x, chunk = blockIdx.y;
+  const int t0 = (p.ntiles * chunk) / p.chunks, t1 = (p.ntiles * (chunk + 1)) / p.chunks;
+  const int nt = t1 - t0;
+  if (tid == 0) {
+    for (int i = 0; i < kTStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(f_full, 1);
+    mbar_init(f_free, 128 * kPg);
+    mbar_init(g_full, 128 * kPg);
+    mbar_init(g_free, 1);
+    mbar_init(u_done, 1);
+    mbar_init(q_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (tid < kTR) ws[tid] = p.w[static_cast<size_t>(group * kPg) * kH + tid];
+  if (warp == 1) tmem_alloc(tmem_slot, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tF = tmem, tU = tmem + 128;
+
+  if (warp == 0 && lane == 0) {
+    // producer: the group's query image once, then the chunk's key tiles
+    mbar_expect_tx(q_bar, kQBytes);
+    bulk_load(qs, p.qimg + static_cast<size_t>(group) * kQBytes, kQBytes, q_bar);
+    const uint64_t pol = evict_first_policy();
+    int issued = 0;
+    for (int i = 0; i < nt; ++i) {
+      const int slot = i % kTStages;
+      if (i >= kTStages && !mbar_wait(&empty[slot], ((i / kTStages) - 1) & 1, abort_flag)) break;
+      uint8_t* dst = keys + slot * kKeyBytes;
+      mbar_expect_tx(&full[slot], kKeyBytes);
+#pragma unroll
+      for (int bx = 0; bx < kBoxes; ++bx)
+        tma_load_3d(dst + bx * kBoxBytes, &mapK, bx * 64, (t0 + i) * kTE, 0, &full[slot], pol);
+      issued = i + 1;
+    }
+    for (int i = (issued > kTStages ? issued - kTStages : 0); i < issued; ++i)
+      wait_timed(&full[i % kTStages], (i / kTStages) & 1);
+    wait_timed(q_bar, 0);
+  } else if (warp == 1 && lane == 0) {
+    // MMA issuer
+    const uint32_t id_f = t_idesc(kTR, false, false), id_b = t_idesc(kDI, true, true);
+    bool ok = mbar_wait(q_bar, 0, abort_flag);
+    const uint32_t q0 = smem_u32(qs), h0 = smem_u32(ghi), l0 = smem_u32(glo);
+    for (int i = 0; ok && i < nt; ++i) {
+      const int slot = i % kTStages;
+      if (!mbar_wait(&full[slot], (i / kTStages) & 1, abort_flag)) { ok = false; break; }
+      if (i > 0 && !mbar_wait(f_free, (i - 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t k0 = smem_u32(keys + slot * kKeyBytes);
+#pragma unroll
+      for (int ks = 0; ks < kDI / 16; ++ks) {
+        const uint32_t off = (ks >> 2) * kBoxBytes + (ks & 3) * 32;
+        mma<false>(tF, desc(k0 + off, 16, 1024), desc(q0 + (ks >> 2) * (kTR * 128) + (ks & 3) * 32, 16, 1024),
+                   id_f, ks > 0 ? 1u : 0u);
+      }
+      mma_commit(f_full);
+      if (!mbar_wait(g_full, i & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int ks = 0; ks < kTE / 16; ++ks) {
+        const uint64_t bk = desc(k0 + ks * 2048, kBoxBytes, 1024);
+        mma<false>(tU, desc(h0 + ks * 2048, kGHalf, 1024), bk, id_b, (i > 0 || ks > 0) ? 1u : 0u);
+        mma<false>(tU, desc(l0 + ks * 2048, kGHalf, 1024), bk, id_b, 1u);
+      }
+      mma_commit(g_free);
+      mma_commit(&empty[slot]);
+    }
+    mma_commit(u_done);          // also after an abort: arrives once issued MMAs are done
+  } else if (warp >= 4) {
+    // epilogue warp (quarter, j): lanes = entries quarter*32 .. +31 of the tile, columns of
+    // position j of the group; at the end the j == 0 warps read U ((p, h) rows)
+    const int we = warp - 4, quarter = we & 3, j = we >> 2;
+    const int e = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const int Nw = (p.N + 31) / 32;
+    const int pp = group * kPg + j;
+    const float inv_n = 1.f / (static_cast<float>(p.P) * static_cast<float>(p.N));
+    const uint32_t* lrow = p.labels + static_cast<size_t>(pp) * Nw;
+    double bce = 0.0, fl = 0.0, gsum = 0.0;
+    for (int i = 0; i < nt; ++i) {
+      if (!mbar_wait(f_full, i & 1, abort_flag)) break;
+      tc_fence_after();
+      float a[kH];
+#pragma unroll
+      for (int c = 0; c < kH / 32; ++c) {
+        float v[32];
+        ld32(tF + lane_off + j * kH + c * 32, v);
+#pragma unroll
+        for (int u = 0; u < 32; ++u) a[c * 32 + u] = v[u];
+      }
+      tc_fence_before();
+      mbar_arrive(f_free);
+      const int s = (t0 + i) * kTE + e;
+      float g = 0.f;
+      if (s < p.N) {
+        float z = p.bias;
+#pragma unroll
+        for (int hh = 0; hh < kH; ++hh) z = fmaf(ws[j * kH + hh], fmaxf(a[hh], 0.f), z);
+        const bool y = (lrow[s >> 5] >> (s & 31)) & 1u;
+        g = pair_grad(z, y, p.gamma, bce, fl) * inv_n;
+        gsum += g;
+      }
+      if (i > 0 && !mbar_wait(g_free, (i - 1) & 1, abort_flag)) break;
+      // G' row e, columns j*kH .. +kH-1: hi and lo parts, MN-major 128-byte swizzle
+      const uint32_t rowoff = (e >> 3) * 1024 + (e & 7) * 128;
+#pragma unroll
+      for (int cidx = 0; cidx < kH / 8; ++cidx) {
+        float gh[8], gl[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float v = a[cidx * 8 + u] > 0.f ? g : 0.f;
+          gh[u] = __bfloat162float(__float2bfloat16_rn(v));
+          gl[u] = v - gh[u];
+        }
+        const int col = j * kH + cidx * 8;               // first (p, h) column of this 16-byte unit
+        const int half = col >> 6, chunk16 = (col & 63) >> 3;
+        const uint32_t off = half * kGHalf + rowoff + ((chunk16 ^ (e & 7)) << 4);
+        *reinterpret_cast<uint4*>(ghi + off) =
+            make_uint4(pack_bf16(gh[0], gh[1]), pack_bf16(gh[2], gh[3]), pack_bf16(gh[4], gh[5]), pack_bf16(gh[6], gh[7]));
+        *reinterpret_cast<uint4*>(glo + off) =
+            make_uint4(pack_bf16(gl[0], gl[1]), pack_bf16(gl[2], gl[3]), pack_bf16(gl[4], gl[5]), pack_bf16(gl[6], gl[7]));
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(g_full);
+    }
+    // all MMAs of the chunk done (or abandoned)
+    const bool got = wait_timed(u_done, 0) && !*abort_flag;
+    tc_fence_after();
+    if (got) {
+      // U rows: (p, h) = TMEM lane e of this quarter; the Pg warps of a quarter split dI
+      float* dst = p.Upart + (static_cast<size_t>(chunk) * p.P * p.H + static_cast<size_t>(group) * kTR + e) * kDI;
+      constexpr int kCols = kDI / kPg >= 32 ? kDI / kPg : 32;
+      for (int c0 = j * kCols; c0 < kDI && c0 < (j + 1) * kCols; c0 += 32) {
+        float v[32];
+        ld32(tU + lane_off + c0, v);
+        if (nt == 0) {                       // an empty chunk: no MMA wrote U
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] = 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 32; u += 4) *reinterpret_cast<float4*>(dst + c0 + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        bce += __shfl_xor_sync(0xffffffffu, bce, o);
+        fl += __shfl_xor_sync(0xffffffffu, fl, o);
+        gsum += __shfl_xor_sync(0xffffffffu, gsum, o);
+      }
+      if (lane == 0) {
+        atomicAdd(&p.acc[0], bce);
+        atomicAdd(&p.acc[1], fl);
+        atomicAdd(&p.acc[2], gsum);
+      }
+    } else if (e == 0 && j == 0) {
+      raise_status(p.status, LSA_ERR_TIMEOUT);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 256);
+}
+
+// K-major, 128-byte-swizzled image of the query rows of each group: row m = (position
+// group*Pg + m / H, head m % H), dI bf16; chunks of 64 columns, each [128 rows x 128 B].
+__global__ void train_qimg_kernel(const __nv_bfloat16* __restrict__ q, int P, int H, int dI, int Pg,
+                                  uint8_t* __restrict__ img) {
+  const int group = blockIdx.y;
+  const int units = kTR * (dI / 8);                    // 16-byte units per group
+  for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < units; u += gridDim.x * blockDim.x) {
+    const int m = u / (dI / 8), c8 = u % (dI / 8);     // row, 8-element unit along dI
+    const int pp = group * Pg + m / H, hh = m % H;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (pp < P) v = *reinterpret_cast<const uint4*>(q + (static_cast<size_t>(pp) * H + hh) * dI + c8 * 8);
+    const int chunk = c8 / 8, unit = c8 % 8;
+    const size_t off = static_cast<size_t>(group) * kTR * dI * 2 + chunk * (kTR * 128) + (m >> 3) * 1024 +
+                       (m & 7) * 128 + ((unit ^ (m & 7)) << 4);
+    *reinterpret_cast<uint4*>(img + off) = v;
+  }
+}
+
+// U = sum over chunks; dq = w U ([P][H*dI]); dw = q . U ([P][H]).  One block per (p, h).
+__global__ void train_finish_kernel(const float* __restrict__ Upart, int chunks, int rows, int dI,
+                                    const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
+                                    float* __restrict__ dq, float* __restrict__ dw) {
+  __shared__ float tmp[32];
+  const int row = blockIdx.x;
+  float part = 0.f;
+  for (int d = threadIdx.x; d < dI; d += blockDim.x) {
+    float u = 0.f;
+    for (int c = 0; c < chunks; ++c) u += Upart[(static_cast<size_t>(c) * rows + row) * dI + d];
+    dq[static_cast<size_t>(row) * dI + d] = w[row] * u;
+    part = fmaf(__bfloat162float(q[static_cast<size_t>(row) * dI + d]), u, part);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  if ((threadIdx.x & 31) == 0) tmp[threadIdx.x >> 5] = part;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) s += tmp[i];
+    dw[row] = s;
+  }
+}
+
+// out[m][n] = sum_p X[p][m] Y[p][n]  (X bf16 [P][M], Y fp32 [P][Nn]); 64 x 64 tiles.
+__global__ void __launch_bounds__(256)
+outer_acc_kernel(const __nv_bfloat16* __restrict__ X, int M, const float* __restrict__ Y, int Nn, int P,
+                 float* __restrict__ out) {
+  __shared__ float xs[16][64], ys[16][64];
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int p0 = 0; p0 < P; p0 += 16) {
+    for (int i = threadIdx.x; i < 16 * 64; i += 256) {
+      const int pp = p0 + i / 64, c = i % 64;
+      xs[i / 64][c] = (pp < P && m0 + c < M) ? __bfloat162float(X[static_cast<size_t>(pp) * M + m0 + c]) : 0.f;
+      ys[i / 64][c] = (pp < P && n0 + c < Nn) ? Y[static_cast<size_t>(pp) * Nn + n0 + c] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(xs[k][ty * 4 + a], ys[k][tx * 4 + b], acc[a][b]);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int m = m0 + ty * 4 + a, n = n0 + tx * 4 + b;
+      if (m < M && n < Nn) out[static_cast<size_t>(m) * Nn + n] = acc[a][b];
+    }
+}
+
+// dc[p][i] = sum_j dq[p][j] W_up[i][j]  (W_up bf16 [r][J]).  Tiles of 64 positions x 64
+// rows i, the reduction split into kDcSplits slices written as partial sums and added in
+// a fixed order by dc_reduce_kernel.
+constexpr int kDcSplits = 16;
+
+__global__ void __launch_bounds__(256)
+dc_kernel(const float* __restrict__ dq, int P, int J, const __nv_bfloat16* __restrict__ Wu, int r,
+          float* __restrict__ part) {
+  __shared__ float as[32][65], bs[32][65];     // [j][p], [j][i]
+  const int i0 = blockIdx.x * 64, p0 = blockIdx.y * 64, sl = blockIdx.z;
+  const int js = (J * sl) / kDcSplits, je = (J * (sl + 1)) / kDcSplits;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int j0 = js; j0 < je; j0 += 32) {
+    for (int t = threadIdx.x; t < 64 * 32; t += 256) {
+      const int row = t / 32, jj = t % 32, j = j0 + jj;
+      as[jj][row] = (p0 + row < P && j < je) ? dq[static_cast<size_t>(p0 + row) * J + j] : 0.f;
+      bs[jj][row] = (i0 + row < r && j < je) ? __bfloat162float(Wu[static_cast<size_t>(i0 + row) * J + j]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k)
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(as[k][ty * 4 + a], bs[k][tx * 4 + b], acc[a][b]);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int pp = p0 + ty * 4 + a, i = i0 + tx * 4 + b;
+      if (pp < P && i < r) part[(static_cast<size_t>(sl) * P + pp) * r + i] = acc[a][b];
+    }
+}
+
+__global__ void dc_reduce_kernel(const float* __restrict__ part, size_t n, float* __restrict__ dc) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    float v = 0.f;
+    for (int s = 0; s < kDcSplits; ++s) v += part[s * n + i];
+    dc[i] = v;
+  }
+}
+
+__global__ void train_loss_kernel(const double* __restrict__ acc, double n, double* __restrict__ loss,
+                                  double* __restrict__ dbias) {
+  if (loss) { loss[0] = acc[0] / n; loss[1] = acc[1] / n; }
+  if (dbias) dbias[0] = acc[2];
+}
+
+__global__ void to_bf16_kernel(const float* __restrict__ x, size_t n, __nv_bfloat16* __restrict__ y) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    y[i] = __float2bfloat16_rn(x[i]);
+}
+
+int train_smem(int dI) {
+  return kTStages * (dI / 64) * kTE * 128 + kTR * dI * 2 + 2 * kTR * kTE * 2 + kTR * 4 + 256 + 1024;
+}
+
+}  // namespace
+
+bool train_supported(int P, int H, int dI, int wdt, int kdt) {
+  return wdt == LSA_BF16 && kdt == LSA_BF16 && (H == 32 || H == 64 || H == 128) && (dI == 64 || dI == 128) &&
+         P >= 1 && P % (kTR / H) == 0 && P <= 4096;
+}
+
+TrainLayout train_layout(int P, int N, int D, int r, int H, int dI) {
+  TrainLayout o{};
+  const size_t Pz = static_cast<size_t>(P), HD = static_cast<size_t>(H) * dI;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t at = off; off = align_up(off + bytes, 1024); return at; };
+  const int groups = P / std::max(1, kTR / std::max(1, H));
+  o.qimg = take(static_cast<size_t>(groups) * kTR * dI * 2);
+  o.upart = take(static_cast<size_t>(kTChunks) * Pz * HD * 4);
+  o.dq = take(Pz * HD * 4);
+  o.dw = take(Pz * H * 4);
+  o.dc = take(Pz * r * 4);
+  o.dcpart = take(static_cast<size_t>(kDcSplits) * Pz * r * 4);
+  o.dq16 = take(Pz * HD * 2);
+  o.acc = take(4 * 8);
+  o.total = off;
+  (void)N; (void)D;
+  return o;
+}
+
+int launch_train(const TrainArgs& a, cudaStream_t st) {
+  const TrainLayout lay = train_layout(a.P, a.N, a.D, a.r, a.H, a.dI);
+  uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  const int Pg = kTR / a.H, groups = a.P / Pg;
+  const size_t HD = static_cast<size_t>(a.H) * a.dI;
+  uint8_t* qimg = ws + lay.qimg;
+  float* Upart = reinterpret_cast<float*>(ws + lay.upart);
+  float* dq = reinterpret_cast<float*>(ws + lay.dq);
+  float* dw = reinterpret_cast<float*>(ws + lay.dw);
+  float* dc = reinterpret_cast<float*>(ws + lay.dc);
+  double* acc = reinterpret_cast<double*>(ws + lay.acc);
+  int rc;
+  if (cudaMemsetAsync(acc, 0, 4 * 8, st) != cudaSuccess) return check_launch("train/memset", 0);
+  train_qimg_kernel<<<dim3((kTR * a.dI / 8 + 255) / 256, groups), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(a.q), a.P, a.H, a.dI, Pg, qimg);
+  if ((rc = check_launch("train/query image")) != LSA_OK) return rc;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(LSA_ERR_CUDA, "train: cuTensorMapEncodeTiled unavailable");
+  CUtensorMap mapK;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(a.dI), static_cast<cuuint64_t>(a.N), 1};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(a.dI) * 2, static_cast<cuuint64_t>(a.N) * a.dI * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kTE), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult cr = enc(&mapK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.K), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return fail(LSA_ERR_CUDA, "train: tensor map encode failed (%d)", (int)cr);
+  TrainParams p{};
+  p.P = a.P; p.N = a.N; p.H = a.H; p.dI = a.dI; p.Pg = Pg; p.chunks = kTChunks;
+  p.ntiles = (a.N + kTE - 1) / kTE;
+  p.qimg = qimg; p.w = a.w; p.bias = a.bias; p.gamma = a.gamma; p.labels = a.labels;
+  p.Upart = Upart; p.acc = acc; p.status = a.status;
+  const int smem = train_smem(a.dI);
+  const dim3 grid(groups, kTChunks);
+  auto go = [&](auto kern, int threads) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    kern<<<grid, threads, smem, st>>>(mapK, p);
+  };
+  switch (a.H * 1000 + a.dI) {
+    case 32064: go(train_tc_kernel<32, 64>, train_threads<32>()); break;
+    case 32128: go(train_tc_kernel<32, 128>, train_threads<32>()); break;
+    case 64064: go(train_tc_kernel<64, 64>, train_threads<64>()); break;
+    case 64128: go(train_tc_kernel<64, 128>, train_threads<64>()); break;
+    case 128064: go(train_tc_kernel<128, 64>, train_threads<128>()); break;
+    case 128128: go(train_tc_kernel<128, 128>, train_threads<128>()); break;
+    default: return fail(LSA_ERR_UNSUPPORTED, "train: H=%d dI=%d", a.H, a.dI);
+  }
+  if ((rc = check_launch("train/fused")) != LSA_OK) return rc;
+  train_finish_kernel<<<a.P * a.H, 128, 0, st>>>(Upart, kTChunks, a.P * a.H, a.dI,
+                                                 static_cast<const __nv_bfloat16*>(a.q), a.w, dq, dw);
+  if ((rc = check_launch("train/finish")) != LSA_OK) return rc;
+  // projection gradients
+  const __nv_bfloat16* c = static_cast<const __nv_bfloat16*>(a.c);
+  const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(a.h);
+  outer_acc_kernel<<<dim3(static_cast<unsigned>((HD + 63) / 64), (a.r + 63) / 64), 256, 0, st>>>(
+      c, a.r, dq, static_cast<int>(HD), a.P, a.dW_up);
+  float* dcpart = reinterpret_cast<float*>(ws + lay.dcpart);
+  dc_kernel<<<dim3((a.r + 63) / 64, (a.P + 63) / 64, kDcSplits), 256, 0, st>>>(
+      dq, a.P, static_cast<int>(HD), static_cast<const __nv_bfloat16*>(a.W_up), a.r, dcpart);
+  const size_t ndc = static_cast<size_t>(a.P) * a.r;
+  dc_reduce_kernel<<<static_cast<unsigned>(std::min<size_t>((ndc + 255) / 256, 1184)), 256, 0, st>>>(dcpart, ndc, dc);
+  outer_acc_kernel<<<dim3((a.r + 63) / 64, (a.D + 63) / 64), 256, 0, st>>>(h, a.D, dc, a.r, a.P, a.dW_down);
+  outer_acc_kernel<<<dim3((a.H + 63) / 64, (a.D + 63) / 64), 256, 0, st>>>(h, a.D, dw, a.H, a.P, a.dW_w);
+  train_loss_kernel<<<1, 1, 0, st>>>(acc, static_cast<double>(a.P) * a.N, a.loss, a.dbias);
+  return check_launch("train/projection gradients", 6);
+}
+
+}  // namespace lsa
