@@ -94,12 +94,6 @@ __device__ __forceinline__ void ld32(uint32_t taddr, float (&v)[32]) {
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(a));
-  const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(b));
-  return lo | (hi << 16);
-}
-
 // dJ/dz of BCE + focal (gamma) for one pair, before the 1/n of the means (zero where
 // the probability clamp [2^-20, 1 - 2^-20] is active); also the pair's BCE and FL terms.
 // Everything is taken from z: the clamp is |z| > ln(2^20 - 1), p = sigmoid(z) and
@@ -149,16 +143,15 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   uint8_t* keys = sm;
   uint8_t* qs = keys + kTStages * kKeyBytes;
-  uint8_t* ghi = qs + kQBytes;
-  uint8_t* glo = ghi + kGBytes;
-  float* ws = reinterpret_cast<float*>(glo + kGBytes);                 // [kTR] head weights of the group
+  uint8_t* gbuf = qs + kQBytes;                                        // [2][hi, lo] G' tiles
+  float* ws = reinterpret_cast<float*>(gbuf + 4 * kGBytes);            // [kTR] head weights of the group
   uint64_t* full = reinterpret_cast<uint64_t*>(ws + kTR);
   uint64_t* empty = full + kTStages;
-  uint64_t* f_full = empty + kTStages;
-  uint64_t* f_free = f_full + 1;
-  uint64_t* g_full = f_free + 1;
-  uint64_t* g_free = g_full + 1;
-  uint64_t* u_done = g_free + 1;
+  uint64_t* f_full = empty + kTStages;          // [2]: forward accumulator b ready
+  uint64_t* f_free = f_full + 2;                // [2]: forward accumulator b read
+  uint64_t* g_full = f_free + 2;                // [2]: G' buffer b written
+  uint64_t* g_free = g_full + 2;                // [2]: G' buffer b consumed
+  uint64_t* u_done = g_free + 2;
   uint64_t* q_bar = u_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -169,22 +162,20 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
   const int nt = t1 - t0;
   if (tid == 0) {
     for (int i = 0; i < kTStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    mbar_init(f_full, 1);
-    mbar_init(f_free, 128 * kPg);
-    mbar_init(g_full, 128 * kPg);
-    mbar_init(g_free, 1);
+    for (int b = 0; b < 2; ++b) { mbar_init(&f_full[b], 1); mbar_init(&f_free[b], 128 * kPg); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&g_full[b], 128 * kPg); mbar_init(&g_free[b], 1); }
     mbar_init(u_done, 1);
     mbar_init(q_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (tid < kTR) ws[tid] = p.w[static_cast<size_t>(group * kPg) * kH + tid];
-  if (warp == 1) tmem_alloc(tmem_slot, 256);
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tF = tmem, tU = tmem + 128;
+  const uint32_t tF = tmem, tU = tmem + 256;     // F buffers at columns 0 and 128, U at 256
 
   if (warp == 0 && lane == 0) {
     // producer: the group's query image once, then the chunk's key tiles
@@ -206,32 +197,42 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
       wait_timed(&full[i % kTStages], (i / kTStages) & 1);
     wait_timed(q_bar, 0);
   } else if (warp == 1 && lane == 0) {
-    // MMA issuer
+    // MMA issuer: the forward product of tile i+1 goes before the backward product of
+    // tile i, so the tensor pipe works while the epilogue handles tile i.
     const uint32_t id_f = t_idesc(kTR, false, false), id_b = t_idesc(kDI, true, true);
     bool ok = mbar_wait(q_bar, 0, abort_flag);
-    const uint32_t q0 = smem_u32(qs), h0 = smem_u32(ghi), l0 = smem_u32(glo);
-    for (int i = 0; ok && i < nt; ++i) {
-      const int slot = i % kTStages;
-      if (!mbar_wait(&full[slot], (i / kTStages) & 1, abort_flag)) { ok = false; break; }
-      if (i > 0 && !mbar_wait(f_free, (i - 1) & 1, abort_flag)) { ok = false; break; }
+    const uint32_t q0 = smem_u32(qs), g0 = smem_u32(gbuf);
+    auto forward = [&](int i) -> bool {
+      const int slot = i % kTStages, fb = i & 1;
+      if (!mbar_wait(&full[slot], (i / kTStages) & 1, abort_flag)) return false;
+      if (i >= 2 && !mbar_wait(&f_free[fb], ((i >> 1) - 1) & 1, abort_flag)) return false;
       tc_fence_after();
       const uint32_t k0 = smem_u32(keys + slot * kKeyBytes);
 #pragma unroll
       for (int ks = 0; ks < kDI / 16; ++ks) {
         const uint32_t off = (ks >> 2) * kBoxBytes + (ks & 3) * 32;
-        mma<false>(tF, desc(k0 + off, 16, 1024), desc(q0 + (ks >> 2) * (kTR * 128) + (ks & 3) * 32, 16, 1024),
-                   id_f, ks > 0 ? 1u : 0u);
+        mma<false>(tF + fb * 128, desc(k0 + off, 16, 1024),
+                   desc(q0 + (ks >> 2) * (kTR * 128) + (ks & 3) * 32, 16, 1024), id_f, ks > 0 ? 1u : 0u);
       }
-      mma_commit(f_full);
-      if (!mbar_wait(g_full, i & 1, abort_flag)) { ok = false; break; }
+      mma_commit(&f_full[fb]);
+      return true;
+    };
+    if (ok && nt > 0) ok = forward(0);
+    for (int i = 0; ok && i < nt; ++i) {
+      if (i + 1 < nt && !forward(i + 1)) { ok = false; break; }
+      const int gb = i & 1;
+      if (!mbar_wait(&g_full[gb], (i >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
+      const int slot = i % kTStages;
+      const uint32_t k0 = smem_u32(keys + slot * kKeyBytes);
+      const uint32_t h0 = g0 + gb * 2 * kGBytes, l0 = h0 + kGBytes;
 #pragma unroll
       for (int ks = 0; ks < kTE / 16; ++ks) {
         const uint64_t bk = desc(k0 + ks * 2048, kBoxBytes, 1024);
         mma<false>(tU, desc(h0 + ks * 2048, kGHalf, 1024), bk, id_b, (i > 0 || ks > 0) ? 1u : 0u);
         mma<false>(tU, desc(l0 + ks * 2048, kGHalf, 1024), bk, id_b, 1u);
       }
-      mma_commit(g_free);
+      mma_commit(&g_free[gb]);
       mma_commit(&empty[slot]);
     }
     mma_commit(u_done);          // also after an abort: arrives once issued MMAs are done
@@ -247,50 +248,65 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
     const uint32_t* lrow = p.labels + static_cast<size_t>(pp) * Nw;
     double bce = 0.0, fl = 0.0, gsum = 0.0;
     for (int i = 0; i < nt; ++i) {
-      if (!mbar_wait(f_full, i & 1, abort_flag)) break;
+      const int s = (t0 + i) * kTE + e;
+      const uint32_t lab = s < p.N ? __ldg(lrow + (s >> 5)) : 0u;   // issued before the wait
+      const int fb = i & 1;
+      if (!mbar_wait(&f_full[fb], (i >> 1) & 1, abort_flag)) break;
       tc_fence_after();
       float a[kH];
 #pragma unroll
       for (int c = 0; c < kH / 32; ++c) {
         float v[32];
-        ld32(tF + lane_off + j * kH + c * 32, v);
+        ld32(tF + fb * 128 + lane_off + j * kH + c * 32, v);
 #pragma unroll
         for (int u = 0; u < 32; ++u) a[c * 32 + u] = v[u];
       }
       tc_fence_before();
-      mbar_arrive(f_free);
-      const int s = (t0 + i) * kTE + e;
+      mbar_arrive(&f_free[fb]);
       float g = 0.f;
       if (s < p.N) {
-        float z = p.bias;
+        float zp[4] = {p.bias, 0.f, 0.f, 0.f};          // four independent chains
+        const float4* w4 = reinterpret_cast<const float4*>(ws + j * kH);
 #pragma unroll
-        for (int hh = 0; hh < kH; ++hh) z = fmaf(ws[j * kH + hh], fmaxf(a[hh], 0.f), z);
-        const bool y = (lrow[s >> 5] >> (s & 31)) & 1u;
+        for (int hh = 0; hh < kH; hh += 4) {
+          const float4 wv = w4[hh >> 2];
+          zp[0] = fmaf(wv.x, fmaxf(a[hh], 0.f), zp[0]);
+          zp[1] = fmaf(wv.y, fmaxf(a[hh + 1], 0.f), zp[1]);
+          zp[2] = fmaf(wv.z, fmaxf(a[hh + 2], 0.f), zp[2]);
+          zp[3] = fmaf(wv.w, fmaxf(a[hh + 3], 0.f), zp[3]);
+        }
+        const float z = (zp[0] + zp[1]) + (zp[2] + zp[3]);
+        const bool y = (lab >> (s & 31)) & 1u;
         g = pair_grad(z, y, p.gamma, bce, fl) * inv_n;
         gsum += g;
       }
-      if (i > 0 && !mbar_wait(g_free, (i - 1) & 1, abort_flag)) break;
-      // G' row e, columns j*kH .. +kH-1: hi and lo parts, MN-major 128-byte swizzle
+      // G' = g 1[a > 0]: the bf16 bit patterns of g's hi and lo parts, masked per column
+      const __nv_bfloat16 bh = __float2bfloat16_rn(g);
+      const uint32_t hb = __bfloat16_as_ushort(bh);
+      const uint32_t lb = __bfloat16_as_ushort(__float2bfloat16_rn(g - __bfloat162float(bh)));
+      const int gb = i & 1;
+      if (i >= 2 && !mbar_wait(&g_free[gb], ((i >> 1) - 1) & 1, abort_flag)) break;
+      uint8_t* ghi = gbuf + gb * 2 * kGBytes;
+      uint8_t* glo = ghi + kGBytes;
+      // G' row e, columns j*kH .. +kH-1, MN-major 128-byte swizzle
       const uint32_t rowoff = (e >> 3) * 1024 + (e & 7) * 128;
 #pragma unroll
       for (int cidx = 0; cidx < kH / 8; ++cidx) {
-        float gh[8], gl[8];
+        uint32_t wh[4], wl[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float v = a[cidx * 8 + u] > 0.f ? g : 0.f;
-          gh[u] = __bfloat162float(__float2bfloat16_rn(v));
-          gl[u] = v - gh[u];
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t m = (a[cidx * 8 + 2 * u] > 0.f ? 0x0000FFFFu : 0u) | (a[cidx * 8 + 2 * u + 1] > 0.f ? 0xFFFF0000u : 0u);
+          wh[u] = (hb | (hb << 16)) & m;
+          wl[u] = (lb | (lb << 16)) & m;
         }
         const int col = j * kH + cidx * 8;               // first (p, h) column of this 16-byte unit
         const int half = col >> 6, chunk16 = (col & 63) >> 3;
         const uint32_t off = half * kGHalf + rowoff + ((chunk16 ^ (e & 7)) << 4);
-        *reinterpret_cast<uint4*>(ghi + off) =
-            make_uint4(pack_bf16(gh[0], gh[1]), pack_bf16(gh[2], gh[3]), pack_bf16(gh[4], gh[5]), pack_bf16(gh[6], gh[7]));
-        *reinterpret_cast<uint4*>(glo + off) =
-            make_uint4(pack_bf16(gl[0], gl[1]), pack_bf16(gl[2], gl[3]), pack_bf16(gl[4], gl[5]), pack_bf16(gl[6], gl[7]));
+        *reinterpret_cast<uint4*>(ghi + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        *reinterpret_cast<uint4*>(glo + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(g_full);
+      mbar_arrive(&g_full[gb]);
     }
     // all MMAs of the chunk done (or abandoned)
     const bool got = wait_timed(u_done, 0) && !*abort_flag;
@@ -326,7 +342,7 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, 256);
+  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // K-major, 128-byte-swizzled image of the query rows of each group: row m = (position
@@ -462,7 +478,7 @@ __global__ void to_bf16_kernel(const float* __restrict__ x, size_t n, __nv_bfloa
 }
 
 int train_smem(int dI) {
-  return kTStages * (dI / 64) * kTE * 128 + kTR * dI * 2 + 2 * kTR * kTE * 2 + kTR * 4 + 256 + 1024;
+  return kTStages * (dI / 64) * kTE * 128 + kTR * dI * 2 + 4 * kTR * kTE * 2 + kTR * 4 + 512 + 1024;
 }
 
 }  // namespace
