@@ -118,6 +118,26 @@ __device__ __forceinline__ float4 load4(const float* x, int s, int N, bool vec) 
   return v;
 }
 
+// 16-byte read-only loads with an L2 eviction priority: a row's first pass keeps it in
+// L2 for the second (evict_last), the second pass is its last use (evict_first).
+__device__ __forceinline__ uint64_t l2_policy_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ float4 ldg4_hint(const float4* p, uint64_t pol) {
+  float4 v;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
 // Calls f(value, index) for every logit of the row, four loads in flight per thread.
 template <typename F>
 __device__ __forceinline__ void row_for_each(const float* x, int N, bool vec, F&& f) {
@@ -429,10 +449,11 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
       zloc += static_cast<double>(ez);
     };
     int g0 = tid;
+    const uint64_t keep = l2_policy_last();
     for (; g0 + 3 * kRowThreads < Gf; g0 += 4 * kRowThreads) {
       float4 v4[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v4[u] = __ldg(reinterpret_cast<const float4*>(x) + g0 + u * kRowThreads);
+      for (int u = 0; u < 4; ++u) v4[u] = ldg4_hint(reinterpret_cast<const float4*>(x) + g0 + u * kRowThreads, keep);
 #pragma unroll
       for (int u = 0; u < 4; ++u) body(std::true_type{}, v4[u], 4 * (g0 + u * kRowThreads));
     }
@@ -547,11 +568,12 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
       }
     };
     int g0 = tid;
+    const uint64_t last = l2_policy_first();
     // whole warps whose four groups are all full
     for (; (g0 - lane) + 31 + 3 * kRowThreads < Gf; g0 += 4 * kRowThreads) {
       float4 v4[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v4[u] = __ldg(reinterpret_cast<const float4*>(x) + g0 + u * kRowThreads);
+      for (int u = 0; u < 4; ++u) v4[u] = ldg4_hint(reinterpret_cast<const float4*>(x) + g0 + u * kRowThreads, last);
 #pragma unroll
       for (int u = 0; u < 4; ++u) body(std::true_type{}, v4[u], 4 * (g0 + u * kRowThreads));
     }
