@@ -116,7 +116,7 @@ struct TrainArgs {
   void* ws;
 };
 struct TrainLayout {
-  size_t qimg, upart, dq, dw, dc, dcpart, dq16, acc, total;
+  size_t qimg, upart, dq, dw, dc, dcpart, acc, total;
 };
 bool train_supported(int P, int H, int dI, int wdt, int kdt);
 TrainLayout train_layout(int P, int N, int D, int r, int H, int dI);

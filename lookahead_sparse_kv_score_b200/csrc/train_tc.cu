@@ -42,7 +42,7 @@ constexpr int kTStages = 2;
 constexpr int kTChunks = 4;       // entry chunks per group
 
 struct TrainParams {
-  int P, N, H, dI, Pg, chunks, ntiles;
+  int P, N, H, dI, chunks, ntiles;
   const uint8_t* qimg;            // [groups][kTR x dI bf16], K-major, 128-byte swizzle
   const float* w;                 // [P][H]
   float bias, gamma;
@@ -471,12 +471,6 @@ __global__ void train_loss_kernel(const double* __restrict__ acc, double n, doub
   if (dbias) dbias[0] = acc[2];
 }
 
-__global__ void to_bf16_kernel(const float* __restrict__ x, size_t n, __nv_bfloat16* __restrict__ y) {
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x)
-    y[i] = __float2bfloat16_rn(x[i]);
-}
-
 int train_smem(int dI) {
   return kTStages * (dI / 64) * kTE * 128 + kTR * dI * 2 + 4 * kTR * kTE * 2 + kTR * 4 + 512 + 1024;
 }
@@ -500,7 +494,6 @@ TrainLayout train_layout(int P, int N, int D, int r, int H, int dI) {
   o.dw = take(Pz * H * 4);
   o.dc = take(Pz * r * 4);
   o.dcpart = take(static_cast<size_t>(kDcSplits) * Pz * r * 4);
-  o.dq16 = take(Pz * HD * 2);
   o.acc = take(4 * 8);
   o.total = off;
   (void)N; (void)D;
@@ -535,7 +528,7 @@ int launch_train(const TrainArgs& a, cudaStream_t st) {
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return fail(LSA_ERR_CUDA, "train: tensor map encode failed (%d)", (int)cr);
   TrainParams p{};
-  p.P = a.P; p.N = a.N; p.H = a.H; p.dI = a.dI; p.Pg = Pg; p.chunks = kTChunks;
+  p.P = a.P; p.N = a.N; p.H = a.H; p.dI = a.dI; p.chunks = kTChunks;
   p.ntiles = (a.N + kTE - 1) / kTE;
   p.qimg = qimg; p.w = a.w; p.bias = a.bias; p.gamma = a.gamma; p.labels = a.labels;
   p.Upart = Upart; p.acc = acc; p.status = a.status;
