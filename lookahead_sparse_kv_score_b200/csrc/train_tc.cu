@@ -34,12 +34,14 @@ using namespace tc;
 
 constexpr int kTE = 128;          // entries per key tile
 constexpr int kTR = 128;          // (position, head) rows per group
-// warp 0 producer, warp 1 MMA, warps 4 .. 4 + 4 Pg - 1 epilogue (one per TMEM lane quarter
-// and position of the group)
+// warp 0 producer, warp 1 MMA, warps 4 .. 19 epilogue: four per TMEM lane quarter, each
+// owning 32 of the 128 (position, head) columns
+constexpr int kEpiWarps = 16;
 template <int kH>
-constexpr int train_threads() { return 128 + 128 * (kTR / kH); }
-constexpr int kTStages = 2;
+constexpr int train_threads() { return 128 + 32 * kEpiWarps; }
+constexpr int kTStages = 3;       // key tiles in flight: the next tile's load must not wait on the MMAs
 constexpr int kTChunks = 4;       // entry chunks per group
+constexpr int kGBufs = 1;         // gated-gradient tiles (hi + lo) in shared memory
 
 struct TrainParams {
   int P, N, H, dI, chunks, ntiles;
@@ -143,9 +145,10 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   uint8_t* keys = sm;
   uint8_t* qs = keys + kTStages * kKeyBytes;
-  uint8_t* gbuf = qs + kQBytes;                                        // [2][hi, lo] G' tiles
-  float* ws = reinterpret_cast<float*>(gbuf + 4 * kGBytes);            // [kTR] head weights of the group
-  uint64_t* full = reinterpret_cast<uint64_t*>(ws + kTR);
+  uint8_t* gbuf = qs + kQBytes;                                        // [kGBufs][hi, lo] G' tiles
+  float* ws = reinterpret_cast<float*>(gbuf + kGBufs * 2 * kGBytes);   // [kTR] head weights of the group
+  float* zsm = ws + kTR;                                               // [2][4 quarters][4][32] partial z
+  uint64_t* full = reinterpret_cast<uint64_t*>(zsm + 2 * 4 * 4 * 32);
   uint64_t* empty = full + kTStages;
   uint64_t* f_full = empty + kTStages;          // [2]: forward accumulator b ready
   uint64_t* f_free = f_full + 2;                // [2]: forward accumulator b read
@@ -153,7 +156,8 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
   uint64_t* g_free = g_full + 2;                // [2]: G' buffer b consumed
   uint64_t* u_done = g_free + 2;
   uint64_t* q_bar = u_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_bar + 1);
+  uint64_t* z_bar = q_bar + 1;                  // [2 parities][4 quarters]: partial z written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(z_bar + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -162,10 +166,11 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
   const int nt = t1 - t0;
   if (tid == 0) {
     for (int i = 0; i < kTStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&f_full[b], 1); mbar_init(&f_free[b], 128 * kPg); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&g_full[b], 128 * kPg); mbar_init(&g_free[b], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&f_full[b], 1); mbar_init(&f_free[b], 32 * kEpiWarps); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&g_full[b], 32 * kEpiWarps); mbar_init(&g_free[b], 1); }
     mbar_init(u_done, 1);
     mbar_init(q_bar, 1);
+    for (int b = 0; b < 8; ++b) mbar_init(&z_bar[b], 128);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -220,8 +225,8 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
     if (ok && nt > 0) ok = forward(0);
     for (int i = 0; ok && i < nt; ++i) {
       if (i + 1 < nt && !forward(i + 1)) { ok = false; break; }
-      const int gb = i & 1;
-      if (!mbar_wait(&g_full[gb], (i >> 1) & 1, abort_flag)) { ok = false; break; }
+      const int gb = i % kGBufs;
+      if (!mbar_wait(&g_full[gb], (i / kGBufs) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const int slot = i % kTStages;
       const uint32_t k0 = smem_u32(keys + slot * kKeyBytes);
@@ -237,9 +242,12 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
     }
     mma_commit(u_done);          // also after an abort: arrives once issued MMAs are done
   } else if (warp >= 4) {
-    // epilogue warp (quarter, j): lanes = entries quarter*32 .. +31 of the tile, columns of
-    // position j of the group; at the end the j == 0 warps read U ((p, h) rows)
-    const int we = warp - 4, quarter = we & 3, j = we >> 2;
+    // epilogue warp (quarter, wq): lanes = entries quarter*32 .. +31 of the tile, columns
+    // wq*32 .. +31 = heads of position j = wq*32 / kH.  The kH/32 warps of a position add
+    // their partial z through shared memory, synchronised by a bounded mbarrier wait.
+    constexpr int kParts = kH / 32;                     // warps per position
+    const int we = warp - 4, quarter = we & 3, wq = we >> 2;
+    const int j = wq / kParts, part = wq % kParts;
     const int e = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int Nw = (p.N + 31) / 32;
@@ -253,45 +261,55 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
       const int fb = i & 1;
       if (!mbar_wait(&f_full[fb], (i >> 1) & 1, abort_flag)) break;
       tc_fence_after();
-      float a[kH];
-#pragma unroll
-      for (int c = 0; c < kH / 32; ++c) {
-        float v[32];
-        ld32(tF + fb * 128 + lane_off + j * kH + c * 32, v);
-#pragma unroll
-        for (int u = 0; u < 32; ++u) a[c * 32 + u] = v[u];
-      }
+      float a[32];
+      ld32(tF + fb * 128 + lane_off + wq * 32, a);
       tc_fence_before();
       mbar_arrive(&f_free[fb]);
+      float zp[4] = {0.f, 0.f, 0.f, 0.f};                 // four independent chains
+      const float4* w4 = reinterpret_cast<const float4*>(ws + wq * 32);
+#pragma unroll
+      for (int hh = 0; hh < 32; hh += 4) {
+        const float4 wv = w4[hh >> 2];
+        zp[0] = fmaf(wv.x, fmaxf(a[hh], 0.f), zp[0]);
+        zp[1] = fmaf(wv.y, fmaxf(a[hh + 1], 0.f), zp[1]);
+        zp[2] = fmaf(wv.z, fmaxf(a[hh + 2], 0.f), zp[2]);
+        zp[3] = fmaf(wv.w, fmaxf(a[hh + 3], 0.f), zp[3]);
+      }
+      float z = (zp[0] + zp[1]) + (zp[2] + zp[3]);
+      if constexpr (kParts > 1) {
+        // this tile parity's buffer is rewritten two tiles later, after the next exchange
+        float* zb = zsm + ((fb * 4 + quarter) * 4) * 32;
+        zb[wq * 32 + lane] = z;
+        mbar_arrive(&z_bar[fb * 4 + quarter]);
+        if (!mbar_wait(&z_bar[fb * 4 + quarter], (i >> 1) & 1, abort_flag)) break;
+        z = 0.f;
+#pragma unroll
+        for (int k = 0; k < kParts; ++k) z += zb[(j * kParts + k) * 32 + lane];
+      }
+      z += p.bias;
       float g = 0.f;
       if (s < p.N) {
-        float zp[4] = {p.bias, 0.f, 0.f, 0.f};          // four independent chains
-        const float4* w4 = reinterpret_cast<const float4*>(ws + j * kH);
-#pragma unroll
-        for (int hh = 0; hh < kH; hh += 4) {
-          const float4 wv = w4[hh >> 2];
-          zp[0] = fmaf(wv.x, fmaxf(a[hh], 0.f), zp[0]);
-          zp[1] = fmaf(wv.y, fmaxf(a[hh + 1], 0.f), zp[1]);
-          zp[2] = fmaf(wv.z, fmaxf(a[hh + 2], 0.f), zp[2]);
-          zp[3] = fmaf(wv.w, fmaxf(a[hh + 3], 0.f), zp[3]);
-        }
-        const float z = (zp[0] + zp[1]) + (zp[2] + zp[3]);
         const bool y = (lab >> (s & 31)) & 1u;
-        g = pair_grad(z, y, p.gamma, bce, fl) * inv_n;
-        gsum += g;
+        double b2 = 0.0, f2 = 0.0;
+        g = pair_grad(z, y, p.gamma, b2, f2) * inv_n;
+        if (part == 0) {                                  // one warp per position counts the pair
+          bce += b2;
+          fl += f2;
+          gsum += g;
+        }
       }
       // G' = g 1[a > 0]: the bf16 bit patterns of g's hi and lo parts, masked per column
       const __nv_bfloat16 bh = __float2bfloat16_rn(g);
       const uint32_t hb = __bfloat16_as_ushort(bh);
       const uint32_t lb = __bfloat16_as_ushort(__float2bfloat16_rn(g - __bfloat162float(bh)));
-      const int gb = i & 1;
-      if (i >= 2 && !mbar_wait(&g_free[gb], ((i >> 1) - 1) & 1, abort_flag)) break;
+      const int gb = i % kGBufs;
+      if (i >= kGBufs && !mbar_wait(&g_free[gb], ((i / kGBufs) - 1) & 1, abort_flag)) break;
       uint8_t* ghi = gbuf + gb * 2 * kGBytes;
       uint8_t* glo = ghi + kGBytes;
-      // G' row e, columns j*kH .. +kH-1, MN-major 128-byte swizzle
+      // G' row e, columns wq*32 .. +31, MN-major 128-byte swizzle
       const uint32_t rowoff = (e >> 3) * 1024 + (e & 7) * 128;
 #pragma unroll
-      for (int cidx = 0; cidx < kH / 8; ++cidx) {
+      for (int cidx = 0; cidx < 4; ++cidx) {
         uint32_t wh[4], wl[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -299,7 +317,7 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
           wh[u] = (hb | (hb << 16)) & m;
           wl[u] = (lb | (lb << 16)) & m;
         }
-        const int col = j * kH + cidx * 8;               // first (p, h) column of this 16-byte unit
+        const int col = wq * 32 + cidx * 8;               // first (p, h) column of this 16-byte unit
         const int half = col >> 6, chunk16 = (col & 63) >> 3;
         const uint32_t off = half * kGHalf + rowoff + ((chunk16 ^ (e & 7)) << 4);
         *reinterpret_cast<uint4*>(ghi + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
@@ -312,10 +330,9 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
     const bool got = wait_timed(u_done, 0) && !*abort_flag;
     tc_fence_after();
     if (got) {
-      // U rows: (p, h) = TMEM lane e of this quarter; the Pg warps of a quarter split dI
+      // U rows: (p, h) = TMEM lane e of this quarter; the four warps of a quarter split dI
       float* dst = p.Upart + (static_cast<size_t>(chunk) * p.P * p.H + static_cast<size_t>(group) * kTR + e) * kDI;
-      constexpr int kCols = kDI / kPg >= 32 ? kDI / kPg : 32;
-      for (int c0 = j * kCols; c0 < kDI && c0 < (j + 1) * kCols; c0 += 32) {
+      for (int c0 = wq * 32; c0 < kDI; c0 += 128) {
         float v[32];
         ld32(tU + lane_off + c0, v);
         if (nt == 0) {                       // an empty chunk: no MMA wrote U
@@ -331,12 +348,12 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
         fl += __shfl_xor_sync(0xffffffffu, fl, o);
         gsum += __shfl_xor_sync(0xffffffffu, gsum, o);
       }
-      if (lane == 0) {
+      if (lane == 0 && part == 0) {
         atomicAdd(&p.acc[0], bce);
         atomicAdd(&p.acc[1], fl);
         atomicAdd(&p.acc[2], gsum);
       }
-    } else if (e == 0 && j == 0) {
+    } else if (e == 0 && wq == 0) {
       raise_status(p.status, LSA_ERR_TIMEOUT);
     }
   }
@@ -472,7 +489,8 @@ __global__ void train_loss_kernel(const double* __restrict__ acc, double n, doub
 }
 
 int train_smem(int dI) {
-  return kTStages * (dI / 64) * kTE * 128 + kTR * dI * 2 + 4 * kTR * kTE * 2 + kTR * 4 + 512 + 1024;
+  return kTStages * (dI / 64) * kTE * 128 + kTR * dI * 2 + kGBufs * 2 * kTR * kTE * 2 + kTR * 4 + 2 * 4 * 4 * 32 * 4 +
+         1024 + 1024;
 }
 
 }  // namespace
