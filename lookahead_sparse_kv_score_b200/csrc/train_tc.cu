@@ -165,10 +165,10 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
   const int t0 = (p.ntiles * chunk) / p.chunks, t1 = (p.ntiles * (chunk + 1)) / p.chunks;
   const int nt = t1 - t0;
   if (tid == 0) {
-    for (int i = 0; i < kTStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < kTStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 2); }   // 2 issuers
     for (int b = 0; b < 2; ++b) { mbar_init(&f_full[b], 1); mbar_init(&f_free[b], 32 * kEpiWarps); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&g_full[b], 32 * kEpiWarps); mbar_init(&g_free[b], 1); }
-    mbar_init(u_done, 1);
+    for (int b = 0; b < 2; ++b) { mbar_init(&g_full[b], 32 * kEpiWarps); mbar_init(&g_free[b], 2); }
+    mbar_init(u_done, 2);
     mbar_init(q_bar, 1);
     for (int b = 0; b < 8; ++b) mbar_init(&z_bar[b], 128);
     *abort_flag = 0;
@@ -180,7 +180,8 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tF = tmem, tU = tmem + 256;     // F buffers at columns 0 and 128, U at 256
+  // F buffers at columns 0 and 128; U from the hi parts at 256, from the lo parts at 384
+  const uint32_t tF = tmem, tU = tmem + 256, tUlo = tmem + 384;
 
   if (warp == 0 && lane == 0) {
     // producer: the group's query image once, then the chunk's key tiles
@@ -201,9 +202,13 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
     for (int i = (issued > kTStages ? issued - kTStages : 0); i < issued; ++i)
       wait_timed(&full[i % kTStages], (i / kTStages) & 1);
     wait_timed(q_bar, 0);
-  } else if (warp == 1 && lane == 0) {
-    // MMA issuer: the forward product of tile i+1 goes before the backward product of
-    // tile i, so the tensor pipe works while the epilogue handles tile i.
+  } else if ((warp == 1 || warp == 2) && lane == 0) {
+    // Two MMA issuers (one thread issues a tcgen05.mma every ~90 cycles): warp 1 issues
+    // the forward products, tile i+1's ahead of tile i's backward ones, and the backward
+    // product of the hi parts of G' into U; warp 2 the backward product of the lo parts
+    // into a second accumulator.  A key tile or a G' tile is free once both have
+    // committed.
+    const bool first = warp == 1;
     const uint32_t id_f = t_idesc(kTR, false, false), id_b = t_idesc(kDI, true, true);
     bool ok = mbar_wait(q_bar, 0, abort_flag);
     const uint32_t q0 = smem_u32(qs), g0 = smem_u32(gbuf);
@@ -222,21 +227,20 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
       mma_commit(&f_full[fb]);
       return true;
     };
-    if (ok && nt > 0) ok = forward(0);
+    if (first && ok && nt > 0) ok = forward(0);
     for (int i = 0; ok && i < nt; ++i) {
-      if (i + 1 < nt && !forward(i + 1)) { ok = false; break; }
+      if (first && i + 1 < nt && !forward(i + 1)) { ok = false; break; }
+      const int slot = i % kTStages;
+      if (!first && !mbar_wait(&full[slot], (i / kTStages) & 1, abort_flag)) { ok = false; break; }
       const int gb = i % kGBufs;
       if (!mbar_wait(&g_full[gb], (i / kGBufs) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const int slot = i % kTStages;
       const uint32_t k0 = smem_u32(keys + slot * kKeyBytes);
-      const uint32_t h0 = g0 + gb * 2 * kGBytes, l0 = h0 + kGBytes;
+      const uint32_t a0 = g0 + gb * 2 * kGBytes + (first ? 0 : kGBytes);
 #pragma unroll
-      for (int ks = 0; ks < kTE / 16; ++ks) {
-        const uint64_t bk = desc(k0 + ks * 2048, kBoxBytes, 1024);
-        mma<false>(tU, desc(h0 + ks * 2048, kGHalf, 1024), bk, id_b, (i > 0 || ks > 0) ? 1u : 0u);
-        mma<false>(tU, desc(l0 + ks * 2048, kGHalf, 1024), bk, id_b, 1u);
-      }
+      for (int ks = 0; ks < kTE / 16; ++ks)
+        mma<false>(first ? tU : tUlo, desc(a0 + ks * 2048, kGHalf, 1024), desc(k0 + ks * 2048, kBoxBytes, 1024),
+                   id_b, (i > 0 || ks > 0) ? 1u : 0u);
       mma_commit(&g_free[gb]);
       mma_commit(&empty[slot]);
     }
@@ -333,8 +337,11 @@ train_tc_kernel(const __grid_constant__ CUtensorMap mapK, const TrainParams p) {
       // U rows: (p, h) = TMEM lane e of this quarter; the four warps of a quarter split dI
       float* dst = p.Upart + (static_cast<size_t>(chunk) * p.P * p.H + static_cast<size_t>(group) * kTR + e) * kDI;
       for (int c0 = wq * 32; c0 < kDI; c0 += 128) {
-        float v[32];
+        float v[32], vl[32];
         ld32(tU + lane_off + c0, v);
+        ld32(tUlo + lane_off + c0, vl);
+#pragma unroll
+        for (int u = 0; u < 32; ++u) v[u] += vl[u];
         if (nt == 0) {                       // an empty chunk: no MMA wrote U
 #pragma unroll
           for (int u = 0; u < 32; ++u) v[u] = 0.f;
