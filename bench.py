@@ -699,6 +699,8 @@ def our_arm(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": traffic_per_launch(),
                          "kernel": "score_tc (lsa_index_score, all layers in one launch)",
+                         "note": "the scoring launch, the kernel the metric's roofline is about; the step's "
+                                 "longest kernel is the host-link gather, reported in roofline_gather",
                          "bytes_per_launch": key_bytes, "launch_ms": score_avg, "peak_kind": peak_kind},
             "cpu_baseline": base,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
