@@ -107,6 +107,7 @@ unsigned long long lsa_kernel_launches(void);
  *   LSA_E4M3 with wdt LSA_BF16 (tensor-core path: dI in {64,128,192,256} for bf16 and
  *   {128,256} for e4m3, H a multiple of 32 from 32 to 256).  Other combinations with
  *   H*dI <= 16384 run on the CUDA-core path; anything else is LSA_ERR_UNSUPPORTED.
+ *   B x (layers scored in the call) <= 65535, else LSA_ERR_UNSUPPORTED (split the batch).
  * ---------------------------------------------------------------------------------- */
 size_t lsa_index_score_workspace_bytes(int B, int L, int N, int D, int r, int H, int dI,
                                        int wdt, int kdt);
@@ -131,6 +132,7 @@ int lsa_index_score(int B, int L, int N, int D, int r, int H, int dI,
  * w_out [L][B][H] fp32 are required.  Feed them to lsa_index_score as q_in / w_in to
  * score several times against one query, or to time the scoring on its own.
  * workspace: lsa_index_project_workspace_bytes(...) bytes, 256-byte aligned.
+ * At most 65535 layers per call (layer = -1), else LSA_ERR_UNSUPPORTED.
  * ---------------------------------------------------------------------------------- */
 size_t lsa_index_project_workspace_bytes(int B, int L, int D, int r, int H, int dI, int wdt);
 
@@ -157,7 +159,8 @@ int lsa_select_union(int B, int Nw, const uint32_t* mask_l, uint32_t* U, uint32_
  *     count[b] = popcount(bits[b]);  idx[b][0..] = ascending indices of the set bits.
  *   bits [B][Nw], idx [B][cap] int32, count [B] int32 (the true count, which may
  *   exceed cap; then only the first cap indices are written and *status is raised to
- *   LSA_ERR_CAPACITY).  status: device int32 or NULL.  N >= 0, cap >= 0.
+ *   LSA_ERR_CAPACITY).  status: device int32 or NULL.  N >= 0, cap >= 0.  One launch
+ *   per block of 65535 sequences.
  * ---------------------------------------------------------------------------------- */
 int lsa_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32_t* count,
                 int32_t* status, void* stream);
@@ -246,7 +249,8 @@ int lsa_gather_cold(int B, int N, size_t row_bytes, const void* cold_host,
  *   cold  HOST pointer [B][N][row_bytes], page-locked and mapped (as lsa_gather_cold);
  *   hot   device [B][slots][row_bytes]; slots >= 1; row_bytes a positive multiple of 16.
  *   workspace: lsa_hot_pool_workspace_bytes(B, N, slots) bytes, 256-byte aligned.
- * Six launches; asynchronous on `stream`; calls on one state must not overlap.
+ * Six launches for B <= 4096 (the move step runs per block of 4096 sequences, the slot
+ * keys per block of 65535); asynchronous on `stream`; calls on one state must not overlap.
  * ---------------------------------------------------------------------------------- */
 size_t lsa_hot_pool_state_bytes(int B, int N, int slots);
 size_t lsa_hot_pool_workspace_bytes(int B, int N, int slots);
@@ -274,8 +278,8 @@ int lsa_hot_pool_update(int B, int N, int slots, size_t row_bytes, uint32_t trig
  *   K [N][dI] bf16 (kdt = LSA_BF16, kscale NULL); labels [P][ceil(N/32)] bits.
  *   c_in [P][r] bf16, q_in [P][H][dI] bf16, w_in [P][H] fp32: all three (the forward
  *   projection, e.g. from lsa_index_project) or none (then projected here; P <= 256).
- *   Supported: H in {32, 64, 128}, dI in {64, 128}, P a multiple of 128/H; else
- *   LSA_ERR_UNSUPPORTED.  workspace: lsa_index_train_step_workspace_bytes bytes.
+ *   Supported: H in {32, 64, 128}, dI in {64, 128}, P a multiple of 128/H and at most
+ *   4096; else LSA_ERR_UNSUPPORTED.  workspace: lsa_index_train_step_workspace_bytes bytes.
  *   The product of the keys with the positions' queries (forward) and with the gated
  *   gradients (backward) runs on the tensor cores; a stalled pipeline ends as
  *   LSA_ERR_TIMEOUT in *status.

@@ -30,6 +30,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kInFlight = 8;
 constexpr int kChunk = kThreads * kInFlight * 4;   // 16-byte pieces per block (128 KB)
+constexpr int kSeqPerLaunch = 4096;   // sequences whose move prefix one assign launch holds in shared memory
 
 __global__ void hot_need_kernel(int B, int N, const uint32_t* __restrict__ U, const uint32_t* __restrict__ R,
                                 uint32_t* __restrict__ need) {
@@ -199,18 +200,32 @@ int launch_hot_update(int B, int N, int slots, size_t row_bytes, uint32_t t, con
   if ((rc = check_launch("hot_pool_update/need")) != LSA_OK) return rc;
   // missing rows beyond the pool raise LSA_ERR_CAPACITY here or in the slot select
   if ((rc = launch_compact(B, N, need_bits, slots, need, need_count, status, s)) != LSA_OK) return rc;
-  hot_slot_keys_kernel<<<dim3((slots + 255) / 256, B), 256, 0, s>>>(N, slots, U, t, entry_of, stamp, keys,
-                                                                   kept_count);
-  if ((rc = check_launch("hot_pool_update/slot_keys")) != LSA_OK) return rc;
+  int launches = 0;
+  for (int b0 = 0; b0 < B; b0 += 65535) {   // the sequence index is gridDim.y
+    const int nb = std::min(65535, B - b0);
+    const size_t so = static_cast<size_t>(b0) * slots;
+    hot_slot_keys_kernel<<<dim3((slots + 255) / 256, nb), 256, 0, s>>>(
+        N, slots, U + static_cast<size_t>(b0) * Nw, t, entry_of + so, stamp + so, keys + so, kept_count + b0);
+    ++launches;
+  }
+  if ((rc = check_launch("hot_pool_update/slot_keys", launches)) != LSA_OK) return rc;
   if ((rc = launch_select_keys(B, slots, keys, need_count, kept_count, status, taken, moved, select_ws, s)) != LSA_OK)
     return rc;
   const int vpr = static_cast<int>(row_bytes / 16);
-  const size_t work = static_cast<size_t>(B) * slots * vpr;
-  const unsigned grid = static_cast<unsigned>(std::max<size_t>(1, std::min<size_t>((work + kChunk - 1) / kChunk, 1u << 30)));
-  hot_assign_kernel<<<grid, kThreads, (B + 1) * sizeof(long long), s>>>(
-      B, N, slots, vpr, t, static_cast<const uint4*>(cold_dev), need, taken, moved, static_cast<uint4*>(hot),
-      slot_of, entry_of, stamp, R, status);
-  return check_launch("hot_pool_update/assign");
+  launches = 0;
+  for (int b0 = 0; b0 < B; b0 += kSeqPerLaunch) {
+    const int nb = std::min(kSeqPerLaunch, B - b0);
+    const size_t so = static_cast<size_t>(b0) * slots, no = static_cast<size_t>(b0) * N;
+    const size_t work = static_cast<size_t>(nb) * slots * vpr;   // upper bound on this launch's 16-byte moves
+    const unsigned grid =
+        static_cast<unsigned>(std::max<size_t>(1, std::min<size_t>((work + kChunk - 1) / kChunk, 1u << 30)));
+    hot_assign_kernel<<<grid, kThreads, (nb + 1) * sizeof(long long), s>>>(
+        nb, N, slots, vpr, t, static_cast<const uint4*>(cold_dev) + no * vpr, need + so, taken + so, moved + b0,
+        static_cast<uint4*>(hot) + so * vpr, slot_of + no, entry_of + so, stamp + so,
+        R + static_cast<size_t>(b0) * Nw, status);
+    ++launches;
+  }
+  return check_launch("hot_pool_update/assign", launches);
 }
 
 }  // namespace lsa

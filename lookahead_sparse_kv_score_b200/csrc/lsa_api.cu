@@ -110,6 +110,8 @@ int lsa_index_project(int B, int L, int D, int r, int H, int dI, int wdt, const 
   if (wdt != LSA_F32 && wdt != LSA_BF16) return fail(LSA_ERR_UNSUPPORTED, "index_project: wdt %d", wdt);
   if (layer < -1 || layer >= L) return fail(LSA_ERR_INVALID_ARG, "index_project: layer %d of %d", layer, L);
   if (B == 0 || L == 0) return LSA_OK;
+  if (layer < 0 && L > 65535)
+    return fail(LSA_ERR_UNSUPPORTED, "index_project: %d layers in one call (at most 65535)", L);
   if (!h || !W_down || !W_up || !W_w || !q_out || !w_out)
     return fail(LSA_ERR_INVALID_ARG, "index_project: null pointer");
   const void* ptrs[] = {h, W_down, W_up, W_w, q_out, w_out};
@@ -159,6 +161,10 @@ int lsa_index_score(int B, int L, int N, int D, int r, int H, int dI,
   if (!valid_dtype(kdt)) return fail(LSA_ERR_UNSUPPORTED, "index_score: kdt %d", kdt);
   if (layer < -1 || layer >= L) return fail(LSA_ERR_INVALID_ARG, "index_score: layer %d of %d", layer, L);
   if (B == 0 || L == 0) return LSA_OK;
+  if (static_cast<long long>(B) * (layer < 0 ? L : 1) > 65535)
+    return fail(LSA_ERR_UNSUPPORTED,
+                "index_score: B x scored layers = %lld (at most 65535 sequence-layer pairs per call)",
+                static_cast<long long>(B) * (layer < 0 ? L : 1));
   if (w_in && !q_in) return fail(LSA_ERR_INVALID_ARG, "index_score: w_in needs q_in");
   const bool need_q = q_in == nullptr, need_w = w_in == nullptr;
   if (need_q && (D <= 0 || r <= 0 || !h || !W_down || !W_up))
@@ -384,7 +390,7 @@ int lsa_index_train_step(int P, int N, int D, int r, int H, int dI, int wdt,
   if (!train_supported(P, H, dI, wdt, kdt) || kscale != nullptr || D % 8 != 0 || r % 8 != 0)
     return fail(LSA_ERR_UNSUPPORTED,
                 "index_train_step: needs bf16 weights and keys, H in {32, 64, 128}, dI in {64, 128}, P a multiple "
-                "of 128/H, D and r multiples of 8");
+                "of 128/H and at most 4096, D and r multiples of 8");
   const bool given = c_in || q_in || w_in;
   if (given && !(c_in && q_in && w_in))
     return fail(LSA_ERR_INVALID_ARG, "index_train_step: give all of c_in, q_in, w_in or none");

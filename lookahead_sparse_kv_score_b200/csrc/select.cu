@@ -337,9 +337,16 @@ int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, in
                    int32_t* status, cudaStream_t s) {
   if (B == 0) return LSA_OK;
   const int Nw = (N + 31) / 32;
-  const dim3 grid(std::max(1, (Nw + kCompactWords - 1) / kCompactWords), B);
-  compact_kernel<<<grid, kCompactThreads, 0, s>>>(bits, Nw, cap, idx, count, status);
-  return check_launch("compact");
+  constexpr int kSeqPerLaunch = 65535;   // the sequence index is gridDim.y
+  int launches = 0;
+  for (int b0 = 0; b0 < B; b0 += kSeqPerLaunch) {
+    const int nb = std::min(kSeqPerLaunch, B - b0);
+    const dim3 grid(std::max(1, (Nw + kCompactWords - 1) / kCompactWords), nb);
+    compact_kernel<<<grid, kCompactThreads, 0, s>>>(bits + static_cast<size_t>(b0) * Nw, Nw, cap,
+                                                    idx + static_cast<size_t>(b0) * cap, count + b0, status);
+    ++launches;
+  }
+  return check_launch("compact", launches);
 }
 
 namespace {

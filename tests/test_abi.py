@@ -66,6 +66,16 @@ def test_host_side_argument_errors(lib):
     rc = lib.lsa_index_score(*args, 0, 256, 256, 256, 256, 256, 0, 256, None, 0,
                              None, None, None, None, 256, None, None, None, None, 0, None)
     assert rc == lsa.LSA_ERR_NOMEM                  # no workspace
+    # size limits: sequence x layer pairs, layers per call, training positions
+    rc = lib.lsa_index_score(30000, 3, 128, 64, 16, 8, 64, 0, 256, 256, 256, 256, 256, 0, 256, None, -1,
+                             None, None, None, None, 256, None, None, None, None, 0, None)
+    assert rc == lsa.LSA_ERR_UNSUPPORTED and b"65535" in lib.lsa_last_error()
+    rc = lib.lsa_index_project(1, 70000, 64, 16, 8, 64, 0, 256, 256, 256, 256, -1, 256, 256, None, 0, None)
+    assert rc == lsa.LSA_ERR_UNSUPPORTED and b"65535" in lib.lsa_last_error()
+    rc = lib.lsa_index_train_step(4097, 256, 64, 16, 128, 64, 1, 256, 256, 256, 256, ctypes.c_float(0.0), 1, 256,
+                                  None, 256, ctypes.c_float(2.0), 256, 256, 256, None, 256, 256, 256, None, None,
+                                  None, 0, None)
+    assert rc == lsa.LSA_ERR_UNSUPPORTED and b"at most 4096" in lib.lsa_last_error()
     upd = lib.lsa_hot_pool_update
     assert upd(1, 64, 8, 1152, 0, 256, 256, 256, 256, None, None, 256, 1 << 20, None) == lsa.LSA_ERR_INVALID_ARG
     assert b"trigger" in lib.lsa_last_error()

@@ -118,3 +118,18 @@ def test_hot_pool_full_size_sequences():
         sets = [drift(g, N, sets[b], int(g.integers(60000, 80000)), keep=0.8) for b in range(B)]
         exp = p.update(sets, t)
         assert p.check(exp) == 0
+
+
+def test_hot_pool_more_sequences_than_one_launch():
+    """4,500 sequences: the move step runs in blocks of 4,096 sequences; one sequence of
+    the second block overflows the pool on trigger 2 and must move nothing."""
+    g = np.random.default_rng(6)
+    B, N, slots, R = 4500, 64, 16, 16
+    p = Pool(B, N, slots, R, 7)
+    sets = [set() for _ in range(B)]
+    for t in range(1, 4):
+        sets = [drift(g, N, sets[b], int(g.integers(0, slots + 1)), keep=0.6) for b in range(B)]
+        if t == 2:
+            sets[4400] = set(range(slots + 3))
+        exp = p.update(sets, t)
+        assert p.check(exp) == (lsa.LSA_ERR_CAPACITY if t == 2 else 0), t

@@ -61,6 +61,27 @@ def test_compact_exact(N, p):
         assert np.array_equal(idx[b, : len(e)].cpu().numpy(), e)
 
 
+@pytest.mark.parametrize("N", [40, 100])
+def test_compact_more_sequences_than_one_launch(N):
+    """70,000 sequences: more than one launch's 65,535 (the sequence is the grid's y
+    index), with word rows that are and are not 16-byte multiples."""
+    g = np.random.default_rng(N + 7)
+    B, cap = 70000, N
+    m = g.random((B, N)) < 0.3
+    idx = torch.full((B, cap), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(B, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lsa.lsa_compact(B, N, bits_tensor(m), cap, idx, cnt, st)
+    torch.cuda.synchronize()
+    assert int(st) == 0
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(B):
+        e = O.compact(m[b])
+        assert cnt[b] == len(e), b
+        assert np.array_equal(idx[b, : len(e)], e), b
+        assert (idx[b, len(e):] == -7).all(), b
+
+
 def test_compact_capacity_overflow_sets_status():
     g = np.random.default_rng(1)
     B, N, cap = 2, 5000, 100
