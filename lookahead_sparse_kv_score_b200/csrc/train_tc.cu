@@ -411,42 +411,95 @@ __global__ void train_finish_kernel(const float* __restrict__ Upart, int chunks,
   }
 }
 
-// out[m][n] = sum_p X[p][m] Y[p][n]  (X bf16 [P][M], Y fp32 [P][Nn]); 64 x 64 tiles.
+// out[m][n] = sum_p X[p][m] Y[p][n]  (X bf16 [P][M], Y fp32 [P][Nn]; M % 8 == 0, Nn % 4 == 0,
+// all three pointers 16-byte aligned).  128 x 128 tiles; a thread owns 8 x 8 outputs, rows
+// ty*4 + {0..3} and 64 + ty*4 + {0..3} and columns likewise from tx, so that every
+// shared-memory read is a 16-byte vector; the positions p are staged 16 at a time.  One
+// launch can serve a second product with the same X: column tiles from nbx1 on belong to
+// (Y2, Nn2, out2).
+constexpr int kOT = 128;   // tile edge
+constexpr int kOK = 16;    // positions per stage
+
 __global__ void __launch_bounds__(256)
 outer_acc_kernel(const __nv_bfloat16* __restrict__ X, int M, const float* __restrict__ Y, int Nn, int P,
-                 float* __restrict__ out) {
-  __shared__ float xs[16][64], ys[16][64];
-  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+                 float* __restrict__ out, int nbx1 = 0x7fffffff, const float* __restrict__ Y2 = nullptr,
+                 int Nn2 = 0, float* __restrict__ out2 = nullptr) {
+  __shared__ __align__(16) float xs[kOK][kOT];
+  __shared__ __align__(16) float ys[kOK][kOT];
+  int bx = blockIdx.x;
+  if (bx >= nbx1) {
+    bx -= nbx1;
+    Y = Y2;
+    Nn = Nn2;
+    out = out2;
+  }
+  const int m0 = blockIdx.y * kOT, n0 = bx * kOT;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4] = {};
-  for (int p0 = 0; p0 < P; p0 += 16) {
-    for (int i = threadIdx.x; i < 16 * 64; i += 256) {
-      const int pp = p0 + i / 64, c = i % 64;
-      xs[i / 64][c] = (pp < P && m0 + c < M) ? __bfloat162float(X[static_cast<size_t>(pp) * M + m0 + c]) : 0.f;
-      ys[i / 64][c] = (pp < P && n0 + c < Nn) ? Y[static_cast<size_t>(pp) * Nn + n0 + c] : 0.f;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  for (int p0 = 0; p0 < P; p0 += kOK) {
+    {   // X: 16 positions x 128 values, one 16-byte load (8 bf16) per thread
+      const int kk = threadIdx.x >> 4, c = (threadIdx.x & 15) * 8;
+      const int pp = p0 + kk, m = m0 + c;
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = 0.f;
+      if (pp < P && m < M) {   // M % 8 == 0: the eight values are all in range
+        const uint4 raw = *reinterpret_cast<const uint4*>(X + static_cast<size_t>(pp) * M + m);
+        const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[2 * e] = __uint_as_float(wv[e] << 16);            // bf16 -> fp32 is exact
+          v[2 * e + 1] = __uint_as_float(wv[e] & 0xffff0000u);
+        }
+      }
+      *reinterpret_cast<float4*>(&xs[kk][c]) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4*>(&xs[kk][c + 4]) = make_float4(v[4], v[5], v[6], v[7]);
+    }
+    for (int t = threadIdx.x; t < kOK * kOT / 4; t += 256) {   // Y: two float4 per thread
+      const int kk = t / (kOT / 4), c = (t % (kOT / 4)) * 4;
+      const int pp = p0 + kk, n = n0 + c;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (pp < P && n < Nn) v = *reinterpret_cast<const float4*>(Y + static_cast<size_t>(pp) * Nn + n);
+      *reinterpret_cast<float4*>(&ys[kk][c]) = v;
     }
     __syncthreads();
 #pragma unroll
-    for (int k = 0; k < 16; ++k)
+    for (int k = 0; k < kOK; ++k) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&xs[k][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&xs[k][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&ys[k][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&ys[k][64 + tx * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(xs[k][ty * 4 + a], ys[k][tx * 4 + b], acc[a][b]);
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
     __syncthreads();
   }
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int i = 0; i < 8; ++i) {
+    const int m = m0 + (i >> 2) * 64 + ty * 4 + (i & 3);
+    if (m >= M) continue;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int m = m0 + ty * 4 + a, n = n0 + tx * 4 + b;
-      if (m < M && n < Nn) out[static_cast<size_t>(m) * Nn + n] = acc[a][b];
+    for (int h = 0; h < 2; ++h) {
+      const int n = n0 + h * 64 + tx * 4;   // Nn % 4 == 0: n < Nn covers all four
+      if (n < Nn)
+        *reinterpret_cast<float4*>(out + static_cast<size_t>(m) * Nn + n) =
+            make_float4(acc[i][4 * h], acc[i][4 * h + 1], acc[i][4 * h + 2], acc[i][4 * h + 3]);
     }
+  }
 }
 
 // dc[p][i] = sum_j dq[p][j] W_up[i][j]  (W_up bf16 [r][J]).  Tiles of 64 positions x 64
 // rows i, the reduction split into kDcSplits slices written as partial sums and added in
 // a fixed order by dc_reduce_kernel.
-constexpr int kDcSplits = 16;
+constexpr int kDcSplits = 64;
 
 __global__ void __launch_bounds__(256)
 dc_kernel(const float* __restrict__ dq, int P, int J, const __nv_bfloat16* __restrict__ Wu, int r,
@@ -579,17 +632,18 @@ int launch_train(const TrainArgs& a, cudaStream_t st) {
   // projection gradients
   const __nv_bfloat16* c = static_cast<const __nv_bfloat16*>(a.c);
   const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(a.h);
-  outer_acc_kernel<<<dim3(static_cast<unsigned>((HD + 63) / 64), (a.r + 63) / 64), 256, 0, st>>>(
+  outer_acc_kernel<<<dim3(static_cast<unsigned>((HD + kOT - 1) / kOT), (a.r + kOT - 1) / kOT), 256, 0, st>>>(
       c, a.r, dq, static_cast<int>(HD), a.P, a.dW_up);
   float* dcpart = reinterpret_cast<float*>(ws + lay.dcpart);
   dc_kernel<<<dim3((a.r + 63) / 64, (a.P + 63) / 64, kDcSplits), 256, 0, st>>>(
       dq, a.P, static_cast<int>(HD), static_cast<const __nv_bfloat16*>(a.W_up), a.r, dcpart);
   const size_t ndc = static_cast<size_t>(a.P) * a.r;
   dc_reduce_kernel<<<static_cast<unsigned>(std::min<size_t>((ndc + 255) / 256, 1184)), 256, 0, st>>>(dcpart, ndc, dc);
-  outer_acc_kernel<<<dim3((a.r + 63) / 64, (a.D + 63) / 64), 256, 0, st>>>(h, a.D, dc, a.r, a.P, a.dW_down);
-  outer_acc_kernel<<<dim3((a.H + 63) / 64, (a.D + 63) / 64), 256, 0, st>>>(h, a.D, dw, a.H, a.P, a.dW_w);
+  const int nb_r = (a.r + kOT - 1) / kOT, nb_h = (a.H + kOT - 1) / kOT;   // dW_down and dW_w in one launch
+  outer_acc_kernel<<<dim3(nb_r + nb_h, (a.D + kOT - 1) / kOT), 256, 0, st>>>(h, a.D, dc, a.r, a.P, a.dW_down, nb_r,
+                                                                           dw, a.H, a.dW_w);
   train_loss_kernel<<<1, 1, 0, st>>>(acc, static_cast<double>(a.P) * a.N, a.loss, a.dbias);
-  return check_launch("train/projection gradients", 6);
+  return check_launch("train/projection gradients", 5);
 }
 
 }  // namespace lsa
