@@ -46,11 +46,15 @@ def dtype_code(t) -> int:
 
 
 def _p(t):
-    """Raw pointer of a tensor (None -> NULL); plain ints pass through."""
+    """Raw pointer of a tensor (None -> NULL); plain ints pass through.  The library reads
+    and writes every array densely in the layout the header gives, so a strided view is
+    refused here rather than read as if it were dense."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_contiguous():
+        raise ValueError(f"tensor of shape {tuple(t.shape)} with strides {t.stride()} is not contiguous")
     return t.data_ptr()
 
 

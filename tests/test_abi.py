@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import lookahead_sparse_kv_score_b200 as lsa
 from lookahead_sparse_kv_score_b200 import _abi, build
@@ -85,6 +86,16 @@ def test_host_side_argument_errors(lib):
     assert upd(1, 64, 8, 1152, 1, 256, 256, 256, 264, None, None, 256, 1 << 20, None) == lsa.LSA_ERR_INVALID_ARG
     assert upd(1, 64, 8, 1152, 1, 256, 256, 256, 256, None, None, 256, 16, None) == lsa.LSA_ERR_NOMEM
     assert lib.lsa_hot_pool_reset(1, 64, 8, None, None) == lsa.LSA_ERR_INVALID_ARG
+
+
+def test_binding_refuses_strided_views(lib):
+    # marshalling only, but a transposed view would be read as dense: refused before the call
+    bits = torch.zeros(2, 4, dtype=torch.int32)
+    with pytest.raises(ValueError, match="not contiguous"):
+        lsa.lsa_compact(4, 64, bits.t(), 8, torch.zeros(4, 8, dtype=torch.int32), torch.zeros(4, dtype=torch.int32),
+                        stream=0)
+    with pytest.raises(lsa.LsaError):       # a dense tensor reaches the library (which refuses the null list)
+        lsa.lsa_compact(4, 64, bits.reshape(4, 2), 8, None, torch.zeros(4, dtype=torch.int32), stream=0)
 
 
 def test_hot_pool_layout():
