@@ -157,10 +157,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap mapW1, const __grid_constant_
   } else if (warp == 1 && lane == 0) {
     // MMA issuer
     const uint32_t idesc = pj_idesc(p.npad);
-    bool ok = true;
     for (int st = 0; st < nst; ++st) {
       const int slot = st % kPStages;
-      if (!mbar_wait(&full[slot], (st / kPStages) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&full[slot], (st / kPStages) & 1, abort_flag)) break;
       tc_fence_after();
       const uint32_t a0 = smem_u32(sm + slot * stage_bytes), x0 = a0 + kABytes;
 #pragma unroll
@@ -168,7 +167,6 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap mapW1, const __grid_constant_
         mma<false>(tmem, desc_mn(a0 + ks * 2048), desc_k(x0 + ks * 32), idesc, (st > 0 || ks > 0) ? 1u : 0u);
       mma_commit(&empty[slot]);
     }
-    (void)ok;
     // also after an abort: the commit arrives once the MMAs already issued are done
     mma_commit(accum);
   }
