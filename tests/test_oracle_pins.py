@@ -70,6 +70,21 @@ def test_worked_example_projection_and_score(bf16):
     np.testing.assert_allclose(O.sigmoid(z), 1 / (1 + np.exp(-np.array(e["z"]))), rtol=0, atol=0)
 
 
+def test_projection_rounds_c_before_the_up_projection():
+    """bf16 boundaries: c = h W_down is rounded to bf16 before q = c W_up.  With
+    c = [1 + 3 * 2^-9, 1] (0.75 of a bf16 ulp above 1: rounds up to 1 + 2^-7) and
+    W_up = [1, -1]^T, q = RNE(1 + 2^-7 - 1) = 2^-7; without the rounding of c it would be
+    3 * 2^-9.  In fp32 mode nothing is rounded."""
+    h = np.array([1.0, 0.0])
+    W_down = np.array([[1.0 + 3 * 2.0 ** -9, 1.0], [0.0, 0.0]])
+    W_up = np.array([[1.0], [-1.0]])
+    W_w = np.array([[2.0], [0.0]])
+    q, w = O.project_query(h, W_down, W_up, W_w, 1, 1, True)
+    assert q.tolist() == [[2.0 ** -7]] and w.tolist() == [2.0]
+    q, w = O.project_query(h, W_down, W_up, W_w, 1, 1, False)
+    assert q.tolist() == [[3 * 2.0 ** -9]]
+
+
 def test_worked_example_through_raw_buffers():
     """The same example through the raw-storage path (bf16 bit patterns)."""
     ex = _worked()
@@ -225,6 +240,11 @@ def test_fetched_key_is_max_over_marking_layers():
     z = np.array([[1.0, -2.0, 0.5], [3.0, -1.0, -0.2], [-5.0, 0.0, 0.7]])
     m = z >= 0
     assert O.fetched_key(z, m).tolist() == [3.0, 0.0, 0.7]
+    # the key follows the marks, not the largest logit: a layer that did not mark the
+    # entry does not count even where its logit is larger; an unmarked entry has no key
+    z = np.array([[5.0, 1.0, 2.0], [7.0, 2.0, 3.0]])
+    m = np.array([[True, True, False], [False, True, False]])
+    assert O.fetched_key(z, m).tolist() == [5.0, 2.0, -np.inf]
 
 
 # ----------------------------------------------------------------------------- nucleus / vote
@@ -246,6 +266,15 @@ def test_nucleus_all_equal_logits_exact_count():
     # every pi = 2**-17 exactly; mass before entry i is i * 2**-17 < 0.6 <=> i <= 78643
     assert int(sel.sum()) == math.ceil(0.6 * n) == 78644
     assert sel[:78644].all() and not sel[78644:].any()
+
+
+def test_nucleus_stops_where_the_mass_reaches_top_p_exactly():
+    # four equal logits: pi = 1/4 each (exact), masses before: 0, 1/4, 1/2, 3/4.  The
+    # smallest prefix with mass >= 1/2 is the first two entries; the third has mass 1/2
+    # before it, not below 1/2.
+    assert O.nucleus(np.zeros(4), 0.5).tolist() == [True, True, False, False]
+    assert O.nucleus(np.zeros(8), 0.25).tolist() == [True, True] + [False] * 6
+    assert O.nucleus(np.zeros(8), 0.2500001).tolist() == [True, True, True] + [False] * 5
 
 
 def test_nucleus_one_hot_and_two_entry_closed_form():
@@ -315,3 +344,7 @@ def test_bias_for_fraction_counts():
     z = g.standard_normal(1000) * 30
     b = O.bias_for_fraction(z, 0.1)
     assert int(((z + b) >= 0).sum()) == 100
+    # the cut is the midpoint of the straddling order statistics: no entry sits on it
+    zs = np.sort(z)
+    assert -b == (zs[899] + zs[900]) / 2 and zs[899] < -b < zs[900]
+    assert not np.any(z + b == 0)

@@ -52,6 +52,23 @@ def test_dloss_dz_closed_form_at_half():
     assert d[1] == pytest.approx(0.5 + 0.125 + ln2 / 4, rel=1e-14)
 
 
+def test_dloss_dz_zero_where_the_clamp_holds():
+    """Beyond |z| = ln(2^20 - 1) ~ 13.863 the clamped probability is constant in z, so the
+    loss is flat there (its central differences vanish) and dJ/dz is exactly zero, for
+    either label; just inside the clamp it is not."""
+    zc = np.log(2.0 ** 20 - 1)
+    for z0 in (-40.0, -20.0, -14.0, 14.0, 20.0, 40.0):
+        for y in (0.0, 1.0):
+            z, yy = np.array([z0]), np.array([y])
+            jp = sum(O.bce_focal(O.sigmoid(z + 1e-3), yy, 2.0))
+            jm = sum(O.bce_focal(O.sigmoid(z - 1e-3), yy, 2.0))
+            assert jp == jm, (z0, y)
+            assert T.dloss_dz(z, yy, 2.0, 1)[0] == 0.0, (z0, y)
+    for z0 in (-13.0, 13.0):
+        assert abs(z0) < zc
+        assert T.dloss_dz(np.array([z0, z0]), np.array([0.0, 1.0]), 2.0, 1).tolist().count(0.0) == 0
+
+
 def test_dloss_dz_matches_differences_of_bce_focal():
     g = np.random.default_rng(3)
     z = g.standard_normal(50) * 4
