@@ -358,7 +358,38 @@ def hot_pool_capacity_on_need(self, U, t, cold=None, hot=None):
     return _hot_update(self, U, t, cold, hot)
 
 
+from oracle import step as OS  # noqa: E402  (the step-level mistakes below patch it)
+
+_select = OS.select
+
+
+def step_topk_over_last_new_set(marks_by_layer, z_by_layer, k):
+    out = _select(marks_by_layer, z_by_layer, k)
+    out["topk"] = O.topk_in_fetched(out["idx_new"][-1], out["key"], k)
+    return out
+
+
+def step_scale_ignored(K_raw, kscale, kdtype):
+    return OS.decode(K_raw, kdtype)
+
+
+def step_scale_divides(K_raw, kscale, kdtype):
+    K = OS.decode(K_raw, kdtype)
+    if kdtype == "e4m3":
+        K = K / np.asarray(kscale, dtype=np.float32).astype(np.float64)[:, None]
+    return K
+
+
+def step_projection_without_bf16_boundaries(h_raw, Wd_raw, Wu_raw, Ww_raw, H, dI, wdtype):
+    return O.project_query(OS.decode(h_raw, wdtype), OS.decode(Wd_raw, wdtype), OS.decode(Wu_raw, wdtype),
+                           OS.decode(Ww_raw, wdtype), H, dI, bf16_boundaries=False)
+
+
 MISTAKES = {
+    "step top-k over the last layer's new set": (OS, "select", step_topk_over_last_new_set),
+    "step e4m3 scale ignored": (OS, "decode_keys", step_scale_ignored),
+    "step e4m3 scale divides": (OS, "decode_keys", step_scale_divides),
+    "step projection without bf16 boundaries": (OS, "project", step_projection_without_bf16_boundaries),
     "sigmoid with the wrong sign": (O, "sigmoid", sigmoid_wrong_sign),
     "bit unpacking shifted by one": (O, "unpack_bits", unpack_shifted),
     "score scaled by 1/sqrt(dI)": (O, "head_fused_logits", score_scaled),

@@ -83,6 +83,17 @@ def test_projection_rounds_c_before_the_up_projection():
     assert q.tolist() == [[2.0 ** -7]] and w.tolist() == [2.0]
     q, w = O.project_query(h, W_down, W_up, W_w, 1, 1, False)
     assert q.tolist() == [[3 * 2.0 ** -9]]
+    # the same through raw storage: a bf16 model gets the bf16 boundaries, an fp32 model
+    # none (h = [1, 1] and W_down = [[1, 1], [3 * 2^-9, 0]] are bf16 values with the same c)
+    h2 = np.array([1.0, 1.0])
+    Wd2 = np.array([[1.0, 1.0], [3 * 2.0 ** -9, 0.0]])
+    def bits(a):
+        return torch.tensor(a, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    q, w = OS.project(bits(h2), bits(Wd2), bits(W_up), bits(W_w), 1, 1, "bf16")
+    assert q.tolist() == [[2.0 ** -7]] and w.tolist() == [2.0]
+    f32 = lambda a: np.asarray(a, dtype=np.float32)
+    q, w = OS.project(f32(h2), f32(Wd2), f32(W_up), f32(W_w), 1, 1, "f32")
+    assert q.tolist() == [[3 * 2.0 ** -9]]
 
 
 def test_worked_example_through_raw_buffers():
@@ -245,6 +256,29 @@ def test_fetched_key_is_max_over_marking_layers():
     z = np.array([[5.0, 1.0, 2.0], [7.0, 2.0, 3.0]])
     m = np.array([[True, True, False], [False, True, False]])
     assert O.fetched_key(z, m).tolist() == [5.0, 2.0, -np.inf]
+
+
+def test_step_select_composes_the_set_operations():
+    """The step's selection from per-layer marks and logits, by brute force: the top-k
+    runs over the union of all layers (not one layer's new set), keyed by the largest
+    logit among the marking layers."""
+    g = np.random.default_rng(21)
+    for _ in range(30):
+        n, k = int(g.integers(1, 50)), int(g.integers(1, 12))
+        z = g.standard_normal((3, n)).round(1)           # coarse values: ties happen
+        marks = z >= 0.3
+        out = OS.select(list(marks), z, k)
+        union = [s for s in range(n) if marks[:, s].any()]
+        assert out["idx_union"].tolist() == union
+        seen = set()
+        for l in range(3):
+            new = [s for s in range(n) if marks[l, s] and s not in seen]
+            assert out["idx_new"][l].tolist() == new
+            seen |= set(new)
+        key = {s: max(z[l, s] for l in range(3) if marks[l, s]) for s in union}
+        top = sorted(s for s in union
+                     if sum(1 for t in union if key[t] > key[s] or (key[t] == key[s] and t < s)) < k)
+        assert out["topk"].tolist() == top
 
 
 # ----------------------------------------------------------------------------- nucleus / vote
