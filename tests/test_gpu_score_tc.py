@@ -77,8 +77,8 @@ def _full_size_check(name, samples_per_unit=192, seqs=None):
     """Full-size workload, all layers in one launch as the benchmark runs it.
     (1) with the oracle's query: sampled logits within the tolerance, sampled mask bits
         exact outside the band; (2) with the projection inside the call: every query
-        element within one bf16 ulp of the oracle's and the mask consistent with the
-        logits on every entry."""
+        element within the rigorous fp32 bound of the oracle's (q_allowed) and the mask
+        consistent with the logits on every entry."""
     w = W.WORKLOADS[name]
     inp = C.make_inputs(w)
     orc = C.OracleCache(inp)
