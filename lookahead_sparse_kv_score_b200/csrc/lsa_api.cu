@@ -104,6 +104,7 @@ size_t lsa_index_project_workspace_bytes(int B, int L, int D, int r, int H, int 
 int lsa_index_project(int B, int L, int D, int r, int H, int dI, int wdt, const void* h,
                       const void* W_down, const void* W_up, const void* W_w, int layer,
                       void* q_out, float* w_out, void* workspace, size_t workspace_bytes, void* stream) {
+  const CallRange range("lsa_index_project");
   g_err[0] = 0;
   if (B < 0 || L < 0 || D <= 0 || r <= 0 || H <= 0 || dI <= 0)
     return fail(LSA_ERR_INVALID_ARG, "index_project: bad size");
@@ -154,6 +155,7 @@ int lsa_index_score(int B, int L, int N, int D, int r, int H, int dI,
                     uint32_t* mask, float* logit, float* score, int32_t* status,
                     void* workspace, size_t workspace_bytes,
                     void* stream) {
+  const CallRange range("lsa_index_score");
   g_err[0] = 0;
   if (B < 0 || L < 0 || N < 0 || D < 0 || r < 0 || H <= 0 || dI <= 0)
     return fail(LSA_ERR_INVALID_ARG, "index_score: negative size or H/dI < 1");
@@ -229,6 +231,7 @@ int lsa_index_score(int B, int L, int N, int D, int r, int H, int dI,
 
 int lsa_select_union(int B, int Nw, const uint32_t* mask_l, uint32_t* U, uint32_t* new_l,
                      void* stream) {
+  const CallRange range("lsa_select_union");
   g_err[0] = 0;
   if (B < 0 || Nw < 0) return fail(LSA_ERR_INVALID_ARG, "select_union: negative size");
   if (static_cast<size_t>(B) * Nw == 0) return LSA_OK;
@@ -240,6 +243,7 @@ int lsa_select_union(int B, int Nw, const uint32_t* mask_l, uint32_t* U, uint32_
 
 int lsa_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32_t* count,
                 int32_t* status, void* stream) {
+  const CallRange range("lsa_compact");
   g_err[0] = 0;
   if (B < 0 || N < 0 || cap < 0) return fail(LSA_ERR_INVALID_ARG, "compact: negative size");
   if (B == 0) return LSA_OK;
@@ -258,6 +262,7 @@ size_t lsa_topk_workspace_bytes(int B, int cap) {
 int lsa_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
              const float* logit, int32_t* topk, int32_t* topk_count,
              void* workspace, size_t workspace_bytes, void* stream) {
+  const CallRange range("lsa_topk");
   g_err[0] = 0;
   if (B < 0 || L <= 0 || N < 0 || k < 0 || cap < 0)
     return fail(LSA_ERR_INVALID_ARG, "topk: bad size (L must be >= 1)");
@@ -275,6 +280,7 @@ int lsa_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int3
 int lsa_gather_cold(int B, int N, size_t row_bytes, const void* cold_host,
                     const int32_t* idx, const int32_t* count, int cap, void* hot,
                     int32_t* status, void* stream) {
+  const CallRange range("lsa_gather_cold");
   g_err[0] = 0;
   if (B < 0 || N < 0 || cap < 0) return fail(LSA_ERR_INVALID_ARG, "gather_cold: negative size");
   if (row_bytes == 0 || row_bytes % 16 != 0)
@@ -316,6 +322,7 @@ int lsa_hot_pool_layout(int B, int N, int slots, size_t offsets[4]) {
 }
 
 int lsa_hot_pool_reset(int B, int N, int slots, void* state, void* stream) {
+  const CallRange range("lsa_hot_pool_reset");
   g_err[0] = 0;
   if (!hot_sizes_ok(B, N, slots)) return fail(LSA_ERR_INVALID_ARG, "hot_pool_reset: negative size");
   if (!state) return fail(LSA_ERR_INVALID_ARG, "hot_pool_reset: null pointer");
@@ -338,6 +345,7 @@ int lsa_hot_pool_update(int B, int N, int slots, size_t row_bytes, uint32_t trig
                         const uint32_t* U, const void* cold_host, void* hot, void* state,
                         int32_t* moved, int32_t* status,
                         void* workspace, size_t workspace_bytes, void* stream) {
+  const CallRange range("lsa_hot_pool_update");
   g_err[0] = 0;
   if (!hot_sizes_ok(B, N, slots)) return fail(LSA_ERR_INVALID_ARG, "hot_pool_update: negative size");
   if (row_bytes == 0 || row_bytes % 16 != 0)
@@ -384,6 +392,7 @@ int lsa_index_train_step(int P, int N, int D, int r, int H, int dI, int wdt,
                          const void* c_in, const void* q_in, const float* w_in,
                          double* loss, float* dW_down, float* dW_up, float* dW_w, double* dbias,
                          int32_t* status, void* workspace, size_t workspace_bytes, void* stream) {
+  const CallRange range("lsa_index_train_step");
   g_err[0] = 0;
   if (P <= 0 || N < 0 || D <= 0 || r <= 0 || H <= 0 || dI <= 0)
     return fail(LSA_ERR_INVALID_ARG, "index_train_step: bad size");
@@ -436,6 +445,7 @@ int lsa_index_train_step(int P, int N, int D, int r, int H, int dI, int wdt,
 }
 
 int lsa_check_bounded_wait(uint32_t limit_us, int32_t* status, void* stream) {
+  const CallRange range("lsa_check_bounded_wait");
   g_err[0] = 0;
   if (!status) return fail(LSA_ERR_INVALID_ARG, "check_bounded_wait: null status");
   if (limit_us == 0 || limit_us > 2000000u)
@@ -455,6 +465,7 @@ int lsa_vote_labels(int L, int P, int N, const float* logits, float top_p, int t
                     uint32_t* golden, uint8_t* counts,
                     const float* scores, float gamma, double* loss,
                     void* workspace, size_t workspace_bytes, void* stream) {
+  const CallRange range("lsa_vote_labels");
   g_err[0] = 0;
   if (L < 0 || P < 0 || N < 0) return fail(LSA_ERR_INVALID_ARG, "vote_labels: negative size");
   if (L > 255) return fail(LSA_ERR_UNSUPPORTED, "vote_labels: L = %d layers (at most 255: counts are bytes)", L);

@@ -7,9 +7,21 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "lsa.h"
 
 namespace lsa {
+
+// One NVTX range per library call, named after the call, so that a profiler's timeline
+// (or an ncu --nvtx filter) shows which call launched which kernels.  With no tool
+// attached a range costs a few nanoseconds.
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 // ------------------------------------------------------------------ host-side errors
 int fail(int code, const char* fmt, ...);   // records the message, returns code

@@ -52,6 +52,7 @@ int scratch_address(uint32_t** out) {
 
 extern "C" int lsa_topk_noalloc(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
                                 const float* logit, int32_t* topk, int32_t* topk_count, void* stream) {
+  const lsa::CallRange range("lsa_topk_noalloc");
   using namespace lsa;
   if (B < 0 || L <= 0 || N < 0 || k < 0 || cap < 0)
     return fail(LSA_ERR_INVALID_ARG, "topk_noalloc: bad size (L must be >= 1)");
