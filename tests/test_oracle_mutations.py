@@ -385,6 +385,42 @@ def step_projection_without_bf16_boundaries(h_raw, Wd_raw, Wu_raw, Ww_raw, H, dI
                            OS.decode(Ww_raw, wdtype), H, dI, bf16_boundaries=False)
 
 
+
+def _forward_variant(relu=True, bias=True, round_c=True, round_q=True, w_from="h", round_w=False,
+                     weight_inside=False):
+    def forward(h, Wd, Wu, Ww, b, K, H, dI, bf16_boundaries):
+        c = h @ Wd
+        if bf16_boundaries and round_c:
+            c = O.round_to_bf16(c)
+        q = c @ Wu
+        if bf16_boundaries and round_q:
+            q = O.round_to_bf16(q)
+        q = q.reshape(h.shape[0], H, dI)
+        w = h @ Ww if w_from == "h" else c @ Ww[: c.shape[1]]
+        if round_w:
+            w = O.round_to_bf16(w)
+        A = np.einsum("phd,sd->phs", q, K)
+        if weight_inside:
+            z = np.maximum(np.einsum("ph,phs->ps", w, A), 0.0)
+        else:
+            z = np.einsum("ph,phs->ps", w, np.maximum(A, 0.0) if relu else A)
+        return c, q, w, A, z + (b if bias else 0.0)
+    return forward
+
+
+def grads_bf16_backward_with_unrounded_c(h, Wd, Wu, Ww, b, K, y, H, dI, gamma, bf16_boundaries):
+    bce, fl, grads = _orig_loss_and_grads(h, Wd, Wu, Ww, b, K, y, H, dI, gamma, bf16_boundaries)
+    h = np.asarray(h, dtype=np.float64)
+    _, q, w, A, z = T.forward(h, Wd, Wu, Ww, b, K, H, dI, bf16_boundaries)
+    g = T.dloss_dz(z, y, gamma, z.size)
+    U = np.einsum("ps,phs,sd->phd", g, (A > 0).astype(np.float64), K)
+    dq = (w[:, :, None] * U).reshape(h.shape[0], H * dI)
+    return bce, fl, {**grads, "W_up": (h @ Wd).T @ dq}     # c before its rounding
+
+
+_orig_loss_and_grads = T.loss_and_grads
+
+
 MISTAKES = {
     "step top-k over the last layer's new set": (OS, "select", step_topk_over_last_new_set),
     "step e4m3 scale ignored": (OS, "decode_keys", step_scale_ignored),
@@ -424,6 +460,14 @@ MISTAKES = {
     "backward without the ReLU gate": (T, "loss_and_grads", grads_without_relu_gate),
     "hot pool pairs in age order": (O.HotPool, "update", hot_pool_pairs_in_age_order),
     "hot pool hit keeps the old stamp": (O.HotPool, "update", hot_pool_keeps_old_stamps),
+    "training forward without the ReLU": (T, "forward", _forward_variant(relu=False)),
+    "training forward drops the bias": (T, "forward", _forward_variant(bias=False)),
+    "training forward with c not rounded": (T, "forward", _forward_variant(round_c=False)),
+    "training forward with q not rounded": (T, "forward", _forward_variant(round_q=False)),
+    "training forward with w from c": (T, "forward", _forward_variant(w_from="c")),
+    "training forward with w rounded to bf16": (T, "forward", _forward_variant(round_w=True)),
+    "training forward with the head weight inside the ReLU": (T, "forward", _forward_variant(weight_inside=True)),
+    "training bf16 backward with unrounded c": (T, "loss_and_grads", grads_bf16_backward_with_unrounded_c),
 }
 
 

@@ -93,3 +93,95 @@ def test_head_weight_gradient_from_its_own_definition():
                           for p in range(h.shape[0])])
     _, _, grads = T.loss_and_grads(h, Wd, Wu, Ww, b, K, y, H, dI, 2.0, False)
     assert np.allclose(grads["W_w"], h.T @ dw_direct, rtol=1e-12, atol=1e-15)
+
+
+# ----------------------------------------------------------------------------- forward pass
+#
+# The backward pins above hold loss_and_grads to finite differences of a J that the same
+# forward() computes, so a mistake in forward() would pass them.  The pins below hold
+# forward() to the separately pinned projection and score (project_query,
+# head_fused_logits, whose own pins include the hand-derived worked example), and the
+# bf16 branch of the backward to finite differences of its straight-through surrogate.
+
+
+def _worked():
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "score_worked_example.json")) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_forward_on_the_worked_example(bf16):
+    """The hand-derived example (every value exact in bf16) through forward() with one
+    position: c, q, w, the per-head dots and z as derived by hand."""
+    ex = _worked()
+    e = ex["expected"]
+    h = np.array([ex["h"]], dtype=np.float64)
+    c, q, w, A, z = T.forward(h, np.array(ex["W_down"], dtype=np.float64), np.array(ex["W_up"], dtype=np.float64),
+                              np.array(ex["W_w"], dtype=np.float64), ex["bias"], np.array(ex["K"], dtype=np.float64),
+                              ex["H"], ex["dI"], bf16)
+    assert np.array_equal(c[0], e["c"])
+    assert np.array_equal(q[0], e["q"])
+    assert np.array_equal(w[0], e["w"])
+    assert np.array_equal(A[0].T, e["dots"])      # A[p][h][s], dots[s][h]
+    assert np.array_equal(z[0], e["z"])
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_forward_matches_the_pinned_projection_and_score(bf16):
+    """Per position, forward()'s q and w are project_query's and its z is
+    head_fused_logits' on them; the per-head dots A reproduce z through the ReLU and the
+    head weights.  Random inputs, so the bf16 roundings of c and q are active."""
+    h, Wd, Wu, Ww, b, K, y, H, dI = small_problem(5, P=4, N=60)
+    c, q, w, A, z = T.forward(h, Wd, Wu, Ww, b, K, H, dI, bf16)
+    for p in range(h.shape[0]):
+        q_ref, w_ref = O.project_query(h[p], Wd, Wu, Ww, H, dI, bf16)
+        if bf16:      # rounded values: equal (an fp64 sum one bit off a midpoint is ~2^-44 rare)
+            assert np.array_equal(q[p], q_ref)
+        else:         # batched and per-row fp64 products may differ in the last bit
+            np.testing.assert_allclose(q[p], q_ref, rtol=1e-13, atol=1e-15)
+        np.testing.assert_allclose(w[p], w_ref, rtol=1e-13, atol=1e-15)
+        z_ref = O.head_fused_logits(q_ref, w_ref, b, K)
+        np.testing.assert_allclose(z[p], z_ref, rtol=1e-13, atol=1e-13)
+        for s in range(K.shape[0]):
+            zs = b + sum(w_ref[hh] * max(0.0, float(q_ref[hh] @ K[s])) for hh in range(H))
+            assert abs(zs - z[p, s]) <= 1e-12 * (1 + abs(zs))
+            assert np.allclose(A[p, :, s], q_ref @ K[s], rtol=1e-13, atol=1e-13)
+    if bf16:   # the rounding really changed something on these inputs
+        q64, _ = O.project_query(h[0], Wd, Wu, Ww, H, dI, False)
+        assert not np.array_equal(q[0], q64)
+
+
+def test_bf16_branch_gradients_are_straight_through():
+    """With bf16 boundaries the gradients are those of the straight-through surrogate:
+    q(Wd', Wu') = q_r + c_r (Wu' - Wu) + (h (Wd' - Wd)) Wu', w = h Ww', where c_r and q_r
+    are the rounded values at the expansion point (c_r is project_query with an identity
+    up-projection, which returns the rounded c).  Finite differences of the surrogate's
+    loss, evaluated through the pinned score and loss, must match the bf16 branch."""
+    h, Wd, Wu, Ww, b, K, y, H, dI = small_problem(6, P=2, N=30)
+    P, r = h.shape[0], Wd.shape[1]
+    gamma = 2.0
+    c_r = np.stack([O.project_query(h[p], Wd, np.eye(r), Ww, 1, r, True)[0][0] for p in range(P)])
+    q_r = np.stack([O.project_query(h[p], Wd, Wu, Ww, H, dI, True)[0].ravel() for p in range(P)])
+
+    def J_st(Wd2, Wu2, Ww2, b2):
+        z = np.stack([O.head_fused_logits((q_r[p] + c_r[p] @ (Wu2 - Wu) + (h[p] @ (Wd2 - Wd)) @ Wu2).reshape(H, dI),
+                                          h[p] @ Ww2, b2, K) for p in range(P)])
+        return sum(O.bce_focal(O.sigmoid(z), y, gamma))
+
+    bce, fl, grads = T.loss_and_grads(h, Wd, Wu, Ww, b, K, y, H, dI, gamma, True)
+    assert bce + fl == pytest.approx(J_st(Wd, Wu, Ww, b), rel=1e-13)
+    eps = 1e-6
+    params = {"W_down": Wd, "W_up": Wu, "W_w": Ww}
+    for name, Wt in params.items():
+        for idx in np.ndindex(Wt.shape):
+            Wp, Wm = Wt.copy(), Wt.copy()
+            Wp[idx] += eps
+            Wm[idx] -= eps
+            a = {**params, name: Wp}
+            m = {**params, name: Wm}
+            fd = (J_st(a["W_down"], a["W_up"], a["W_w"], b) - J_st(m["W_down"], m["W_up"], m["W_w"], b)) / (2 * eps)
+            assert abs(fd - grads[name][idx]) <= 1e-6 + 1e-5 * abs(fd), (name, idx, fd, grads[name][idx])
+    fd_b = (J_st(Wd, Wu, Ww, b + eps) - J_st(Wd, Wu, Ww, b - eps)) / (2 * eps)
+    assert abs(fd_b - grads["b"]) <= 1e-6 + 1e-5 * abs(fd_b)
