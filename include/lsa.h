@@ -193,9 +193,12 @@ int lsa_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int3
  *   Scratch: a file-scope device array of 2^23 uint32 slots (32 MiB) that every GPU
  *   which loads this part of the library's device code keeps until the process exits.  B * cap must not exceed
  *   8,388,608; larger calls return LSA_ERR_NOMEM and launch nothing.
- *   Set-up: the first call on each device resolves the array's device address
- *   (cudaGetSymbolAddress, with that device current); make that first call before any
- *   stream capture.
+ *   Set-up: a call resolves the array's device address (cudaGetSymbolAddress, with the
+ *   call's device current) and remembers it per device.  A call made while its stream
+ *   is capturing reuses the remembered address instead, so make the first call on each
+ *   device before any stream capture (a first call during capture returns
+ *   LSA_ERR_UNSUPPORTED).  A device reset moves the array: the next call outside capture
+ *   picks up the new address, but a capture begun before that call still holds the old one.
  *   Sharing: all calls on a device use the same array, which keeps the last call's
  *   contents (nothing needs clearing: a call writes each slot before reading it).
  *   Calls that overlap on the GPU (for example on two streams) race on the array;

@@ -24,6 +24,8 @@ int fail(int code, const char* fmt, ...) {
   return code;
 }
 
+void clear_error() { g_err[0] = 0; }
+
 // Host-side fault injection for the error-path tests: with LSA_FAULT=launch in the
 // environment every launch check reports a failed launch (read once per process).
 static bool injected_launch_fault() {

@@ -25,6 +25,7 @@ struct CallRange {
 
 // ------------------------------------------------------------------ host-side errors
 int fail(int code, const char* fmt, ...);   // records the message, returns code
+void clear_error();                         // empties the calling thread's last message
 int check_launch(const char* what, int kernels = 1);   // LSA_OK or LSA_ERR_CUDA after launching
                                                         // `kernels` kernels (counted when OK)
 
