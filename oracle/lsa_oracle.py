@@ -22,6 +22,8 @@ Readings taken where the pages are silent (each is listed in the design notes):
   * threshold: marked  <=>  I >= 0.5  <=>  z >= 0.
   * top-k inside the fetched set ranks by the largest logit over the layers that
     marked the entry; equal keys -> lower entry index first; |U| <= k -> all of U.
+  * the native indexer's fine selection scores the fetched entries with the same
+    head-fused ReLU form, its own per-token query and keys, no bias or gate.
   * nucleus: descending probability, equal probability -> lower index first; the
     smallest prefix whose mass reaches top_p (an entry is in it iff the mass strictly
     before it is < top_p).
@@ -193,6 +195,30 @@ def fetched_key(z_by_layer, marks_by_layer) -> np.ndarray:
     z = np.asarray(z_by_layer, dtype=np.float64)
     m = np.asarray(marks_by_layer, dtype=bool)
     return np.where(m, z, -np.inf).max(axis=0)
+
+
+def fine_index_scores(q_f, w_f, K_f, fetched_idx) -> np.ndarray:
+    """Native-indexer score of every fetched entry for the current token ([SUMMARY] §2.1,
+    hierarchical selection: once the fetched subset is in GPU memory, the backbone's own
+    Lightning Indexer makes a fine top-k choice inside it for the core attention).
+
+    The pages name the native indexer but do not print its formula.  Reading: the same
+    head-fused ReLU form as the lookahead score, with the backbone indexer's per-token
+    query (q_f [H][dI], head weights w_f [H]) and its own keys K_f [N][dI]; no bias and no
+    sigmoid (neither changes an ordering).  Returns the scores of fetched_idx, in its order.
+    """
+    idx = np.asarray(fetched_idx, dtype=np.int64)
+    K = np.asarray(K_f, dtype=np.float64)[idx]
+    return head_fused_logits(q_f, w_f, 0.0, K)
+
+
+def fine_topk(q_f, w_f, K_f, fetched_idx, k: int) -> np.ndarray:
+    """The fine top-k of the fetched subset by the native-indexer score: candidates are the
+    fetched entries only; ties and ordering as in topk_in_fetched."""
+    idx = np.asarray(fetched_idx, dtype=np.int64)
+    key = np.full(np.asarray(K_f).shape[0], -np.inf)
+    key[idx] = fine_index_scores(q_f, w_f, K_f, idx)
+    return topk_in_fetched(idx, key, k)
 
 
 # ----------------------------------------------------------------------------- gather

@@ -421,6 +421,22 @@ def grads_bf16_backward_with_unrounded_c(h, Wd, Wu, Ww, b, K, y, H, dI, gamma, b
 _orig_loss_and_grads = T.loss_and_grads
 
 
+
+def fine_scores_with_bias(q_f, w_f, K_f, fetched_idx):
+    return O.head_fused_logits(q_f, w_f, 1.0, np.asarray(K_f, dtype=np.float64)[np.asarray(fetched_idx, dtype=np.int64)])
+
+
+def fine_scores_without_relu(q_f, w_f, K_f, fetched_idx):
+    K = np.asarray(K_f, dtype=np.float64)[np.asarray(fetched_idx, dtype=np.int64)]
+    return (K @ np.asarray(q_f, dtype=np.float64).T) @ np.asarray(w_f, dtype=np.float64)
+
+
+def fine_topk_over_all_entries(q_f, w_f, K_f, fetched_idx, k):
+    allidx = np.arange(np.asarray(K_f).shape[0])
+    key = O.fine_index_scores(q_f, w_f, K_f, allidx)
+    return O.topk_in_fetched(allidx, key, k)
+
+
 MISTAKES = {
     "step top-k over the last layer's new set": (OS, "select", step_topk_over_last_new_set),
     "step e4m3 scale ignored": (OS, "decode_keys", step_scale_ignored),
@@ -460,6 +476,9 @@ MISTAKES = {
     "backward without the ReLU gate": (T, "loss_and_grads", grads_without_relu_gate),
     "hot pool pairs in age order": (O.HotPool, "update", hot_pool_pairs_in_age_order),
     "hot pool hit keeps the old stamp": (O.HotPool, "update", hot_pool_keeps_old_stamps),
+    "fine score with a bias": (O, "fine_index_scores", fine_scores_with_bias),
+    "fine score without the ReLU": (O, "fine_index_scores", fine_scores_without_relu),
+    "fine top-k over all entries": (O, "fine_topk", fine_topk_over_all_entries),
     "training forward without the ReLU": (T, "forward", _forward_variant(relu=False)),
     "training forward drops the bias": (T, "forward", _forward_variant(bias=False)),
     "training forward with c not rounded": (T, "forward", _forward_variant(round_c=False)),

@@ -247,6 +247,44 @@ def test_topk_brute_force_with_ties():
         assert len(got) == min(k, n)
 
 
+def test_fine_topk_brute_force_loops():
+    """The native-indexer fine selection written out with loops on tiny inputs: per
+    fetched entry sum_h w_h max(0, sum_d q_hd k_d); the top-k of those among the fetched
+    entries only (ties to the lower index), in ascending entry order."""
+    g = np.random.default_rng(21)
+    for _ in range(60):
+        N, H, dI = int(g.integers(1, 25)), int(g.integers(1, 4)), int(g.integers(1, 5))
+        q = np.round(g.standard_normal((H, dI)), 1)
+        w = np.round(g.standard_normal(H), 1)
+        K = np.round(g.standard_normal((N, dI)), 1)
+        n = int(g.integers(0, N + 1))
+        fetched = np.sort(g.choice(N, size=n, replace=False))
+        k = int(g.integers(0, N + 2))
+        scores = [sum(w[h] * max(0.0, sum(q[h, d] * K[e, d] for d in range(dI))) for h in range(H)) for e in fetched]
+        got = O.fine_index_scores(q, w, K, fetched)
+        assert np.allclose(got, scores, rtol=1e-12, atol=1e-12)
+        key = {int(e): sc for e, sc in zip(fetched, got)}
+        want = sorted(e for e in key if sum(1 for t in key if key[t] > key[e] or (key[t] == key[e] and t < e)) < k)
+        assert O.fine_topk(q, w, K, fetched, k).tolist() == want
+
+
+def test_fine_topk_ignores_entries_outside_the_fetched_set():
+    """An entry that was not fetched is never chosen, whatever its score would be; the
+    fine query, not any other, decides the order."""
+    K = np.array([[10.0, 0.0], [1.0, 0.0], [0.0, 1.0], [0.0, 3.0]])
+    q = np.array([[1.0, 0.0]])
+    w = np.array([1.0])
+    assert O.fine_topk(q, w, K, [1, 2, 3], 1).tolist() == [1]       # entry 0 (score 10) not fetched
+    q2 = np.array([[0.0, 1.0]])
+    assert O.fine_topk(q2, w, K, [1, 2, 3], 1).tolist() == [3]
+    assert O.fine_topk(q2, w, K, [1, 2, 3], 2).tolist() == [2, 3]
+    # |fetched| <= k: everything fetched, in ascending order
+    assert O.fine_topk(q, w, K, [3, 1], 5).tolist() == [1, 3]
+    # a negative head weight ranks larger dot products lower; ReLU zeroes negative dots
+    assert O.fine_index_scores(np.array([[1.0, 1.0]]), np.array([-2.0]), K, [0, 3]).tolist() == [-20.0, -6.0]
+    assert O.fine_index_scores(np.array([[-1.0, 0.0]]), np.array([1.0]), K, [0, 1]).tolist() == [0.0, 0.0]
+
+
 def test_fetched_key_is_max_over_marking_layers():
     z = np.array([[1.0, -2.0, 0.5], [3.0, -1.0, -0.2], [-5.0, 0.0, 0.7]])
     m = z >= 0
