@@ -256,6 +256,24 @@ int lsa_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32
   return launch_compact(B, N, bits, cap, idx, count, status, static_cast<cudaStream_t>(stream));
 }
 
+int lsa_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* new_l, int cap,
+                     int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
+                     void* stream) {
+  const CallRange range("lsa_select_fetch");
+  g_err[0] = 0;
+  if (B < 0 || L < 0 || N < 0 || cap < 0) return fail(LSA_ERR_INVALID_ARG, "select_fetch: negative size");
+  if (L < 1 || L > 8) return fail(LSA_ERR_UNSUPPORTED, "select_fetch: L = %d layers (1 to 8)", L);
+  if (B == 0) return LSA_OK;
+  if (!cnt_new || !cnt_U || (N > 0 && !mask) || (cap > 0 && (!idx_new || !idx_U)))
+    return fail(LSA_ERR_INVALID_ARG, "select_fetch: null pointer");
+  if ((mask && !aligned(mask, 16)) || (U && !aligned(U, 16)) || (new_l && !aligned(new_l, 16)) ||
+      (idx_new && !aligned(idx_new, 16)) || (idx_U && !aligned(idx_U, 16)) || !aligned(cnt_new, 4) ||
+      !aligned(cnt_U, 4))
+    return fail(LSA_ERR_INVALID_ARG, "select_fetch: misaligned pointer");
+  return launch_select_fetch(B, L, N, mask, U, new_l, cap, idx_new, cnt_new, idx_U, cnt_U, status,
+                             static_cast<cudaStream_t>(stream));
+}
+
 size_t lsa_topk_workspace_bytes(int B, int cap) {
   if (B < 0 || cap < 0) return 0;
   return align_up(static_cast<size_t>(B) * cap * 4, 256) + 256;
@@ -456,9 +474,12 @@ int lsa_check_bounded_wait(uint32_t limit_us, int32_t* status, void* stream) {
                            static_cast<cudaStream_t>(stream));
 }
 
+// Per-row selection words in the vote kernels' blocked order: 4 per 128 entries.
+static size_t vote_row_words(int N) { return 4 * ((static_cast<size_t>(N) + 127) / 128); }
+
 size_t lsa_vote_labels_workspace_bytes(int L, int P, int N) {
   if (L < 0 || P < 0 || N < 0) return 0;
-  const size_t Nw = (static_cast<size_t>(N) + 31) / 32;
+  const size_t Nw = vote_row_words(N);
   return align_up(static_cast<size_t>(L) * P * Nw * 4, 256) +
          align_up(static_cast<size_t>(L) * P * 4 * 4, 256) + 256;
 }
@@ -479,7 +500,7 @@ int lsa_vote_labels(int L, int P, int N, const float* logits, float top_p, int t
   const size_t need = lsa_vote_labels_workspace_bytes(L, P, N);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
     return fail(LSA_ERR_NOMEM, "vote_labels: workspace %zu bytes (need %zu)", workspace_bytes, need);
-  const size_t Nw = (static_cast<size_t>(N) + 31) / 32;
+  const size_t Nw = vote_row_words(N);
   uint8_t* base = static_cast<uint8_t*>(workspace);
   VoteArgs va{};
   va.L = L; va.P = P; va.N = N; va.logits = logits; va.top_p = top_p; va.theta = theta;

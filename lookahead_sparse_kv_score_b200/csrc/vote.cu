@@ -51,6 +51,30 @@ __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
+// Selection words of a row (workspace) are kept in blocked order, which one ballot per
+// element of a warp's float4 loads produces directly: for the 128 entries
+// 128j .. 128j+127, word 4j + e holds in bit i the entry 128j + 4i + e.  A row has
+// 4 ceil(N / 128) words; vote_count_kernel returns the labels to entry order.
+__device__ __forceinline__ size_t sel_word(uint32_t idx) { return 4 * static_cast<size_t>(idx >> 7) + (idx & 3); }
+__device__ __forceinline__ uint32_t sel_bit(uint32_t idx) { return 1u << ((idx >> 2) & 31); }
+
+// 2^x by the hardware approximation (relative error ~2^-22; flushes denormals).
+// e^(x - m) = 2^(x log2 e - m log2 e): one fma and one approximation per entry.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+// The mass term e^(x - m0) of the window path, given nm = -m0 log2 e; every mass of a
+// row's window path (Z, the mass above the run, the run's entries) uses this one form.
+__device__ __forceinline__ float win_term(float x, float nm) { return ex2_approx(fmaf(x, kLog2e, nm)); }
+
+// One count into the shared-memory histogram at a 32-bit shared address.
+__device__ __forceinline__ void red_shared_inc(uint32_t addr) {
+  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
+}
+
 template <typename T, typename Op>
 __device__ __forceinline__ T block_reduce(T v, T* tmp, Op op) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -157,15 +181,6 @@ __device__ __forceinline__ void row_for_each(const float* x, int N, bool vec, F&
     for (int u = 0; u < 4; ++u) run(v[u], 4 * (g + u * kRowThreads));
   }
   for (; g < G; g += kRowThreads) run(load4(x, 4 * g, N, vec), 4 * g);
-}
-
-// Linear bin of x in the window [a - kFineBins / inv_w, a]: floor(t) for
-// t = a inv_w - x inv_w (one fma), by an add of 2^23 rounded down (exact for
-// 0 <= t < 2^23); larger t, infinities and NaN give values >= kFineBins, x > a negative
-// values (or bin 0 within a rounding of a).
-__device__ __forceinline__ int fine_bin(float x, float a_inv_w, float inv_w) {
-  const float t = fmaf(-x, inv_w, a_inv_w);
-  return __float_as_int(__fadd_rd(t, 8388608.f)) - 0x4B000000;
 }
 
 // Ascending bitonic sort of n entries (n a power of two, >= 64).  Stages whose partner
@@ -358,10 +373,11 @@ __device__ bool sorted_run_crossing(unsigned long long* list, int C, double abov
   for (int i = C + tid; i < P2; i += kRowThreads) list[i] = ~0ull;
   __syncthreads();
   bitonic_sort(list, P2);
+  const float nm = -m0 * kLog2e;
   const int chunk = (C + kRowThreads - 1) / kRowThreads;
   const int j0 = tid * chunk < C ? tid * chunk : C, j1 = j0 + chunk < C ? j0 + chunk : C;
   double loc = 0.0;
-  for (int j = j0; j < j1; ++j) loc += static_cast<double>(__expf(key_value(~static_cast<uint32_t>(list[j] >> 32)) - m0));
+  for (int j = j0; j < j1; ++j) loc += static_cast<double>(win_term(key_value(~static_cast<uint32_t>(list[j] >> 32)), nm));
   double ex, ex2;
   block_scan2(loc, 0.0, sh.d2tmp, ex, ex2);
   if (tid == 0) sh.jstar = C + 1;     // C + 1: the crossing lies below the run
@@ -370,7 +386,7 @@ __device__ bool sorted_run_crossing(unsigned long long* list, int C, double abov
     double run = ex;
     for (int j = j0; j < j1; ++j) {
       if (above + run >= target) { atomicMin(&sh.jstar, j); break; }
-      run += static_cast<double>(__expf(key_value(~static_cast<uint32_t>(list[j] >> 32)) - m0));
+      run += static_cast<double>(win_term(key_value(~static_cast<uint32_t>(list[j] >> 32)), nm));
     }
     // every entry of the run selected, the first one below it not
     if (j1 == C && j0 < j1 && above + run >= target) atomicMin(&sh.jstar, C);
@@ -380,7 +396,7 @@ __device__ bool sorted_run_crossing(unsigned long long* list, int C, double abov
   if (js == 0 || js > C) return false;
   for (int j = tid; j < js; j += kRowThreads) {
     const uint32_t idx = static_cast<uint32_t>(list[j] & 0xffffffffu);
-    atomicOr(&out[idx >> 5], 1u << (idx & 31));
+    atomicOr(&out[sel_word(idx)], sel_bit(idx));
   }
   const unsigned long long last = list[js - 1];
   res = make_int2(static_cast<int>(~static_cast<uint32_t>(last >> 32)), static_cast<int>(last & 0xffffffffu));
@@ -431,22 +447,28 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
     double zloc = 0.0;
     // Entries above a (only when the row gets re-anchored) and NaN spoil Z, which is
     // then discarded; entries outside the window land in the trash bin.
-    // a inv_w rounded up: every x <= a then gets t >= 0, bin 0 included
+    // a inv_w rounded up: every x <= a then gets t >= 0, bin 0 included.  The bin of x:
+    // u = sat((a inv_w - x inv_w) / kFineBins) by one saturating fma, then
+    // 2^23 + floor(u kFineBins) by a round-down fma; that float's bit pattern times 4
+    // plus a constant is the bin's shared-memory address (u = 1: the trash bin).
     const float ainv = __fmul_ru(a, inv_w);
-    auto body = [&](auto full, const float4& v, int s) {
+    const float c1 = -inv_w / kFineBins, c0 = ainv / kFineBins;
+    const uint32_t hbase = static_cast<uint32_t>(__cvta_generic_to_shared(hist)) - 0x4B000000u * 4u;
+    const float nm = -m0 * kLog2e;
+    auto body = [&](auto full, const float4& v, int s) -> float {
       constexpr bool kFull = decltype(full)::value;
       const float xs[4] = {v.x, v.y, v.z, v.w};
-      float ez = 0.f;              // at most four terms <= e^4 before the fp64 sum
+      float ez = 0.f;              // at most four terms <= e^4
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         if (kFull || s + j < N) {
           mloc = fmaxf(mloc, xs[j]);
-          ez += __expf(xs[j] - m0);
-          const unsigned b = static_cast<unsigned>(fine_bin(xs[j], ainv, inv_w));
-          atomicAdd(&hist[b < static_cast<unsigned>(kFineBins) ? b : kFineBins], 1);
+          ez += ex2_approx(fmaf(xs[j], kLog2e, nm));
+          const float u = __saturatef(fmaf(xs[j], c1, c0));
+          red_shared_inc(__float_as_uint(__fmaf_rd(u, static_cast<float>(kFineBins), 8388608.f)) * 4u + hbase);
         }
       }
-      zloc += static_cast<double>(ez);
+      return ez;
     };
     int g0 = tid;
     const uint64_t keep = l2_policy_last();
@@ -454,15 +476,19 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
       float4 v4[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) v4[u] = ldg4_hint(reinterpret_cast<const float4*>(x) + g0 + u * kRowThreads, keep);
+      float ez = 0.f;              // sixteen terms in fp32, then the fp64 sum
 #pragma unroll
-      for (int u = 0; u < 4; ++u) body(std::true_type{}, v4[u], 4 * (g0 + u * kRowThreads));
+      for (int u = 0; u < 4; ++u) ez += body(std::true_type{}, v4[u], 4 * (g0 + u * kRowThreads));
+      zloc += static_cast<double>(ez);
     }
     for (; g0 < G; g0 += 4 * kRowThreads) {
       float4 v4[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) v4[u] = load4(x, 4 * (g0 + u * kRowThreads), N, vec);
+      float ez = 0.f;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) body(std::false_type{}, v4[u], 4 * (g0 + u * kRowThreads));
+      for (int u = 0; u < 4; ++u) ez += body(std::false_type{}, v4[u], 4 * (g0 + u * kRowThreads));
+      zloc += static_cast<double>(ez);
     }
     m = block_reduce(mloc, sh.ftmp, [](float p, float q) { return fmaxf(p, q); });
     Z = block_reduce(zloc, sh.dtmp, [](double p, double q) { return p + q; });
@@ -532,40 +558,48 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
   __syncthreads();
   double aloc = 0.0;
   {
-    const int Nw = (N + 31) >> 5;
+    // A warp's lanes hold 32 consecutive float4 groups, i.e. one 128-entry block: one
+    // ballot per element gives that block's four selection words (blocked order).
     const int Gr = (G + 31) & ~31;      // whole warps per iteration
-    auto body = [&](auto full, const float4& v, int s) {
+    const float nm = -m0 * kLog2e;
+    auto body = [&](auto full, const float4& v, int s) -> float {
       constexpr bool kFull = decltype(full)::value;
-      const float xs[4] = {v.x, v.y, v.z, v.w};
-      uint32_t nib = 0, inm = 0;
+      const float xs[4] = {v.x, v.y, v.z, v.w};   // NaN past N: neither above nor in the run
       float ea = 0.f;
+      uint32_t wd[4];
+      bool run[4];
+      bool any_run = false;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (kFull || s + j < N) {
-          const bool up = xs[j] > xu;
-          const float e = __expf(xs[j] - m0);
-          ea += up ? e : 0.f;
-          nib |= static_cast<uint32_t>(up) << j;
-          inm |= static_cast<uint32_t>(!up && xs[j] > xl) << j;
-        }
+        const bool up = (kFull || s + j < N) && xs[j] > xu;
+        wd[j] = __ballot_sync(0xffffffffu, up);
+        run[j] = !up && xs[j] > xl;
+        any_run |= run[j];
+        const float e = ex2_approx(fmaf(xs[j], kLog2e, nm));
+        ea += up ? e : 0.f;
       }
-      aloc += static_cast<double>(ea);
-      uint32_t word = nib << (4 * (lane & 7));
-      word |= __shfl_xor_sync(0xffffffffu, word, 1);
-      word |= __shfl_xor_sync(0xffffffffu, word, 2);
-      word |= __shfl_xor_sync(0xffffffffu, word, 4);
-      if ((lane & 7) == 0 && (kFull || s < Nw * 32)) out[s >> 5] = word;
-      if (inm) {
-        int pos = atomicAdd(&sh.count, __popc(inm));
+      if (lane == 0 && s < N) *reinterpret_cast<uint4*>(out + 4 * (s >> 7)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+      if (__any_sync(0xffffffffu, any_run)) {
+        uint32_t rb[4];
+        int tot = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          if ((inm >> j) & 1u) {
-            if (pos < kListCap)
-              list[pos] = (static_cast<unsigned long long>(~order_key(xs[j])) << 32) | static_cast<uint32_t>(s + j);
-            ++pos;
-          }
+          rb[j] = __ballot_sync(0xffffffffu, run[j]);
+          tot += __popc(rb[j]);
+        }
+        int pos = 0;
+        if (lane == 0) pos = atomicAdd(&sh.count, tot);
+        pos = __shfl_sync(0xffffffffu, pos, 0);
+        const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int at = pos + __popc(rb[j] & lt);
+          if (run[j] && at < kListCap)
+            list[at] = (static_cast<unsigned long long>(~order_key(xs[j])) << 32) | static_cast<uint32_t>(s + j);
+          pos += __popc(rb[j]);
         }
       }
+      return ea;
     };
     int g0 = tid;
     const uint64_t last = l2_policy_first();
@@ -574,15 +608,19 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
       float4 v4[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) v4[u] = ldg4_hint(reinterpret_cast<const float4*>(x) + g0 + u * kRowThreads, last);
+      float ea = 0.f;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) body(std::true_type{}, v4[u], 4 * (g0 + u * kRowThreads));
+      for (int u = 0; u < 4; ++u) ea += body(std::true_type{}, v4[u], 4 * (g0 + u * kRowThreads));
+      aloc += static_cast<double>(ea);
     }
     for (; g0 < Gr; g0 += 4 * kRowThreads) {
       float4 v4[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) v4[u] = load4(x, 4 * (g0 + u * kRowThreads), N, vec);
+      float ea = 0.f;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) body(std::false_type{}, v4[u], 4 * (g0 + u * kRowThreads));
+      for (int u = 0; u < 4; ++u) ea += body(std::false_type{}, v4[u], 4 * (g0 + u * kRowThreads));
+      aloc += static_cast<double>(ea);
     }
   }
   const double above = block_reduce(aloc, sh.dtmp, [](double p, double q) { return p + q; });
@@ -594,6 +632,7 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
   // entries are ranked by (key descending, index ascending) in one warp.
   int* scnt = hist;
   double* smass = reinterpret_cast<double*>(dsm + kSubBins * 4);
+  const float nm = -m0 * kLog2e;
   const float inv_ws = static_cast<float>(kSubBins) / fmaxf(xu - xl, 1e-30f);
   auto sub_bin = [&](unsigned long long ent) {
     const float xv = key_value(~static_cast<uint32_t>(ent >> 32));
@@ -607,7 +646,7 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
     const unsigned long long ent = list[j];
     const int sb = sub_bin(ent);
     atomicAdd(&scnt[sb], 1);
-    atomicAdd(&smass[sb], static_cast<double>(__expf(key_value(~static_cast<uint32_t>(ent >> 32)) - m0)));
+    atomicAdd(&smass[sb], static_cast<double>(win_term(key_value(~static_cast<uint32_t>(ent >> 32)), nm)));
   }
   __syncthreads();
   constexpr int kSubPer = kSubBins / kRowThreads;
@@ -646,7 +685,7 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
   if (tid < 32) {
     const unsigned long long mine = lane < nS ? sh.sub[lane] : ~0ull;
     const double em =
-        lane < nS ? static_cast<double>(__expf(key_value(~static_cast<uint32_t>(mine >> 32)) - m0)) : 0.0;
+        lane < nS ? static_cast<double>(win_term(key_value(~static_cast<uint32_t>(mine >> 32)), nm)) : 0.0;
     double mb = 0.0;                  // mass of the sub-bin's entries before this one
     for (int o = 0; o < nS; ++o) {
       const unsigned long long other = __shfl_sync(0xffffffffu, mine, o);
@@ -672,7 +711,7 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
     const int sb = sub_bin(ent);
     if (sb < S || (sb == S && ent <= last)) {
       const uint32_t idx = static_cast<uint32_t>(ent & 0xffffffffu);
-      atomicOr(&out[idx >> 5], 1u << (idx & 31));
+      atomicOr(&out[sel_word(idx)], sel_bit(idx));
     }
   }
   res = make_int2(static_cast<int>(~static_cast<uint32_t>(last >> 32)), static_cast<int>(last & 0xffffffffu));
@@ -680,18 +719,19 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
   return true;
 }
 
-// One row per iteration of the block.  selbits [L*P][Nw]; rowparam [L*P] = (T, cutoff index).
+// One row per iteration of the block.  selbits [L*P][4 ceil(N/128)] in blocked order;
+// rowparam [L*P] = (T, cutoff index).
 __global__ void __launch_bounds__(kRowThreads, kRowThreads >= 1024 ? 1 : 2)
 vote_rows_kernel(const float* __restrict__ logits, int rows, int N, float top_p, float R,
                  uint32_t* __restrict__ selbits, int2* __restrict__ rowparam) {
   extern __shared__ __align__(16) uint8_t vsm[];
   __shared__ RowShared sh;
   const int tid = threadIdx.x, lane = tid & 31;
-  const int Nw = (N + 31) / 32;
+  const size_t Nwb = 4 * static_cast<size_t>((N + 127) / 128);   // blocked words per row
   for (int row = blockIdx.x; row < rows; row += gridDim.x) {
     const float* x = logits + static_cast<size_t>(row) * N;
     const bool vec = (N % 4 == 0) && (reinterpret_cast<uintptr_t>(x) % 16 == 0);
-    uint32_t* out = selbits + static_cast<size_t>(row) * Nw;
+    uint32_t* out = selbits + static_cast<size_t>(row) * Nwb;
     int2 tc;
     const bool ok = top_p < 1.f && window_nucleus(x, N, vec, top_p, R, vsm, sh, out, tc);
     if (tid == 0 && ok) rowparam[row] = tc;
@@ -703,8 +743,9 @@ vote_rows_kernel(const float* __restrict__ logits, int rows, int N, float top_p,
     if (tid == 0) rowparam[row] = tc;
     const uint32_t T = static_cast<uint32_t>(tc.x);
     const int cut = tc.y;
-    // selection bits: lanes 8k .. 8k+7 hold the 32 entries of one word
-    const int Gr = (Nw * 8 + 31) & ~31;
+    // selection words in blocked order: one ballot per element of a warp's float4 groups
+    const int G = (N + 3) >> 2;
+    const int Gr = (G + 31) & ~31;
     for (int g0 = tid; g0 < Gr; g0 += 4 * kRowThreads) {
       float4 v4[4];
 #pragma unroll
@@ -713,101 +754,123 @@ vote_rows_kernel(const float* __restrict__ logits, int rows, int N, float top_p,
       for (int u = 0; u < 4; ++u) {
         const int s = 4 * (g0 + u * kRowThreads);
         const float xs[4] = {v4[u].x, v4[u].y, v4[u].z, v4[u].w};
-        uint32_t nib = 0;
+        uint32_t wd[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          if (s + j < N) {
-            const uint32_t k = order_key(xs[j]);
-            nib |= static_cast<uint32_t>(k > T || (k == T && s + j <= cut)) << j;
-          }
+          const uint32_t k = order_key(xs[j]);
+          wd[j] = __ballot_sync(0xffffffffu, s + j < N && (k > T || (k == T && s + j <= cut)));
         }
-        uint32_t word = nib << (4 * (lane & 7));
-        word |= __shfl_xor_sync(0xffffffffu, word, 1);
-        word |= __shfl_xor_sync(0xffffffffu, word, 2);
-        word |= __shfl_xor_sync(0xffffffffu, word, 4);
-        if ((lane & 7) == 0 && s < Nw * 32) out[s >> 5] = word;
+        if (lane == 0 && s < N) *reinterpret_cast<uint4*>(out + 4 * (s >> 7)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
       }
     }
     __syncthreads();
   }
 }
 
-// Per (position, word): the 32 entries' layer counts as a bit-sliced counter (plane k
-// holds bit k of every count), golden bits (count >= theta) and optional byte counts.
+// Bits 0..7 of x moved to bits 0, 4, 8, .., 28.
+__device__ __forceinline__ uint32_t spread_byte(uint32_t x) {
+  x &= 0xFFu;
+  x = (x | (x << 12)) & 0x000F000Fu;
+  x = (x | (x << 6)) & 0x03030303u;
+  x = (x | (x << 3)) & 0x11111111u;
+  return x;
+}
+
+// Per (position, 128-entry block): the layer counts of its entries as bit-sliced
+// counters (plane k holds bit k of every count) over the block's four blocked-order
+// selection words, golden bits (count >= theta) turned back into entry order, and the
+// optional byte counts.
 template <int kPlanes>
 __global__ void vote_count_kernel(const uint32_t* __restrict__ selbits, int L, int P, int N, int theta,
                                   uint32_t* __restrict__ golden, uint8_t* __restrict__ counts) {
+  const int Nb = (N + 127) / 128;
   const int Nw = (N + 31) / 32;
   const int p = blockIdx.y;
-  const int w = blockIdx.x * blockDim.x + threadIdx.x;
-  if (w >= Nw) return;
-  uint32_t pl[kPlanes];
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= Nb) return;
+  uint32_t pl[4][kPlanes];
 #pragma unroll
-  for (int k = 0; k < kPlanes; ++k) pl[k] = 0u;
-  const uint32_t* src = selbits + static_cast<size_t>(p) * Nw + w;
-  const size_t stride = static_cast<size_t>(P) * Nw;
-  int l = 0;
-  for (; l + 4 <= L; l += 4) {
-    uint32_t b[4];
+  for (int e = 0; e < 4; ++e)
 #pragma unroll
-    for (int u = 0; u < 4; ++u) b[u] = __ldg(src + (l + u) * stride);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      uint32_t carry = b[u];
-#pragma unroll
-      for (int k = 0; k < kPlanes; ++k) {
-        const uint32_t t = pl[k] & carry;
-        pl[k] ^= carry;
-        carry = t;
-      }
-    }
-  }
-  for (; l < L; ++l) {
-    uint32_t carry = __ldg(src + l * stride);
+    for (int k = 0; k < kPlanes; ++k) pl[e][k] = 0u;
+  const uint4* src = reinterpret_cast<const uint4*>(selbits) + static_cast<size_t>(p) * Nb + j;
+  const size_t stride = static_cast<size_t>(P) * Nb;
+  auto add = [&](uint32_t carry, uint32_t* plane) {
 #pragma unroll
     for (int k = 0; k < kPlanes; ++k) {
-      const uint32_t t = pl[k] & carry;
-      pl[k] ^= carry;
+      const uint32_t t = plane[k] & carry;
+      plane[k] ^= carry;
       carry = t;
     }
+  };
+  int l = 0;
+  for (; l + 2 <= L; l += 2) {
+    const uint4 b0 = __ldg(src + l * stride), b1 = __ldg(src + (l + 1) * stride);
+    add(b0.x, pl[0]); add(b0.y, pl[1]); add(b0.z, pl[2]); add(b0.w, pl[3]);
+    add(b1.x, pl[0]); add(b1.y, pl[1]); add(b1.z, pl[2]); add(b1.w, pl[3]);
+  }
+  for (; l < L; ++l) {
+    const uint4 b = __ldg(src + l * stride);
+    add(b.x, pl[0]); add(b.y, pl[1]); add(b.z, pl[2]); add(b.w, pl[3]);
   }
   // count >= theta  <=>  no borrow out of count - theta (0 < theta < 2^kPlanes)
-  uint32_t g;
-  if (theta <= 0) {
-    g = 0xffffffffu;
-  } else if (theta >= (1 << kPlanes)) {
-    g = 0u;
-  } else {
-    uint32_t borrow = 0u;
+  uint32_t g[4];
 #pragma unroll
-    for (int k = 0; k < kPlanes; ++k)
-      borrow = ((theta >> k) & 1) ? (~pl[k] | borrow) : (~pl[k] & borrow);
-    g = ~borrow;
-  }
-  const int valid = N - w * 32;
-  if (valid < 32) g &= (1u << valid) - 1u;
-  golden[static_cast<size_t>(p) * Nw + w] = g;
-  if (counts) {
-    uint32_t packed[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      uint32_t v = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int bit = 4 * q + j;
-        uint32_t c = 0;
-#pragma unroll
-        for (int k = 0; k < kPlanes; ++k) c |= ((pl[k] >> bit) & 1u) << k;
-        v |= c << (8 * j);
-      }
-      packed[q] = v;
-    }
-    uint8_t* c = counts + static_cast<size_t>(p) * N + static_cast<size_t>(w) * 32;
-    if (valid >= 32 && (reinterpret_cast<uintptr_t>(c) & 15) == 0) {
-      reinterpret_cast<uint4*>(c)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-      reinterpret_cast<uint4*>(c)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+  for (int e = 0; e < 4; ++e) {
+    if (theta <= 0) {
+      g[e] = 0xffffffffu;
+    } else if (theta >= (1 << kPlanes)) {
+      g[e] = 0u;
     } else {
-      for (int b = 0; b < 32 && b < valid; ++b) c[b] = static_cast<uint8_t>(packed[b >> 2] >> (8 * (b & 3)));
+      uint32_t borrow = 0u;
+#pragma unroll
+      for (int k = 0; k < kPlanes; ++k)
+        borrow = ((theta >> k) & 1) ? (~pl[e][k] | borrow) : (~pl[e][k] & borrow);
+      g[e] = ~borrow;
+    }
+  }
+  // entry order: bit 4k + e of word 4j + m is entry 128j + 32m + 4k + e = 128j + 4(8m + k) + e,
+  // i.e. bit 8m + k of blocked word e
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int w = 4 * j + m;
+    if (w >= Nw) break;
+    uint32_t gw = spread_byte(g[0] >> (8 * m)) | (spread_byte(g[1] >> (8 * m)) << 1) |
+                  (spread_byte(g[2] >> (8 * m)) << 2) | (spread_byte(g[3] >> (8 * m)) << 3);
+    const int valid = N - w * 32;
+    if (valid < 32) gw &= (1u << valid) - 1u;
+    golden[static_cast<size_t>(p) * Nw + w] = gw;
+  }
+  if (counts) {
+    // byte 128j + 4i + e = count of blocked word e, bit i
+    uint8_t* c = counts + static_cast<size_t>(p) * N + static_cast<size_t>(j) * 128;
+    const int valid = N - j * 128;
+    const bool vec = valid >= 128 && (reinterpret_cast<uintptr_t>(c) & 15) == 0;
+#pragma unroll
+    for (int i4 = 0; i4 < 32; i4 += 4) {
+      uint32_t v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = i4 + q;
+        uint32_t word = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint32_t cnt = 0;
+#pragma unroll
+          for (int k = 0; k < kPlanes; ++k) cnt |= ((pl[e][k] >> i) & 1u) << k;
+          word |= cnt << (8 * e);
+        }
+        v[q] = word;
+      }
+      if (vec) {
+        reinterpret_cast<uint4*>(c)[i4 / 4] = make_uint4(v[0], v[1], v[2], v[3]);
+      } else {
+        for (int q = 0; q < 4; ++q)
+          for (int e = 0; e < 4; ++e) {
+            const int at = 4 * (i4 + q) + e;
+            if (at < valid) c[at] = static_cast<uint8_t>(v[q] >> (8 * e));
+          }
+      }
     }
   }
 }
@@ -879,7 +942,6 @@ __global__ void vote_loss_finalize(const double* __restrict__ acc, double n, dou
 
 int launch_vote(const VoteArgs& a, cudaStream_t st) {
   const int rows = a.L * a.P;
-  const int Nw = (a.N + 31) / 32;
   int rc = LSA_OK;
   if (rows > 0 && a.N > 0) {
     const int smem = kRowSmem;
@@ -897,11 +959,12 @@ int launch_vote(const VoteArgs& a, cudaStream_t st) {
                                                       reinterpret_cast<int2*>(a.rowparam));
     if ((rc = check_launch("vote_labels/rows")) != LSA_OK) return rc;
   }
-  const dim3 cgrid((Nw + 255) / 256, a.P);
+  constexpr int kCountThreads = 128;
+  const dim3 cgrid(((a.N + 127) / 128 + kCountThreads - 1) / kCountThreads, a.P);
   if (a.L <= 31)
-    vote_count_kernel<5><<<cgrid, 256, 0, st>>>(a.selbits, a.L, a.P, a.N, a.theta, a.golden, a.counts);
+    vote_count_kernel<5><<<cgrid, kCountThreads, 0, st>>>(a.selbits, a.L, a.P, a.N, a.theta, a.golden, a.counts);
   else
-    vote_count_kernel<8><<<cgrid, 256, 0, st>>>(a.selbits, a.L, a.P, a.N, a.theta, a.golden, a.counts);
+    vote_count_kernel<8><<<cgrid, kCountThreads, 0, st>>>(a.selbits, a.L, a.P, a.N, a.theta, a.golden, a.counts);
   if ((rc = check_launch("vote_labels/count")) != LSA_OK) return rc;
   if (a.scores) {
     cudaMemsetAsync(a.lossacc, 0, 2 * sizeof(double), st);
