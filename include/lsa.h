@@ -166,6 +166,26 @@ int lsa_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32
                 int32_t* status, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * lsa_select_fetch -- the union, the per-layer new sets and all fetch lists of one
+ * trigger in one launch ([SUMMARY] §2.4 OR mode over the indexer layers; §2.1 dynamic
+ * fetch: every marked entry is fetched, incrementally as layers finish).  Equal to
+ * zeroing U, calling lsa_select_union for layers 0..L-1 in order and lsa_compact on
+ * each new set and on the union:
+ *     new_l = mask_l & ~(mask_0 | .. | mask_{l-1}),   U = mask_0 | .. | mask_{L-1},
+ *     idx_new[l][b][..] = ascending entries of new_l[b], cnt_new[l][b] = |new_l[b]|,
+ *     idx_U[b][..] = ascending entries of U[b],           cnt_U[b] = |U[b]|.
+ *   mask [L][B][Nw] (Nw = ceil(N/32); bits past N must be zero, as lsa_index_score
+ *   leaves them); U [B][Nw] and new_l [L][B][Nw] outputs or NULL; idx_new [L][B][cap],
+ *   cnt_new [L][B], idx_U [B][cap], cnt_U [B] int32 outputs.  A count above cap is
+ *   reported as is, only cap indices are written and *status (device int32 or NULL) is
+ *   raised to LSA_ERR_CAPACITY.  1 <= L <= 8, else LSA_ERR_UNSUPPORTED.  Device
+ *   pointers 16-byte aligned (counts 4-byte).  One launch per block of 65535 sequences.
+ * ---------------------------------------------------------------------------------- */
+int lsa_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* new_l, int cap,
+                     int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
+                     void* stream);
+
+/* ------------------------------------------------------------------------------------
  * lsa_topk -- fine top-k inside the fetched subset ([SUMMARY] §2.1 hierarchical
  * selection: once the critical subset is in GPU memory, a top-k runs inside it).
  * Candidate j of sequence b is entry e = idx[b][j], j < min(count[b], cap); its key is

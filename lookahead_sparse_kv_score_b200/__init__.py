@@ -122,6 +122,11 @@ def lsa_compact(B, N, bits, cap, idx, count, status=None, stream=None):
            "lsa_compact")
 
 
+def lsa_select_fetch(B, L, N, mask, U, new_l, cap, idx_new, cnt_new, idx_U, cnt_U, status=None, stream=None):
+    _check(lib().lsa_select_fetch(B, L, N, _p(mask), _p(U), _p(new_l), cap, _p(idx_new), _p(cnt_new), _p(idx_U),
+                                  _p(cnt_U), _p(status), _stream(stream)), "lsa_select_fetch")
+
+
 def lsa_topk_workspace_bytes(B, cap) -> int:
     return int(lib().lsa_topk_workspace_bytes(B, cap))
 

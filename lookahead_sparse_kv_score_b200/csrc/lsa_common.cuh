@@ -112,6 +112,9 @@ int launch_score_tc(const TcArgs& a, cudaStream_t s);
 int launch_union(int B, int Nw, const uint32_t* m, uint32_t* U, uint32_t* nw, cudaStream_t s);
 int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32_t* count,
                    int32_t* status, cudaStream_t s);
+int launch_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* nw, int cap,
+                        int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
+                        cudaStream_t s);
 int launch_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
                 const float* logit, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws,
                 cudaStream_t s);

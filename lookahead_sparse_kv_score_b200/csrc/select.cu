@@ -125,6 +125,125 @@ compact_kernel(const uint32_t* __restrict__ bits, int Nw, int cap, int32_t* __re
   }
 }
 
+// ------------------------------------------------------------------ union + fetch lists
+// The whole selection of one trigger in one pass over the L layer masks: per word,
+// new_l = mask_l & ~(mask_0 | .. | mask_{l-1}) and U = mask_0 | .. | mask_{L-1}, and the
+// L + 1 fetch lists (new_0 .. new_{L-1}, U) with their counts.  Block (chunk, b) owns
+// words [chunk*kCompactWords, ...) of sequence b; the output bases of its lists are the
+// same popcounts over all earlier words of the sequence, recomputed from the masks
+// (re-read from L2).  Indices are staged in shared memory and written coalesced.
+constexpr int kSelMaxLayers = 8;
+
+__global__ void __launch_bounds__(kCompactThreads)
+select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, int Nw, int cap,
+                    uint32_t* __restrict__ U, uint32_t* __restrict__ nw, int32_t* __restrict__ idx_new,
+                    int32_t* __restrict__ cnt_new, size_t cstride, int32_t* __restrict__ idx_U,
+                    int32_t* __restrict__ cnt_U, int32_t* status) {
+  __shared__ int warp_tmp[32];
+  __shared__ int total;
+  __shared__ int sred[kSelMaxLayers + 1][kCompactThreads / 32];
+  __shared__ int32_t sidx[kCompactWords * 32];
+  const int b = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t* mb = mask + static_cast<size_t>(b) * Nw;
+  const int w0 = chunk * kCompactWords;
+  // bases: the lists' set bits in words [0, w0) of this sequence
+  int pc[kSelMaxLayers + 1];
+#pragma unroll
+  for (int j = 0; j <= kSelMaxLayers; ++j) pc[j] = 0;
+  auto count_word = [&](const uint32_t* m) {
+    uint32_t acc = 0;
+#pragma unroll
+    for (int l = 0; l < kSelMaxLayers; ++l) {
+      if (l < L) {
+        pc[l] += __popc(m[l] & ~acc);
+        acc |= m[l];
+      }
+    }
+    pc[kSelMaxLayers] += __popc(acc);
+  };
+  if ((Nw & 3) == 0 && (lstride & 3) == 0) {
+    for (int i = tid; i < w0 / 4; i += kCompactThreads) {
+      uint4 v[kSelMaxLayers];
+#pragma unroll
+      for (int l = 0; l < kSelMaxLayers; ++l)
+        if (l < L) v[l] = __ldg(reinterpret_cast<const uint4*>(mb + l * lstride) + i);
+      uint32_t m[kSelMaxLayers];
+#pragma unroll
+      for (int l = 0; l < kSelMaxLayers; ++l) m[l] = v[l].x;
+      count_word(m);
+#pragma unroll
+      for (int l = 0; l < kSelMaxLayers; ++l) m[l] = v[l].y;
+      count_word(m);
+#pragma unroll
+      for (int l = 0; l < kSelMaxLayers; ++l) m[l] = v[l].z;
+      count_word(m);
+#pragma unroll
+      for (int l = 0; l < kSelMaxLayers; ++l) m[l] = v[l].w;
+      count_word(m);
+    }
+  } else {
+    for (int i = tid; i < w0; i += kCompactThreads) {
+      uint32_t m[kSelMaxLayers];
+#pragma unroll
+      for (int l = 0; l < kSelMaxLayers; ++l) m[l] = l < L ? __ldg(mb + l * lstride + i) : 0u;
+      count_word(m);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j <= kSelMaxLayers; ++j) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) pc[j] += __shfl_xor_sync(0xffffffffu, pc[j], o);
+    if (lane == 0) sred[j][warp] = pc[j];
+  }
+  __syncthreads();
+  // own word
+  const int wi = w0 + tid;
+  uint32_t word[kSelMaxLayers + 1];
+  {
+    uint32_t acc = 0;
+#pragma unroll
+    for (int l = 0; l < kSelMaxLayers; ++l) {
+      word[l] = 0u;
+      if (l < L && wi < Nw) {
+        const uint32_t m = __ldg(mb + l * lstride + wi);
+        word[l] = m & ~acc;
+        acc |= m;
+        if (nw) nw[l * lstride + static_cast<size_t>(b) * Nw + wi] = word[l];
+      }
+    }
+    word[kSelMaxLayers] = acc;
+    if (U && wi < Nw) U[static_cast<size_t>(b) * Nw + wi] = acc;
+  }
+  const bool last = chunk == static_cast<int>(gridDim.x) - 1;
+#pragma unroll 1
+  for (int j = 0; j <= L; ++j) {
+    const int jj = j == L ? kSelMaxLayers : j;
+    int base = 0;
+    for (int w = 0; w < kCompactThreads / 32; ++w) base += sred[jj][w];
+    uint32_t bits = 0;
+#pragma unroll
+    for (int q = 0; q <= kSelMaxLayers; ++q)
+      if (q == jj) bits = word[q];
+    int pos = block_exclusive_scan(__popc(bits), warp_tmp, &total);
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      sidx[pos++] = wi * 32 + bit;
+    }
+    __syncthreads();
+    const int n = total;
+    int32_t* out = (j == L ? idx_U + static_cast<size_t>(b) * cap : idx_new + j * cstride * cap + static_cast<size_t>(b) * cap);
+    for (int i = tid; i < n; i += kCompactThreads)
+      if (base + i < cap) out[base + i] = sidx[i];
+    if (last && tid == 0) {
+      int32_t* cnt = j == L ? cnt_U + b : cnt_new + j * cstride + b;
+      *cnt = base + n;
+      if (base + n > cap) raise_status(status, LSA_ERR_CAPACITY);
+    }
+    __syncthreads();
+  }
+}
+
 // ------------------------------------------------------------------ top-k
 __device__ __forceinline__ uint32_t order_key(float x) {
   const uint32_t u = __float_as_uint(x);
@@ -347,6 +466,27 @@ int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, in
     ++launches;
   }
   return check_launch("compact", launches);
+}
+
+int launch_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* nw, int cap,
+                        int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
+                        cudaStream_t s) {
+  if (B == 0) return LSA_OK;
+  const int Nw = (N + 31) / 32;
+  const size_t lstride = static_cast<size_t>(B) * Nw;
+  constexpr int kSeqPerLaunch = 65535;   // the sequence index is gridDim.y
+  int launches = 0;
+  for (int b0 = 0; b0 < B; b0 += kSeqPerLaunch) {
+    const int nb = std::min(kSeqPerLaunch, B - b0);
+    const dim3 grid(std::max(1, (Nw + kCompactWords - 1) / kCompactWords), nb);
+    const size_t o = static_cast<size_t>(b0) * Nw;
+    select_fetch_kernel<<<grid, kCompactThreads, 0, s>>>(
+        mask + o, L, lstride, Nw, cap, U ? U + o : nullptr, nw ? nw + o : nullptr,
+        idx_new + static_cast<size_t>(b0) * cap, cnt_new + b0, static_cast<size_t>(B),
+        idx_U + static_cast<size_t>(b0) * cap, cnt_U + b0, status);
+    ++launches;
+  }
+  return check_launch("select_fetch", launches);
 }
 
 namespace {

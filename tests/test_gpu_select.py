@@ -98,6 +98,95 @@ def test_compact_capacity_overflow_sets_status():
         assert np.array_equal(idx[b].cpu().numpy(), e[:cap])
 
 
+def _select_fetch(marks, cap, want_words=True):
+    """lsa_select_fetch on layer marks [L][B][N] (bool); host copies of its outputs."""
+    L, B, N = marks.shape
+    Nw = (N + 31) // 32
+    mask = torch.from_numpy(O.pack_bits(marks).view(np.int32).copy()).cuda()
+    U = torch.full((B, Nw), -5, dtype=torch.int32, device="cuda") if want_words else None
+    new = torch.full((L, B, Nw), -5, dtype=torch.int32, device="cuda") if want_words else None
+    capd = max(cap, 1)
+    idx_new = torch.full((L, B, capd), -7, dtype=torch.int32, device="cuda")
+    cnt_new = torch.full((L, B), -7, dtype=torch.int32, device="cuda")
+    idx_U = torch.full((B, capd), -7, dtype=torch.int32, device="cuda")
+    cnt_U = torch.full((B,), -7, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lsa.lsa_select_fetch(B, L, N, mask, U, new, cap, idx_new, cnt_new, idx_U, cnt_U, st)
+    torch.cuda.synchronize()
+    out = dict(idx_new=idx_new.cpu().numpy(), cnt_new=cnt_new.cpu().numpy(), idx_U=idx_U.cpu().numpy(),
+               cnt_U=cnt_U.cpu().numpy(), status=int(st.item()))
+    if want_words:
+        out["U"] = C.unpack(U, N)
+        out["new"] = C.unpack(new, N)
+    return out
+
+
+@pytest.mark.parametrize("L,B,N,cap", [(3, 5, 3000, 3000), (1, 2, 33, 33), (3, 4, 262144, 262144),
+                                       (8, 3, 70001, 70001), (2, 3, 5000, 120)])
+def test_select_fetch_exact(L, B, N, cap):
+    """The fused union / new sets / fetch lists against the oracle's set operations, and
+    the capacity report when a list overflows."""
+    g = np.random.default_rng(L * 1000 + N)
+    dens = g.uniform(0.0, 0.35, size=(L, B, 1))
+    marks = g.random((L, B, N)) < dens
+    marks[:, 0, : min(N, 40)] = True                      # a dense head and an empty tail
+    if B > 2:
+        marks[:, -1, :] = False
+    out = _select_fetch(marks, cap)
+    over = False
+    for b in range(B):
+        Ue, news = O.or_union([marks[l, b] for l in range(L)])
+        assert np.array_equal(out["U"][b], Ue), b
+        e = O.compact(Ue)
+        assert out["cnt_U"][b] == e.size, b
+        assert np.array_equal(out["idx_U"][b, : min(cap, e.size)], e[:cap]), b
+        over |= e.size > cap
+        for l in range(L):
+            assert np.array_equal(out["new"][l, b], news[l]), (l, b)
+            e = O.compact(news[l])
+            assert out["cnt_new"][l, b] == e.size, (l, b)
+            assert np.array_equal(out["idx_new"][l, b, : min(cap, e.size)], e[:cap]), (l, b)
+            over |= e.size > cap
+    assert out["status"] == (lsa.LSA_ERR_CAPACITY if over else 0)
+
+
+def test_select_fetch_equals_the_separate_calls_without_word_outputs():
+    g = np.random.default_rng(3)
+    L, B, N = 3, 6, 40000
+    marks = g.random((L, B, N)) < 0.12
+    out = _select_fetch(marks, N, want_words=False)
+    Nw = (N + 31) // 32
+    U = torch.zeros(B, Nw, dtype=torch.int32, device="cuda")
+    for l in range(L):
+        nw = torch.zeros(B, Nw, dtype=torch.int32, device="cuda")
+        lsa.lsa_select_union(B, Nw, bits_tensor(marks[l]), U, nw)
+        idx = torch.full((B, N), -7, dtype=torch.int32, device="cuda")
+        cnt = torch.zeros(B, dtype=torch.int32, device="cuda")
+        lsa.lsa_compact(B, N, nw, N, idx, cnt)
+        torch.cuda.synchronize()
+        assert np.array_equal(cnt.cpu().numpy(), out["cnt_new"][l])
+        assert np.array_equal(idx.cpu().numpy(), out["idx_new"][l])
+    idx = torch.full((B, N), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(B, dtype=torch.int32, device="cuda")
+    lsa.lsa_compact(B, N, U, N, idx, cnt)
+    torch.cuda.synchronize()
+    assert np.array_equal(cnt.cpu().numpy(), out["cnt_U"])
+    assert np.array_equal(idx.cpu().numpy(), out["idx_U"])
+
+
+def test_select_fetch_more_sequences_than_one_launch():
+    g = np.random.default_rng(11)
+    L, B, N = 2, 70000, 100
+    marks = g.random((L, B, N)) < 0.2
+    out = _select_fetch(marks, N)
+    for b in range(0, B, 997):
+        Ue, news = O.or_union([marks[l, b] for l in range(L)])
+        assert np.array_equal(out["idx_U"][b, : out["cnt_U"][b]], O.compact(Ue)), b
+        for l in range(L):
+            assert np.array_equal(out["idx_new"][l, b, : out["cnt_new"][l, b]], O.compact(news[l])), (l, b)
+    assert (out["cnt_U"] == marks.any(axis=0).sum(axis=1)).all()
+
+
 def run_topk(idx_list, logits, k, N):
     L, B = logits.shape[0], len(idx_list)
     cap = max(1, max(len(x) for x in idx_list))
