@@ -205,6 +205,30 @@ int lsa_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int3
              void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * lsa_fine_score -- the backbone's native indexer scores the fetched subset for the
+ * current token ([SUMMARY] §2.1 hierarchical selection: once the critical subset is in
+ * GPU memory, the native Lightning Indexer makes a fine top-k choice inside it).  The
+ * pages do not print the native indexer's formula; the reading taken is the lookahead
+ * score's head-fused ReLU form with its own per-token query and keys, no bias or gate:
+ *     score[b][e] = kscale[b][e] * sum_h w[b][h] * ReLU(q[b][h] . khat[b][e])
+ * for every candidate e = idx[b][j], j < min(count[b], cap); other entries of score are
+ * not written.  Ranking the candidates with lsa_topk(B, 1, N, k, idx, cap, count, score,
+ * ...) then gives the fine top-k.
+ *   q [B][H][dI] (qdt: LSA_F32 or LSA_BF16), w [B][H] fp32, K [B][N][dI] (kdt: LSA_F32,
+ *   LSA_BF16 or LSA_E4M3 codes with kscale [B][N] fp32; NULL otherwise), idx [B][cap]
+ *   entries in [0, N) (others are skipped), count [B], score [B][N] fp32.
+ *   bf16 queries with H in {32, 64, 128, 256} and the key shapes of lsa_index_score run
+ *   on the tensor cores (key rows gathered by entry, four rows per TMA gather), other
+ *   shapes on the CUDA cores.  B * N < 2^31.  K 128-byte aligned; q, w, idx 16-byte.
+ * workspace: lsa_fine_score_workspace_bytes(B, H, dI, kdt) bytes, 256-byte aligned.
+ * ---------------------------------------------------------------------------------- */
+size_t lsa_fine_score_workspace_bytes(int B, int H, int dI, int kdt);
+
+int lsa_fine_score(int B, int N, int H, int dI, int qdt, const void* q, const float* w, int kdt, const void* K,
+                   const float* kscale, const int32_t* idx, int cap, const int32_t* count, float* score,
+                   int32_t* status, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * lsa_topk_noalloc -- lsa_topk without a workspace argument.  The pages have no
  * counterpart of this call: it exists for callers that cannot allocate device memory
  * when they call the library, such as a plugin inside a host framework that owns every

@@ -137,6 +137,17 @@ def lsa_topk(B, L, N, k, idx, cap, count, logit, topk, topk_count, workspace, st
                           _stream(stream)), "lsa_topk")
 
 
+def lsa_fine_score_workspace_bytes(B, H, dI, kdt) -> int:
+    return int(lib().lsa_fine_score_workspace_bytes(B, H, dI, kdt))
+
+
+def lsa_fine_score(B, N, H, dI, qdt, q, w, kdt, K, kscale, idx, cap, count, score, workspace, status=None,
+                   stream=None):
+    _check(lib().lsa_fine_score(B, N, H, dI, qdt, _p(q), _p(w), kdt, _p(K), _p(kscale), _p(idx), cap, _p(count),
+                                _p(score), _p(status), _p(workspace), 0 if workspace is None else workspace.numel(),
+                                _stream(stream)), "lsa_fine_score")
+
+
 def lsa_topk_noalloc(B, L, N, k, idx, cap, count, logit, topk, topk_count, stream=None):
     """lsa_topk with its scratch in the library's built-in device array (no workspace)."""
     _check(lib().lsa_topk_noalloc(B, L, N, k, _p(idx), cap, _p(count), _p(logit), _p(topk), _p(topk_count),

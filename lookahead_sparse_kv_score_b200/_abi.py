@@ -32,6 +32,9 @@ SIGNATURES = {
     "lsa_topk_workspace_bytes": (c_size_t, [c_int, c_int]),
     "lsa_topk": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
                          c_void_p, c_void_p, c_size_t, c_void_p]),
+    "lsa_fine_score_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
+    "lsa_fine_score": (c_int, [c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p,
+                               c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "lsa_topk_noalloc": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
                                  c_void_p, c_void_p]),
     "lsa_gather_cold": (c_int, [c_int, c_int, c_size_t, c_void_p, c_void_p, c_void_p, c_int, c_void_p,

@@ -274,6 +274,60 @@ int lsa_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uin
                              static_cast<cudaStream_t>(stream));
 }
 
+// Workspace of lsa_fine_score: query images, folded head weights, tile prefix.
+struct FineWs {
+  size_t qimg, wfold, tiles, total;
+};
+static FineWs fine_ws(int B, int H, int dI, int kdt) {
+  FineWs o{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t at = off; off = align_up(off + bytes, 1024); return at; };
+  o.qimg = take(static_cast<size_t>(B) * tc_image_bytes(H, dI, kdt));
+  o.wfold = take(static_cast<size_t>(B) * H * 4);
+  o.tiles = take((static_cast<size_t>(B) + 1) * 4);
+  o.total = off;
+  return o;
+}
+
+size_t lsa_fine_score_workspace_bytes(int B, int H, int dI, int kdt) {
+  if (B < 0 || H < 0 || dI < 0) return 0;
+  return fine_ws(B, H, dI, kdt).total + 256;
+}
+
+int lsa_fine_score(int B, int N, int H, int dI, int qdt, const void* q, const float* w, int kdt, const void* K,
+                   const float* kscale, const int32_t* idx, int cap, const int32_t* count, float* score,
+                   int32_t* status, void* workspace, size_t workspace_bytes, void* stream) {
+  const CallRange range("lsa_fine_score");
+  g_err[0] = 0;
+  if (B < 0 || N < 0 || H <= 0 || dI <= 0 || cap < 0) return fail(LSA_ERR_INVALID_ARG, "fine_score: bad size");
+  if (B == 0 || N == 0 || cap == 0) return LSA_OK;
+  if (qdt != LSA_F32 && qdt != LSA_BF16) return fail(LSA_ERR_UNSUPPORTED, "fine_score: query dtype %d", qdt);
+  if (kdt != LSA_F32 && kdt != LSA_BF16 && kdt != LSA_E4M3)
+    return fail(LSA_ERR_UNSUPPORTED, "fine_score: key dtype %d", kdt);
+  if (!q || !w || !K || !idx || !count || !score || (kdt == LSA_E4M3 && !kscale))
+    return fail(LSA_ERR_INVALID_ARG, "fine_score: null pointer (e4m3 keys need kscale)");
+  if (static_cast<long long>(B) * N > 0x7fffffffLL)
+    return fail(LSA_ERR_UNSUPPORTED, "fine_score: B*N = %lld rows (at most 2^31 - 1)", static_cast<long long>(B) * N);
+  const bool tc = tc_supported(H, dI, qdt, kdt);
+  if (!tc && (static_cast<size_t>(H) * dI + H) * 4 > 227 * 1024)
+    return fail(LSA_ERR_UNSUPPORTED, "fine_score: H*dI = %d too large for the CUDA-core path", H * dI);
+  if (!aligned(K, 128) || !aligned(q, 16) || !aligned(w, 16) || !aligned(idx, 16) || !aligned(count, 4) ||
+      !aligned(score, 4) || (kscale && !aligned(kscale, 4)))
+    return fail(LSA_ERR_INVALID_ARG, "fine_score: misaligned pointer (K 128 bytes, q, w, idx 16)");
+  const FineWs ws = fine_ws(B, H, dI, kdt);
+  if (tc && (!workspace || workspace_bytes < ws.total || !aligned(workspace, 256)))
+    return fail(LSA_ERR_NOMEM, "fine_score: workspace %zu bytes (need %zu)", workspace_bytes, ws.total);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  FineArgs fa{};
+  fa.B = B; fa.N = N; fa.H = H; fa.dI = dI; fa.qdt = qdt; fa.kdt = kdt; fa.cap = cap;
+  fa.q = q; fa.w = w; fa.K = K; fa.kscale = kscale; fa.idx = idx; fa.count = count; fa.score = score;
+  fa.qimg = tc ? base + ws.qimg : nullptr;
+  fa.wfold = tc ? reinterpret_cast<float*>(base + ws.wfold) : nullptr;
+  fa.tile_start = tc ? reinterpret_cast<int32_t*>(base + ws.tiles) : nullptr;
+  fa.status = status;
+  return launch_fine_score(fa, static_cast<cudaStream_t>(stream));
+}
+
 size_t lsa_topk_workspace_bytes(int B, int cap) {
   if (B < 0 || cap < 0) return 0;
   return align_up(static_cast<size_t>(B) * cap * 4, 256) + 256;

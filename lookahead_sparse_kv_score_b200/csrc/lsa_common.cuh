@@ -108,6 +108,26 @@ size_t tc_image_bytes(int H, int dI, int kdt);
 bool tc_supported(int H, int dI, int wdt, int kdt);
 int launch_score_tc(const TcArgs& a, cudaStream_t s);
 
+// Native-indexer fine score of gathered candidates (tensor cores when tc_supported,
+// else CUDA cores): score[b][idx[b][j]] for j < min(count[b], cap).
+struct FineArgs {
+  int B, N, H, dI, qdt, kdt, cap;
+  const void* q;            // [B][H][dI] qdt (f32 or bf16)
+  const float* w;           // [B][H]
+  const void* K;            // [B][N][dI] kdt
+  const float* kscale;      // [B][N] or null
+  const int32_t* idx;       // [B][cap]
+  const int32_t* count;     // [B]
+  float* score;             // [B][N]
+  uint8_t* qimg;            // workspace [B][img_bytes] (tensor-core path)
+  float* wfold;             // workspace [B][H]
+  int32_t* tile_start;      // workspace [B + 1]
+  int32_t* status;
+};
+int launch_fine_score(const FineArgs& a, cudaStream_t s);
+int launch_fine_score_tc(const FineArgs& a, cudaStream_t s);
+int launch_fine_score_simt(const FineArgs& a, cudaStream_t s);
+
 // Selection.
 int launch_union(int B, int Nw, const uint32_t* m, uint32_t* U, uint32_t* nw, cudaStream_t s);
 int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32_t* count,

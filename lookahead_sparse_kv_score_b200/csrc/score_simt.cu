@@ -88,7 +88,81 @@ int launch_k(const ScoreArgs& a, cudaStream_t st) {
   return check_launch("score_simt");
 }
 
+// Gathered candidates (the native indexer's fine score): thread j of sequence b scores
+// entry e = idx[b][j] for j < min(count[b], cap) and writes score[b][e].
+template <typename KT, typename QT>
+__global__ void __launch_bounds__(kThreads)
+fine_simt_kernel(const QT* __restrict__ q, const float* __restrict__ w, const KT* __restrict__ K,
+                 const float* __restrict__ kscale, const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
+                 int cap, int N, int H, int dI, float* __restrict__ score) {
+  extern __shared__ float sm[];
+  float* qs = sm;                 // [H][dI]
+  float* ws = sm + H * dI;        // [H]
+  const int b = blockIdx.y;
+  const int n = min(count[b], cap);
+  if (static_cast<int>(blockIdx.x) * kThreads >= n) return;
+  for (int i = threadIdx.x; i < H * dI; i += kThreads) qs[i] = load_elem(q, static_cast<size_t>(b) * H * dI + i);
+  for (int i = threadIdx.x; i < H; i += kThreads) ws[i] = w[static_cast<size_t>(b) * H + i];
+  __syncthreads();
+  const int j = blockIdx.x * kThreads + threadIdx.x;
+  if (j >= n) return;
+  const int e = idx[static_cast<size_t>(b) * cap + j];
+  if (e < 0 || e >= N) return;
+  const KT* kr = K + (static_cast<size_t>(b) * N + e) * dI;
+  float z = 0.f;
+  for (int h0 = 0; h0 < H; h0 += kHeadChunk) {
+    const int hn = min(kHeadChunk, H - h0);
+    float acc[kHeadChunk];
+#pragma unroll
+    for (int t = 0; t < kHeadChunk; ++t) acc[t] = 0.f;
+    for (int d = 0; d < dI; ++d) {
+      const float kd = load_elem(kr, d);
+#pragma unroll
+      for (int t = 0; t < kHeadChunk; ++t)
+        if (t < hn) acc[t] = fmaf(qs[(h0 + t) * dI + d], kd, acc[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < kHeadChunk; ++t)
+      if (t < hn) z = fmaf(ws[h0 + t], fmaxf(acc[t], 0.f), z);
+  }
+  if (kscale != nullptr) z *= kscale[static_cast<size_t>(b) * N + e];
+  score[static_cast<size_t>(b) * N + e] = z;
+}
+
+template <typename KT, typename QT>
+int launch_fine_k(const FineArgs& a, cudaStream_t st) {
+  const dim3 grid((a.cap + kThreads - 1) / kThreads, a.B);
+  const size_t smem = (static_cast<size_t>(a.H) * a.dI + a.H) * sizeof(float);
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(fine_simt_kernel<KT, QT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  fine_simt_kernel<KT, QT><<<grid, kThreads, smem, st>>>(static_cast<const QT*>(a.q), a.w,
+                                                         static_cast<const KT*>(a.K), a.kscale, a.idx, a.count, a.cap,
+                                                         a.N, a.H, a.dI, a.score);
+  return check_launch("fine_score_simt");
+}
+
+template <typename KT>
+int launch_fine_q(const FineArgs& a, cudaStream_t st) {
+  return a.qdt == LSA_BF16 ? launch_fine_k<KT, __nv_bfloat16>(a, st) : launch_fine_k<KT, float>(a, st);
+}
+
 }  // namespace
+
+int launch_fine_score_simt(const FineArgs& a, cudaStream_t s) {
+  if (a.N == 0 || a.B == 0 || a.cap == 0) return LSA_OK;
+  switch (a.kdt) {
+    case LSA_F32: return launch_fine_q<float>(a, s);
+    case LSA_BF16: return launch_fine_q<__nv_bfloat16>(a, s);
+    case LSA_E4M3: return launch_fine_q<uint8_t>(a, s);
+  }
+  return fail(LSA_ERR_UNSUPPORTED, "fine_score: key dtype %d", a.kdt);
+}
+
+int launch_fine_score(const FineArgs& a, cudaStream_t s) {
+  if (a.N == 0 || a.B == 0 || a.cap == 0) return LSA_OK;
+  if (tc_supported(a.H, a.dI, a.qdt, a.kdt)) return launch_fine_score_tc(a, s);
+  return launch_fine_score_simt(a, s);
+}
 
 int launch_score_simt(const ScoreArgs& a, cudaStream_t s) {
   if (a.N == 0 || a.B == 0 || a.nL == 0) return LSA_OK;

@@ -109,6 +109,14 @@ __host__ __device__ inline TcLayout tc_layout(int H, int dI, bool fp8) {
 
 struct TcParams {
   int B, N, H, dI, l0, nUnits, tiles_per_unit;
+  // Gathered mode (the fine indexer): unit b scores the candidates idx[b][0..n_b),
+  // n_b = min(count[b], cap), in tiles of 128; tile_start [nUnits + 1] is the prefix of
+  // the units' tile counts.  Key rows are gathered by entry; logit is written at the
+  // entry (logit[b][idx[b][j]]); no mask, score or bias.
+  const int32_t* idx;      // [B][cap] or null
+  const int32_t* count;    // [B]
+  const int32_t* tile_start;
+  int cap;
   const uint8_t* qimg;     // [L][B][img_bytes]
   const float* wfold;      // [L][B][H]
   const float* bias;       // [L]
@@ -148,7 +156,7 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t t0, uint32_t t1, float (&v0
 // Local tile i uses accumulator i % kNumAcc, drained by epilogue group i % kNumAcc
 // (warps 4+4g .. 7+4g).  The pipelines share the query slots (loaded by producer 0 and
 // released by both MMA issuers) and nothing else.
-template <bool kFp8, int kH, int kKSteps>
+template <bool kFp8, int kH, int kKSteps, bool kGather>
 __global__ void __launch_bounds__(TcShape<kFp8, kH>::kThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
   using S = TcShape<kFp8, kH>;
@@ -188,26 +196,59 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const long long T = static_cast<long long>(p.nUnits) * p.tiles_per_unit;
+  // Tiles of a unit, the unit holding a flat tile index, and the walk to a later tile.
+  auto tiles_of = [&](int u) -> int {
+    if constexpr (kGather) return __ldg(p.tile_start + u + 1) - __ldg(p.tile_start + u);
+    else return p.tiles_per_unit;
+  };
+  auto unit_of = [&](long long t) -> int {   // the last unit whose first tile is <= t
+    if constexpr (kGather) {
+      int lo = 0, hi = p.nUnits - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(p.tile_start + mid) <= t) lo = mid; else hi = mid - 1;
+      }
+      return lo;
+    } else {
+      return static_cast<int>(t / p.tiles_per_unit);
+    }
+  };
+  auto first_tile = [&](int u) -> long long {
+    if constexpr (kGather) return __ldg(p.tile_start + u);
+    else return static_cast<long long>(u) * p.tiles_per_unit;
+  };
+  auto advance = [&](int& unit, int& tile, int by) {
+    tile += by;
+    if constexpr (kGather) {
+      while (unit < p.nUnits && tile >= tiles_of(unit)) { tile -= tiles_of(unit); ++unit; }
+    } else {
+      while (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
+    }
+  };
+  const long long T = kGather ? static_cast<long long>(__ldg(p.tile_start + p.nUnits))
+                              : static_cast<long long>(p.nUnits) * p.tiles_per_unit;
   const long long t_begin = T * blockIdx.x / gridDim.x, t_end = T * (blockIdx.x + 1) / gridDim.x;
   const int n_local = static_cast<int>(t_end - t_begin);
-  const int unit0 = static_cast<int>(t_begin / p.tiles_per_unit);
-  const int tile0 = static_cast<int>(t_begin - static_cast<long long>(unit0) * p.tiles_per_unit);
+  const int unit0 = n_local > 0 ? unit_of(t_begin) : 0;
+  const int tile0 = n_local > 0 ? static_cast<int>(t_begin - first_tile(unit0)) : 0;
   const int Nw = (p.N + 31) / 32;
   const int uabs0 = p.l0 * p.B;
 
   // Local tile i of this CTA belongs to unit (i + t_begin) / tiles_per_unit; query slot
   // k = unit - unit0 of every unit in the range is loaded once by producer 0 and
   // released by both MMA issuers, in unit order.
-  const int k_last = n_local > 0 ? static_cast<int>((t_end - 1) / p.tiles_per_unit) - unit0 : -1;
-  if (warp < 2 && lane == 0) {
+  const int k_last = n_local > 0 ? unit_of(t_end - 1) - unit0 : -1;
+  if (warp < 2 && (kGather || lane == 0)) {
     // ---------------------------------------------------------------- producers
     // Producer pp loads the key tiles of parity pp (local tiles pp, pp+2, ...) into
     // stages [pp*S2, pp*S2+S2); producer 0 also loads the query image of every unit.
+    // Tiled mode: lane 0 alone, one TMA box per 128-byte K chunk.  Gathered mode: the
+    // whole warp, lane l fetching candidates 4l .. 4l+3 of the tile with one four-row
+    // gather per K chunk; lane 0 keeps the barriers.
     const int pp = warp;
     const uint64_t policy = evict_first_policy();
-    int unit = unit0, tile = tile0 + pp;
-    if (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
+    int unit = unit0, tile = tile0;
+    advance(unit, tile, pp);
     int kq = -1;                              // last query slot loaded (producer 0)
     auto load_q_through = [&](int k_to) -> bool {
       while (kq < k_to) {
@@ -224,26 +265,48 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
     uint32_t ph = 0;
     bool ok = true;
     for (int i = pp; i < n_local; i += 2) {
-      if (pp == 0 && !(ok = load_q_through(unit - unit0))) break;
       const int st = pp * S2 + s;
-      if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag))) break;
-      mbar_expect_tx(&full[st], lay.a_bytes);
+      if (lane == 0) {
+        if (pp == 0) ok = load_q_through(unit - unit0);
+        if (ok) ok = mbar_wait(&empty[st], ph ^ 1, abort_flag);
+        if (ok) mbar_expect_tx(&full[st], lay.a_bytes);
+      }
+      if constexpr (kGather) ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
       uint8_t* dst = a_ring + static_cast<size_t>(st) * lay.a_bytes;
+      if constexpr (kGather) {
+        const int32_t* ib = p.idx + static_cast<size_t>(unit) * p.cap;
+        const int nb = min(__ldg(p.count + unit), p.cap);
+        const int first = __ldg(ib + tile * kTileM);      // a tile's first candidate always exists
+        int r[4];
 #pragma unroll
-      for (int c = 0; c < kKSteps / 4; ++c)     // 128-byte K chunks of a key row
-        tma_load_3d(dst + c * (kTileM * 128), &kmap, c * (kFp8 ? 128 : 64), tile * kTileM, uabs0 + unit,
-                    &full[st], policy);
+        for (int e = 0; e < 4; ++e) {
+          const int jj = tile * kTileM + 4 * lane + e;
+          int ent = jj < nb ? __ldg(ib + jj) : first;       // rows past the list repeat a real row
+          ent = min(max(ent, 0), p.N - 1);
+          r[e] = (uabs0 + unit) * p.N + ent;
+        }
+#pragma unroll
+        for (int c = 0; c < kKSteps / 4; ++c)
+          tma_gather4_2d(dst + c * (kTileM * 128) + lane * 4 * 128, &kmap, c * (kFp8 ? 128 : 64), r[0], r[1], r[2],
+                         r[3], &full[st], policy);
+      } else {
+#pragma unroll
+        for (int c = 0; c < kKSteps / 4; ++c)     // 128-byte K chunks of a key row
+          tma_load_3d(dst + c * (kTileM * 128), &kmap, c * (kFp8 ? 128 : 64), tile * kTileM, uabs0 + unit,
+                      &full[st], policy);
+      }
       ++j;
       if (++s == S2) { s = 0; ph ^= 1; }
-      tile += 2;
-      if (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
-      if (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
+      advance(unit, tile, 2);
     }
-    if (pp == 0 && ok) load_q_through(k_last);
-    // drain: every key tile this thread issued has landed before the CTA exits
-    for (int jj = j > S2 ? j - S2 : 0; jj < j; ++jj) {
-      volatile int no_abort = 0;
-      if (!mbar_wait(&full[pp * S2 + jj % S2], (jj / S2) & 1, &no_abort)) break;
+    if (lane == 0) {
+      if (pp == 0 && ok) load_q_through(k_last);
+      // drain: every key tile this warp issued has landed before the CTA exits
+      for (int jj = j > S2 ? j - S2 : 0; jj < j; ++jj) {
+        volatile int no_abort = 0;
+        if (!mbar_wait(&full[pp * S2 + jj % S2], (jj / S2) & 1, &no_abort)) break;
+      }
     }
   } else if ((warp == 2 || warp == 3) && lane == 0) {
     // ---------------------------------------------------------------- MMA issuers
@@ -251,8 +314,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
     const uint32_t idesc = instr_desc(kFp8, kN);
     const uint64_t dhi = smem_desc(0);
     const uint32_t a_ring_u = smem_u32(a_ring), q_slot_u = smem_u32(q_slot);
-    int unit = unit0, tile = tile0 + pp;
-    if (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
+    int unit = unit0, tile = tile0;
+    advance(unit, tile, pp);
     int kq = -1;                              // query slot in use
     // release the current slot and acquire every later one through k_to, in order
     auto acquire_q_through = [&](int k_to) -> bool {
@@ -286,9 +349,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
       mma_commit(&tfull[a]);
       aph ^= 1u << a;
       if (++s == S2) { s = 0; ph ^= 1; }
-      tile += 2;
-      if (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
-      if (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
+      advance(unit, tile, 2);
     }
     if (ok && acquire_q_through(k_last) && kq >= 0) mma_commit(&qempty[kq & 1]);
     // drain: all MMAs issued by this thread have completed
@@ -300,38 +361,46 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
     const int g = (warp - 4) >> 2;            // accumulator: local tiles i = g, g + kNumAcc, ...
     const int quad = warp & 3;                // TMEM lane quadrant of this warp
     const int row = quad * 32 + lane;
-    int unit = unit0, tile = tile0 + g;
-    while (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
+    int unit = unit0, tile = tile0;
+    advance(unit, tile, g);
     int cur = -1;
     float bias_l = 0.f;
     const float4* wf4 = nullptr;
     uint32_t aph = 0;
+    // Gathered mode: the entry this thread's row scores in a tile (the candidate's entry
+    // index, -1 past the unit's list); tiled mode: the row of the tile itself.
+    auto entry_of = [&](int u, int t) -> int {
+      const int jj = t * kTileM + row;
+      return jj < min(__ldg(p.count + u), p.cap) ? __ldg(p.idx + static_cast<size_t>(u) * p.cap + jj) : -1;
+    };
+    int e_next = 0;
+    if constexpr (kGather) e_next = g < n_local ? entry_of(unit, tile) : -1;
     // per-entry scale of the next tile, loaded one tile ahead
     float ks_next = 1.f;
     if (kFp8 && g < n_local) {
-      const int n = tile * kTileM + row;
-      if (n < p.N) ks_next = __ldg(p.kscale + static_cast<size_t>(uabs0 + unit) * p.N + n);
+      const int n = kGather ? e_next : tile * kTileM + row;
+      if (n >= 0 && n < p.N) ks_next = __ldg(p.kscale + static_cast<size_t>(uabs0 + unit) * p.N + n);
     }
     for (int i = g; i < n_local; i += kNumAcc) {
       const size_t uabs = static_cast<size_t>(uabs0 + unit);
       if (unit != cur) {
         cur = unit;
-        bias_l = __ldg(p.bias + p.l0 + unit / p.B);
+        bias_l = p.bias ? __ldg(p.bias + p.l0 + unit / p.B) : 0.f;
         wf4 = reinterpret_cast<const float4*>(p.wfold + uabs * kH);
       }
       const int n0 = tile * kTileM;
-      const int n = n0 + row;
-      const bool valid = n < p.N;
+      const int n = kGather ? e_next : n0 + row;
+      const bool valid = n >= 0 && n < p.N;
       const float ks = ks_next;
-      // advance to this group's next tile and prefetch its scale
-      const int cur_tile = tile;
-      tile += kNumAcc;
-      while (tile >= p.tiles_per_unit) { tile -= p.tiles_per_unit; ++unit; }
-      if (kFp8 && i + kNumAcc < n_local) {
-        const int nn = tile * kTileM + row;
-        ks_next = nn < p.N ? __ldg(p.kscale + static_cast<size_t>(uabs0 + unit) * p.N + nn) : 1.f;
+      // advance to this group's next tile and prefetch its scale (and entry)
+      advance(unit, tile, kNumAcc);
+      if (i + kNumAcc < n_local) {
+        if constexpr (kGather) e_next = entry_of(unit, tile);
+        if (kFp8) {
+          const int nn = kGather ? e_next : tile * kTileM + row;
+          ks_next = nn >= 0 && nn < p.N ? __ldg(p.kscale + static_cast<size_t>(uabs0 + unit) * p.N + nn) : 1.f;
+        }
       }
-      (void)cur_tile;
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[g], aph, abort_flag))) break;
       aph ^= 1;
       tc_fence_after();
@@ -379,9 +448,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
         if (p.logit) p.logit[uabs * p.N + n] = z;
         if (p.score) p.score[uabs * p.N + n] = sigmoid_f(z);
       }
-      const unsigned bits = __ballot_sync(0xffffffffu, valid && z >= 0.f);
-      const int word = (n0 + quad * 32) >> 5;
-      if (lane == 0 && word < Nw) p.mask[uabs * Nw + word] = bits;
+      if (p.mask) {
+        const unsigned bits = __ballot_sync(0xffffffffu, valid && z >= 0.f);
+        const int word = (n0 + quad * 32) >> 5;
+        if (lane == 0 && word < Nw) p.mask[uabs * Nw + word] = bits;
+      }
     }
   }
   tc_fence_before();
@@ -460,7 +531,13 @@ __global__ void build_qimg_fp8_kernel(const __nv_bfloat16* __restrict__ q, const
 // ------------------------------------------------------------------ tensor map
 template <bool kFp8, int kH, int kKSteps>
 int launch_kernel(const CUtensorMap& map, const TcParams& p, const TcLayout& lay, int grid, cudaStream_t st) {
-  auto kern = score_tc_kernel<kFp8, kH, kKSteps>;
+  if (p.idx != nullptr) {
+    auto kern = score_tc_kernel<kFp8, kH, kKSteps, true>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.smem);
+    kern<<<grid, TcShape<kFp8, kH>::kThreads, lay.smem, st>>>(map, p);
+    return check_launch("fine_score_tc");
+  }
+  auto kern = score_tc_kernel<kFp8, kH, kKSteps, false>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.smem);
   kern<<<grid, TcShape<kFp8, kH>::kThreads, lay.smem, st>>>(map, p);
   return check_launch("score_tc");
@@ -494,7 +571,74 @@ int launch_h(const CUtensorMap& map, const TcParams& p, const TcLayout& lay, int
   return fail(LSA_ERR_UNSUPPORTED, "score_tc: H=%d", p.H);
 }
 
+// tile_start[b] = sum over b' < b of ceil(min(count[b'], cap) / 128), b = 0..B (one block).
+__global__ void tile_prefix_kernel(const int32_t* __restrict__ count, int B, int cap, int32_t* __restrict__ tile_start) {
+  __shared__ int wsum[32];
+  __shared__ int carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int b0 = 0; b0 < B; b0 += blockDim.x) {
+    const int b = b0 + tid;
+    const int n = b < B ? min(max(count[b], 0), cap) : 0;
+    const int t = (n + kTileM - 1) / kTileM;
+    int incl = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int before = carry;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    if (b < B) tile_start[b] = before + incl - t;
+    __syncthreads();
+    if (tid == blockDim.x - 1) carry = before + incl;
+    __syncthreads();
+  }
+  if (tid == 0) tile_start[B] = carry;
+}
+
 }  // namespace
+
+int launch_fine_score_tc(const FineArgs& a, cudaStream_t st) {
+  const bool fp8 = a.kdt == LSA_E4M3;
+  const TcLayout lay = tc_layout(a.H, a.dI, fp8);
+  const dim3 ig(fp8 ? (a.H + 7) / 8 : (a.H * a.dI / 8 + 255) / 256, a.B);
+  if (fp8)
+    build_qimg_fp8_kernel<<<ig, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.q), a.w, a.B, a.H, a.dI, 0,
+                                              a.qimg, a.wfold);
+  else
+    build_qimg_bf16_kernel<<<ig, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.q), a.w, a.B, a.H, a.dI, 0,
+                                               a.qimg, a.wfold);
+  tile_prefix_kernel<<<1, 1024, 0, st>>>(a.count, a.B, a.cap, a.tile_start);
+  int rc = check_launch("fine_score/query image and tile prefix", 2);
+  if (rc != LSA_OK) return rc;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(LSA_ERR_CUDA, "fine_score: cuTensorMapEncodeTiled unavailable");
+  CUtensorMap map;
+  const int esz = fp8 ? 1 : 2;
+  // rows of all sequences' keys, one row per box: the four-row gathers pick them by entry
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.dI), static_cast<cuuint64_t>(a.B) * a.N};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.dI) * esz};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), 1};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult cr = enc(&map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                          const_cast<void*>(a.K), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return fail(LSA_ERR_CUDA, "fine_score: tensor map encode failed (%d)", (int)cr);
+  TcParams p{};
+  p.B = a.B; p.N = a.N; p.H = a.H; p.dI = a.dI; p.l0 = 0; p.nUnits = a.B; p.tiles_per_unit = 0;
+  p.qimg = a.qimg; p.wfold = a.wfold; p.bias = nullptr; p.kscale = a.kscale;
+  p.mask = nullptr; p.logit = a.score; p.score = nullptr; p.status = a.status;
+  p.idx = a.idx; p.count = a.count; p.tile_start = a.tile_start; p.cap = a.cap;
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // the tile count is on the device: one CTA per SM, each takes an equal share of it
+  return fp8 ? launch_h<true>(map, p, lay, sms, st) : launch_h<false>(map, p, lay, sms, st);
+}
 
 bool tc_supported(int H, int dI, int wdt, int kdt) {
   if (wdt != LSA_BF16) return false;

@@ -39,6 +39,7 @@ from . import rng
 _S_H, _S_WDOWN, _S_WUP, _S_WW, _S_FRAC, _S_PLANT, _S_KNOISE, _S_COLD = range(1, 9)
 _S_VOTE_X, _S_VOTE_BOOST_SET, _S_VOTE_BOOST_LAYERS, _S_VOTE_NLAYERS, _S_POS_H = range(20, 25)
 _S_DRIFT = 30
+_S_FINE_Q, _S_FINE_W = 40, 41
 
 E4M3_MAX = 448.0
 
@@ -232,6 +233,20 @@ def keys(w: ScoreWorkload, b: int, l: int, direction, start: int = 0, n: int | N
     if w.kdtype == "e4m3":
         return encode_e4m3(x)
     return _to_storage(x, w.kdtype), None
+
+
+def fine_query(w: ScoreWorkload, device="cpu"):
+    """The backbone indexer's per-token query of each sequence for the fine selection
+    inside the fetched subset: (q_f [B][H][dI] bf16 ~ N(0, 1), w_f [B][H] fp32 ~ N(0, 1)).
+    The fine keys are a [B][N][dI] key array drawn like K_IComp (the benchmark reuses
+    layer 0's keys for them)."""
+    q = torch.empty(w.B, w.H, w.dI, dtype=torch.bfloat16, device=device)
+    wv = torch.empty(w.B, w.H, dtype=torch.float32, device=device)
+    for b in range(w.B):
+        q[b] = _to_storage(rng.normal(rng.stream_key(w.seed, _S_FINE_Q, b), rng.arange(w.H * w.dI, device=device)),
+                           "bf16").reshape(w.H, w.dI)
+        wv[b] = rng.normal(rng.stream_key(w.seed, _S_FINE_W, b), rng.arange(w.H, device=device)).to(torch.float32)
+    return q, wv
 
 
 # ----------------------------------------------------------------------------- cold pool
