@@ -31,13 +31,31 @@ def bf16(x):
     return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16)
 
 
-def problem(seed, P, N, D, r, H, dI, pos=0.08):
+# Head weights drawn N(0, 1/D) scaled by W_SCALE: the logits then have a spread of a few
+# units (z ~ 64 * W_SCALE * 8 for H = 64, dI = 128) instead of ~64, so that nearly every
+# (position, entry) pair lies inside the probability clamp |z| < ln(2^20 - 1) and the
+# gradient comparison exercises the unclamped path; a few pairs still reach the clamp.
+W_SCALE = 1.0 / 16
+Z_CLAMP = float(np.log(2.0 ** 20 - 1))
+
+
+def problem(seed, P, N, D, r, H, dI, pos=0.08, w_scale=W_SCALE):
     g = np.random.default_rng(seed)
     t = dict(h=bf16(g.standard_normal((P, D))), Wd=bf16(g.standard_normal((D, r)) / np.sqrt(D)),
-             Wu=bf16(g.standard_normal((r, H * dI)) / np.sqrt(r)), Ww=bf16(g.standard_normal((D, H)) / np.sqrt(D)),
+             Wu=bf16(g.standard_normal((r, H * dI)) / np.sqrt(r)),
+             Ww=bf16(g.standard_normal((D, H)) / np.sqrt(D) * w_scale),
              K=bf16(g.standard_normal((N, dI))))
     y = g.random((P, N)) < pos
     return {k: v.double().numpy() for k, v in t.items()}, t, y
+
+
+def clamped_fraction(f, bias, H, dI, n=2048):
+    """Share of (position, entry) pairs over the first n entries whose probability the
+    loss clamps (zero gradient there), from the oracle's projection and score."""
+    K = f["K"][:n]
+    z = np.stack([O.head_fused_logits(*O.project_query(f["h"][p], f["Wd"], f["Wu"], f["Ww"], H, dI, True), bias, K)
+                  for p in range(f["h"].shape[0])])
+    return float((np.abs(z) > Z_CLAMP).mean())
 
 
 def oracle_forward(f, H, dI):
@@ -97,6 +115,7 @@ def check(got, exp_grads, bnd, exp_loss):
 def test_train_step_matches_oracle(H, dI, P):
     D, r, N, bias, gamma = 256, 64, 3001, -1.5, 2.0
     f, t, y = problem(H + dI, P, N, D, r, H, dI)
+    assert clamped_fraction(f, bias, H, dI) < 0.1
     c, q, w = oracle_forward(f, H, dI)
     bce, fl, grads = T.loss_and_grads(f["h"], f["Wd"], f["Wu"], f["Ww"], bias, f["K"], y, H, dI, gamma, True)
     got = run_gpu(t, y, bias, gamma, H, dI, c, q, w)
@@ -127,6 +146,7 @@ def test_train_step_full_size_against_chunked_oracle():
     (each with the full normalisation) and the chunk results are added."""
     H, dI, P, D, r, N = 64, 128, 64, 4096, 512, 131072
     f, t, y = problem(9, P, N, D, r, H, dI, pos=0.01)
+    assert clamped_fraction(f, -2.0, H, dI) < 0.1
     c, q, w = oracle_forward(f, H, dI)
     got = run_gpu(t, y, -2.0, 2.0, H, dI, c, q, w)
     grads = {"W_up": 0.0, "W_down": 0.0, "W_w": 0.0, "b": 0.0}

@@ -2,6 +2,8 @@
 focal loss) with the fp64 oracle.  Entries whose nucleus membership lies within the
 summation tolerance of the top-p boundary are excluded from exact comparison."""
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import pytest
@@ -152,7 +154,9 @@ def test_vote_one_hot_and_theta_special_cases():
     assert not g5.any()                                              # theta > L: no label
 
 
-def test_vote_full_size_sampled_positions():
+def test_vote_full_size_every_position():
+    """The full vote workload (24 layers x 64 positions x 2^17 logits) in one call; every
+    position's counts and labels against the oracle (positions checked on a thread pool)."""
     v = W.VOTE_WORKLOADS["vote_labels_l24_p64_n131072"]
     x = torch.empty(v.L, v.P, v.N, dtype=torch.float32, device="cuda")
     for p in range(v.P):
@@ -165,14 +169,19 @@ def test_vote_full_size_sampled_positions():
     ws = lsa.workspace(lsa.lsa_vote_labels_workspace_bytes(v.L, v.P, v.N))
     lsa.lsa_vote_labels(v.L, v.P, v.N, x, v.top_p, v.theta, golden, counts, None, v.gamma, None, ws)
     torch.cuda.synchronize()
-    for p in (0, 31, 63):
-        xp = x[:, p:p + 1].cpu().numpy()
-        gp = C.unpack(golden[p:p + 1], v.N)
-        cp = counts[p:p + 1].cpu().numpy().astype(np.int64)
-        golden_o, _ = check_vote(xp, v.top_p, v.theta, gp, cp)
+    x_h = x.cpu().numpy()
+    g_h = C.unpack(golden, v.N)
+    c_h = counts.cpu().numpy().astype(np.int64)
+
+    def one(p):
+        golden_o, _ = check_vote(x_h[:, p:p + 1], v.top_p, v.theta, g_h[p:p + 1], c_h[p:p + 1])
         # the boosted entries (shared by >= 3 layers) dominate the labels
         bs = W.vote_boost_set(v, p).numpy()
-        assert golden_o[0, bs].mean() > 0.9
+        assert golden_o[0, bs].mean() > 0.9, p
+        return p
+
+    with ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as ex:
+        assert sorted(ex.map(one, range(v.P))) == list(range(v.P))
 
 
 def test_vote_loss_parity():
