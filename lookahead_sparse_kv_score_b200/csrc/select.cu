@@ -131,7 +131,8 @@ compact_kernel(const uint32_t* __restrict__ bits, int Nw, int cap, int32_t* __re
 // L + 1 fetch lists (new_0 .. new_{L-1}, U) with their counts.  Block (chunk, b) owns
 // words [chunk*kCompactWords, ...) of sequence b; the output bases of its lists are the
 // same popcounts over all earlier words of the sequence, recomputed from the masks
-// (re-read from L2).  Indices are staged in shared memory and written coalesced.
+// (re-read from L2).  Each thread writes its own word's indices; a warp's threads cover
+// one contiguous run of every list.
 constexpr int kSelMaxLayers = 8;
 
 __global__ void __launch_bounds__(kCompactThreads)
@@ -139,10 +140,8 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
                     uint32_t* __restrict__ U, uint32_t* __restrict__ nw, int32_t* __restrict__ idx_new,
                     int32_t* __restrict__ cnt_new, size_t cstride, int32_t* __restrict__ idx_U,
                     int32_t* __restrict__ cnt_U, int32_t* status) {
-  __shared__ int warp_tmp[32];
-  __shared__ int total;
   __shared__ int sred[kSelMaxLayers + 1][kCompactThreads / 32];
-  __shared__ int32_t sidx[kCompactWords * 32];
+  __shared__ int wsum[kSelMaxLayers + 1][kCompactThreads / 32];
   const int b = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t* mb = mask + static_cast<size_t>(b) * Nw;
   const int w0 = chunk * kCompactWords;
@@ -215,32 +214,50 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
     if (U && wi < Nw) U[static_cast<size_t>(b) * Nw + wi] = acc;
   }
   const bool last = chunk == static_cast<int>(gridDim.x) - 1;
+  // every list's offsets for the block in one pass: warp prefix sums of the popcounts,
+  // one barrier, then the warps' bases; each thread writes its word's indices directly
+  // (a warp's threads cover one contiguous run of each list)
+  int incl[kSelMaxLayers + 1];
+#pragma unroll
+  for (int q = 0; q <= kSelMaxLayers; ++q) {
+    const int v = (q < L || q == kSelMaxLayers) ? __popc(word[q]) : 0;
+    incl[q] = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl[q], o);
+      if (lane >= o) incl[q] += t;
+    }
+    if (lane == 31) wsum[q][warp] = incl[q];
+  }
+  __syncthreads();
 #pragma unroll 1
   for (int j = 0; j <= L; ++j) {
     const int jj = j == L ? kSelMaxLayers : j;
-    int base = 0;
-    for (int w = 0; w < kCompactThreads / 32; ++w) base += sred[jj][w];
+    int base = 0, before = 0, total = 0;
+    for (int w = 0; w < kCompactThreads / 32; ++w) {
+      base += sred[jj][w];
+      const int ws = wsum[jj][w];
+      before += w < warp ? ws : 0;
+      total += ws;
+    }
     uint32_t bits = 0;
+    int inc = 0;
 #pragma unroll
     for (int q = 0; q <= kSelMaxLayers; ++q)
-      if (q == jj) bits = word[q];
-    int pos = block_exclusive_scan(__popc(bits), warp_tmp, &total);
+      if (q == jj) { bits = word[q]; inc = incl[q]; }
+    int pos = base + before + inc - __popc(bits);
+    int32_t* out = (j == L ? idx_U + static_cast<size_t>(b) * cap : idx_new + j * cstride * cap + static_cast<size_t>(b) * cap);
     while (bits) {
       const int bit = __ffs(bits) - 1;
       bits &= bits - 1;
-      sidx[pos++] = wi * 32 + bit;
+      if (pos < cap) out[pos] = wi * 32 + bit;
+      ++pos;
     }
-    __syncthreads();
-    const int n = total;
-    int32_t* out = (j == L ? idx_U + static_cast<size_t>(b) * cap : idx_new + j * cstride * cap + static_cast<size_t>(b) * cap);
-    for (int i = tid; i < n; i += kCompactThreads)
-      if (base + i < cap) out[base + i] = sidx[i];
     if (last && tid == 0) {
       int32_t* cnt = j == L ? cnt_U + b : cnt_new + j * cstride + b;
-      *cnt = base + n;
-      if (base + n > cap) raise_status(status, LSA_ERR_CAPACITY);
+      *cnt = base + total;
+      if (base + total > cap) raise_status(status, LSA_ERR_CAPACITY);
     }
-    __syncthreads();
   }
 }
 
@@ -252,19 +269,21 @@ __device__ __forceinline__ uint32_t order_key(float x) {
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kTopkSmemKeys = 49152;   // keys of one CTA's candidate slice held in shared memory
-constexpr int kSubHists = 16;          // digit sub-histograms, one per pair of warps
+constexpr int kTopkSmemKeys = 45056;   // keys of one CTA's candidate slice held in shared memory
+constexpr int kDigitBins = 2048;       // radix digits of 11, 11 and 10 bits
+constexpr int kBinsPerThread = kDigitBins / kTopkThreads;
+static_assert(kBinsPerThread == 2, "two digit bins per thread");
 
 struct TopkShared {
-  int sub[kSubHists][256];
-  int hist[2][256];   // this CTA's digit histogram by pass parity, read by the whole cluster
-  int tot[256];
+  int sub[2][kDigitBins];    // digit histograms, one per half of the warps
+  int hist[2][kDigitBins];   // this CTA's digit histogram by pass parity, read by the whole cluster
   int warp_tmp[32];
-  int total;
-  int cnt[2];         // this CTA's counts of keys above T and equal to T, read by the cluster
+  int wgt[kTopkWarps], weq[kTopkWarps];   // per-warp counts of keys above T and equal to T
+  int cnt[2];                // this CTA's counts above T and equal to T, read by the cluster
   int gbase, ebase;
   uint32_t prefix;
   int kk;
+  int total;
 };
 
 // Candidates and keys come in one of two ways.  Fetched-set mode: candidate j is entry
@@ -275,12 +294,14 @@ struct TopkShared {
 // stride is then cap.
 //
 // One thread-block cluster per sequence; CTA `rank` owns the contiguous candidate slice
-// [rank m, (rank + 1) m), m = ceil(n / cluster size).  Its keys go to shared memory (to the key workspace when the slice exceeds kTopkSmemKeys).  Four
-// radix passes of 8 bits find the k-th largest key T and the number kk of keys equal to
-// T to keep; each pass adds the CTAs' digit histograms through distributed shared
-// memory.  The kept entries, all keys above T and the kk lowest-index ties, are written
-// in ascending candidate (= entry) order: each CTA's offsets come from the counts of the
-// CTAs before it, and inside a CTA from block scans over rounds of 4096 candidates.
+// [rank m, (rank + 1) m), m = ceil(n / cluster size).  Its keys go to shared memory (to
+// the key workspace when the slice exceeds kTopkSmemKeys).  Three radix passes (digits
+// of 11, 11 and 10 bits, most significant first) find the k-th largest key T and the
+// number kk of keys equal to T to keep; each pass adds the CTAs' digit histograms
+// through distributed shared memory and picks the digit with one block-wide scan.  The
+// kept entries, all keys above T and the kk lowest-index ties, are written in ascending
+// candidate (= entry) order: each warp owns a contiguous part of its CTA's slice, and
+// its output offset comes from the counts of the CTAs and warps before it.
 __global__ void __launch_bounds__(kTopkThreads, 1)
 topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx, int cap,
                     const int32_t* __restrict__ count, const float* __restrict__ logit,
@@ -323,61 +344,88 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
   if (direct) {
     for (int j = tid; j < mloc; j += kTopkThreads) key[j] = __ldg(dkeys + static_cast<size_t>(b) * cap + j0 + j);
   } else {
-#pragma unroll 4
-    for (int j = tid; j < mloc; j += kTopkThreads) {
-      const int e = __ldg(ib + j0 + j);
-      float z = -INFINITY;
-      if (e >= 0 && e < N)
-        for (int l = 0; l < L; ++l) z = fmaxf(z, __ldg(logit + (static_cast<size_t>(l) * B + b) * N + e));
-      key[j] = order_key(z);
+    // eight candidates per thread in flight: their entries first, then every layer's logits
+    constexpr int kBatch = 8;
+    for (int jb = 0; jb < mloc; jb += kBatch * kTopkThreads) {
+      int e[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int j = jb + u * kTopkThreads + tid;
+        e[u] = j < mloc ? __ldg(ib + j0 + j) : -1;
+      }
+      float z[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) z[u] = -INFINITY;
+      for (int l = 0; l < L; ++l) {
+        const float* lb = logit + (static_cast<size_t>(l) * B + b) * N;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+          if (e[u] >= 0 && e[u] < N) z[u] = fmaxf(z[u], __ldg(lb + e[u]));
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int j = jb + u * kTopkThreads + tid;
+        if (j < mloc) key[j] = order_key(z[u]);
+      }
     }
   }
   __syncthreads();
   uint32_t prefix = 0, himask = 0;
   int kk = kb;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = tid; i < kSubHists * 256; i += kTopkThreads) (&sh.sub[0][0])[i] = 0;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const uint32_t dmask = pass == 2 ? 1023u : 2047u;
+    for (int i = tid; i < 2 * kDigitBins; i += kTopkThreads) (&sh.sub[0][0])[i] = 0;
     __syncthreads();
+    int* mysub = sh.sub[warp & 1];
     for (int j = tid; j < mloc; j += kTopkThreads) {
       const uint32_t u = key[j];
-      if ((u & himask) == prefix) atomicAdd(&sh.sub[warp >> 1][(u >> shift) & 255u], 1);
+      if ((u & himask) == prefix) atomicAdd(&mysub[(u >> shift) & dmask], 1);
     }
     __syncthreads();
-    if (tid < 256) {
-      int h = 0;
 #pragma unroll
-      for (int w = 0; w < kSubHists; ++w) h += sh.sub[w][tid];
-      sh.hist[pass & 1][tid] = h;
+    for (int q = 0; q < kBinsPerThread; ++q) {
+      const int d = tid * kBinsPerThread + q;
+      sh.hist[pass & 1][d] = sh.sub[0][d] + sh.sub[1][d];
     }
     // After this barrier every CTA's histogram of the pass is complete.  A CTA rewrites
     // hist[pass & 1] two passes later, after the next barrier, which no CTA passes
     // before it has finished reading this pass's histograms.
     cl.sync();
-    if (tid < 256) {
+    // thread t holds the totals of digits D - 1 - 2t and D - 2 - 2t (descending order),
+    // so an exclusive scan in thread order counts the keys in higher digits
+    int tot[kBinsPerThread], mine = 0;
+#pragma unroll
+    for (int q = 0; q < kBinsPerThread; ++q) {
+      const int d = kDigitBins - 1 - (tid * kBinsPerThread + q);
       int t = 0;
-      for (int r = 0; r < cs; ++r) t += cl.map_shared_rank(&sh.hist[pass & 1][0], r)[tid];
-      sh.tot[tid] = t;
+      for (int r = 0; r < cs; ++r) t += cl.map_shared_rank(&sh.hist[pass & 1][0], r)[d];
+      tot[q] = t;
+      mine += t;
     }
-    __syncthreads();
-    if (tid == 0) {
-      int cum = 0, sel = 0;
-      for (int d = 255; d >= 0; --d) {
-        if (cum + sh.tot[d] >= kk) { sel = d; break; }
-        cum += sh.tot[d];
+    int above = block_exclusive_scan(mine, sh.warp_tmp, &sh.total);
+#pragma unroll
+    for (int q = 0; q < kBinsPerThread; ++q) {
+      const int d = kDigitBins - 1 - (tid * kBinsPerThread + q);
+      if (above < kk && above + tot[q] >= kk) {   // the digit holding the kk-th largest key
+        sh.kk = kk - above;
+        sh.prefix = prefix | (static_cast<uint32_t>(d) << shift);
       }
-      sh.kk = kk - cum;
-      sh.prefix = prefix | (static_cast<uint32_t>(sel) << shift);
+      above += tot[q];
     }
     __syncthreads();
     kk = sh.kk;
     prefix = sh.prefix;
-    himask |= 255u << shift;
+    himask |= dmask << shift;
   }
   const uint32_t T = prefix;
+  // this warp's contiguous part of the slice
+  const int per = (mloc + kTopkWarps - 1) / kTopkWarps;
+  const int w0 = min(mloc, warp * per), w1 = min(mloc, w0 + per);
   {
     int gt = 0, eq = 0;
-    for (int j = tid; j < mloc; j += kTopkThreads) {
+    for (int j = w0 + lane; j < w1; j += 32) {
       const uint32_t u = key[j];
       gt += u > T;
       eq += u == T;
@@ -387,13 +435,16 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
       gt += __shfl_xor_sync(0xffffffffu, gt, o);
       eq += __shfl_xor_sync(0xffffffffu, eq, o);
     }
-    if (lane == 0) { sh.sub[0][warp] = gt; sh.sub[1][warp] = eq; }
+    if (lane == 0) { sh.wgt[warp] = gt; sh.weq[warp] = eq; }
     __syncthreads();
-    if (tid == 0) {
-      int g = 0, q = 0;
-      for (int w = 0; w < kTopkWarps; ++w) { g += sh.sub[0][w]; q += sh.sub[1][w]; }
-      sh.cnt[0] = g;
-      sh.cnt[1] = q;
+    if (warp == 0) {
+      int g = sh.wgt[lane], q = sh.weq[lane];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        g += __shfl_xor_sync(0xffffffffu, g, o);
+        q += __shfl_xor_sync(0xffffffffu, q, o);
+      }
+      if (lane == 0) { sh.cnt[0] = g; sh.cnt[1] = q; }
     }
     cl.sync();
     if (tid == 0) {
@@ -408,36 +459,20 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
     }
     cl.sync();   // no CTA leaves while another may still read its shared memory
   }
-  int gt_base = sh.gbase, eq_base = sh.ebase;
-  for (int r0 = 0; r0 < mloc; r0 += 4 * kTopkThreads) {
-    const int j = r0 + 4 * tid;
-    uint32_t u[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) u[e] = j + e < mloc ? key[j + e] : 0u;
-    int gt = 0, eq = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      gt += j + e < mloc && u[e] > T;
-      eq += j + e < mloc && u[e] == T;
-    }
-    int gt_before = gt_base + block_exclusive_scan(gt, sh.warp_tmp, &sh.total);
-    const int gt_round = sh.total;
-    int eq_before = eq_base + block_exclusive_scan(eq, sh.warp_tmp, &sh.total);
-    const int eq_round = sh.total;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (j + e >= mloc) break;
-      const int c = j0 + j + e;
-      if (u[e] > T) {
-        ob[gt_before + min(eq_before, kk)] = direct ? c : __ldg(ib + c);
-        ++gt_before;
-      } else if (u[e] == T) {
-        if (eq_before < kk) ob[gt_before + eq_before] = direct ? c : __ldg(ib + c);
-        ++eq_before;
-      }
-    }
-    gt_base += gt_round;
-    eq_base += eq_round;
+  int gt_before = sh.gbase, eq_before = sh.ebase;
+  for (int w = 0; w < warp; ++w) { gt_before += sh.wgt[w]; eq_before += sh.weq[w]; }
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int jb = w0; jb < w1; jb += 32) {
+    const int j = jb + lane;
+    const uint32_t u = j < w1 ? key[j] : 0u;
+    const bool g = j < w1 && u > T, q = j < w1 && u == T;
+    const uint32_t gm = __ballot_sync(0xffffffffu, g), qm = __ballot_sync(0xffffffffu, q);
+    const int gb = gt_before + __popc(gm & lt), qb = eq_before + __popc(qm & lt);
+    const int c = j0 + j;
+    if (g) ob[gb + min(qb, kk)] = direct ? c : __ldg(ib + c);
+    else if (q && qb < kk) ob[gb + qb] = direct ? c : __ldg(ib + c);
+    gt_before += __popc(gm);
+    eq_before += __popc(qm);
   }
   if (rank == 0 && tid == 0 && topk_count) topk_count[b] = kb;
 }
@@ -496,11 +531,16 @@ int launch_topk_cluster(int B, int L, int N, int k, const int32_t* idx, int cap,
                         int32_t* status, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws, cudaStream_t s) {
   const int smem = kTopkSmemKeys * 4;
   cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // CTAs per sequence: as many as keep B x cs within one wave, at most 8 (portable)
+  // CTAs per sequence: as many as keep B x cs within one wave, at most 8 (portable), but
+  // at least enough that a full list (cap candidates) keeps every CTA's slice in shared
+  // memory: the busiest sequence sets the kernel's time, and a slice in global memory
+  // costs more than a second wave of clusters.
   int cs = 8;
   while (cs > 1 && B * cs > sms) cs >>= 1;
+  while (cs < 8 && (cap + cs - 1) / cs > kTopkSmemKeys) cs <<= 1;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
