@@ -89,17 +89,23 @@ def test_tiny_fp32_full_parity():
     assert 0.05 < frac < 0.2
 
 
-def test_128k_bf16_projection_within_fp32_bound():
+def test_128k_bf16_projection_statistics_and_bound():
+    """The device query equals the oracle's on >= 97% of the elements and is within one
+    bf16 step on >= 99.5% (lsa_cases.assert_q_statistics says why not everywhere); every
+    element inside the rigorous per-element fp32 bound q_allowed; head weights within one
+    fp32 summation bound."""
     w = W.WORKLOADS["lsa_step_128k_b1_bf16"]
     inp = C.make_inputs(w)
     orc = C.OracleCache(inp)
     out = run_score(inp)
+    C.assert_q_statistics(out["q"][:, 0].cpu().double().numpy(), np.stack([orc.qw(l, 0)[0] for l in range(w.L)]),
+                          w.name)
     for l in range(w.L):
         q, wv = orc.qw(l, 0)
-        qc = out["q"][l, 0].double().cpu().numpy()
+        qc = out["q"][l, 0].cpu().double().numpy()
         ok = C.q_within(qc, q, orc.q_allowed(l, 0))
         assert ok.all(), f"layer {l}: {int((~ok).sum())} query elements outside the bound"
-        np.testing.assert_allclose(out["w"][l, 0].double().cpu().numpy(), wv, rtol=1e-4, atol=1e-4)
+        assert np.all(np.abs(out["w"][l, 0].cpu().double().numpy() - wv) <= orc.w_allowed(l, 0) * (1 + 1e-9))
 
 
 def test_128k_bf16_score_with_oracle_query():
