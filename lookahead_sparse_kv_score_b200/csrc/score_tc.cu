@@ -264,6 +264,26 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
     int j = 0, s = 0;
     uint32_t ph = 0;
     bool ok = true;
+    // Gathered mode: the rows (tensor-map row coordinates) of this lane's four candidates
+    // of a tile; loaded one tile ahead so their latency overlaps the barrier waits.
+    // Rows past the list repeat the tile's first candidate (always present).
+    int rows[4] = {0, 0, 0, 0};
+    auto rows_of = [&](int u, int t) {
+      const int32_t* ib = p.idx + static_cast<size_t>(u) * p.cap;
+      const int nb = min(__ldg(p.count + u), p.cap);
+      const int first = __ldg(ib + t * kTileM);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int jj = t * kTileM + 4 * lane + e;
+        int ent = __ldg(ib + min(jj, p.cap - 1));
+        ent = jj < nb ? ent : first;
+        ent = min(max(ent, 0), p.N - 1);
+        rows[e] = (uabs0 + u) * p.N + ent;
+      }
+    };
+    if constexpr (kGather) {
+      if (pp < n_local) rows_of(unit, tile);
+    }
     for (int i = pp; i < n_local; i += 2) {
       const int st = pp * S2 + s;
       if (lane == 0) {
@@ -275,21 +295,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
       if (!ok) break;
       uint8_t* dst = a_ring + static_cast<size_t>(st) * lay.a_bytes;
       if constexpr (kGather) {
-        const int32_t* ib = p.idx + static_cast<size_t>(unit) * p.cap;
-        const int nb = min(__ldg(p.count + unit), p.cap);
-        const int first = __ldg(ib + tile * kTileM);      // a tile's first candidate always exists
-        int r[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int jj = tile * kTileM + 4 * lane + e;
-          int ent = jj < nb ? __ldg(ib + jj) : first;       // rows past the list repeat a real row
-          ent = min(max(ent, 0), p.N - 1);
-          r[e] = (uabs0 + unit) * p.N + ent;
-        }
 #pragma unroll
         for (int c = 0; c < kKSteps / 4; ++c)
-          tma_gather4_2d(dst + c * (kTileM * 128) + lane * 4 * 128, &kmap, c * (kFp8 ? 128 : 64), r[0], r[1], r[2],
-                         r[3], &full[st], policy);
+          tma_gather4_2d(dst + c * (kTileM * 128) + lane * 4 * 128, &kmap, c * (kFp8 ? 128 : 64), rows[0], rows[1],
+                         rows[2], rows[3], &full[st], policy);
       } else {
 #pragma unroll
         for (int c = 0; c < kKSteps / 4; ++c)     // 128-byte K chunks of a key row
@@ -299,6 +308,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
       ++j;
       if (++s == S2) { s = 0; ph ^= 1; }
       advance(unit, tile, 2);
+      if constexpr (kGather) {
+        if (i + 2 < n_local) rows_of(unit, tile);
+      }
     }
     if (lane == 0) {
       if (pp == 0 && ok) load_q_through(k_last);
