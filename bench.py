@@ -55,6 +55,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-vote", action="store_true", help="skip the vote-label measurement")
     ap.add_argument("--no-hot-pool", action="store_true", help="skip the residency measurement")
+    ap.add_argument("--schedule", choices=["batched", "per_layer"], default="batched",
+                    help="fetch schedule of the timed step (batched: all layers scored in one launch, then the "
+                         "selection, then the gathers; per_layer: each layer's gather runs beside the next "
+                         "layer's scoring; both are timed side by side in gather_overlap)")
     return ap.parse_args(argv)
 
 
@@ -151,7 +155,9 @@ class Trigger:
         self.new = torch.empty(L, B, self.Nw, dtype=torch.int32, device=device)
         self.idx_new = torch.empty(L, B, self.cap, dtype=torch.int32, device=device)
         self.cnt_new = torch.zeros(L, B, dtype=torch.int32, device=device)
-        self.hot = torch.empty(L, B, self.cap, w.row_bytes, dtype=torch.uint8, device=device)
+        # the hot pool (one region per layer's new rows); not needed without a cold pool
+        self.hot = (torch.empty(L, B, self.cap, w.row_bytes, dtype=torch.uint8, device=device)
+                    if cold is not None else None)
         self.idx_U = torch.empty(B, N, dtype=torch.int32, device=device)
         self.cnt_U = torch.zeros(B, dtype=torch.int32, device=device)
         self.topk = torch.empty(B, w.k, dtype=torch.int32, device=device)
@@ -167,49 +173,122 @@ class Trigger:
         # the selection first.
         self.main = torch.cuda.Stream(device, priority=-1)
         self.side = torch.cuda.Stream(device, priority=0)
-        self.timing = []     # per step: [(score_start, score_end, gather_start, gather_end) per layer]
+        self.timing = []     # per recorded step: the events of its score, gather and main-stream spans
+        self.schedule = "batched"
 
-    def run(self, record=False):
-        """One trigger.  The three layers are scored in one launch (HBM-bound, ~0.55 ms),
-        then the union, the compactions and the top-k run (~0.3 ms; the top-k ranks by the
-        indexer logits, so it does not wait for the rows), and then the side stream
-        gathers the new rows of each layer over the host link (tens of ms).  Running the
-        gathers beside the scoring or the selection would only take SMs from them."""
+    def run(self, record=False, schedule=None):
+        """One trigger on the chosen fetch schedule (self.schedule unless given)."""
+        if (schedule or self.schedule) == "per_layer":
+            return self.run_per_layer(record)
+        return self.run_batched(record)
+
+    def _events(self, record):
+        L = self.w.L
+        mk = lambda: torch.cuda.Event(enable_timing=record)
+        return {"score": [(mk(), mk()) for _ in range(L)], "gather": [(mk(), mk()) for _ in range(L)],
+                "select": (mk(), mk())}
+
+    def run_batched(self, record=False):
+        """One trigger, all layers scored in one launch (HBM-bound, ~0.55 ms), then one
+        launch forms the union, the per-layer new sets and all fetch lists, and the top-k
+        runs (it ranks by the indexer logits, so it does not wait for the rows); then the
+        side stream gathers the new rows of each layer over the host link (tens of ms)."""
         lsa, w, inp = self.lsa, self.w, self.inp
         B, L, N = w.B, w.L, w.N
         m, sd = self.main, self.side
-        e = [torch.cuda.Event(enable_timing=record) for _ in range(4 + 2 * L)]
+        e = self._events(record)
         if record:
-            e[2 + 2 * L].record(m)
+            e["select"][0].record(m)
         lsa.lsa_index_project(B, L, w.D, w.r, w.H, w.dI, self.wdt, inp["h"], inp["Wd"], inp["Wu"], inp["Ww"], -1,
                               self.q, self.wv, self.ws_proj, stream=m)
         if record:
-            e[0].record(m)
+            e["score"][0][0].record(m)
         lsa.lsa_index_score(B, L, N, w.D, w.r, w.H, w.dI, self.wdt, None, None, None, None, inp["bias"],
                             self.kdt, inp["K"], inp["kscale"], -1, self.q, self.wv, None, None,
                             self.mask, self.logit, None, self.ws_score, status=self.status, stream=m)
         if record:
-            e[1].record(m)
-        with torch.cuda.stream(m):
-            self.U.zero_()
-        for l in range(L):
-            lsa.lsa_select_union(B, self.Nw, self.mask[l], self.U, self.new[l], stream=m)
-            lsa.lsa_compact(B, N, self.new[l], self.cap, self.idx_new[l], self.cnt_new[l], self.status, stream=m)
-        lsa.lsa_compact(B, N, self.U, N, self.idx_U, self.cnt_U, self.status, stream=m)
+            e["score"][0][1].record(m)
+            for l in range(1, L):       # one launch covers every layer
+                e["score"][l][0].record(m)
+                e["score"][l][1].record(m)
+        lsa.lsa_select_fetch(B, L, N, self.mask, self.U, self.new, self.cap, self.idx_new, self.cnt_new,
+                             self.idx_U, self.cnt_U, self.status, stream=m)
         lsa.lsa_topk(B, L, N, w.k, self.idx_U, N, self.cnt_U, self.logit, self.topk, self.topk_cnt, self.ws_topk,
                      stream=m)
         if record:
-            e[3 + 2 * L].record(m)
+            e["select"][1].record(m)
         selected = torch.cuda.Event()
         selected.record(m)
         sd.wait_event(selected)
         for l in range(L):
             if record:
-                e[2 + 2 * l].record(sd)
+                e["gather"][l][0].record(sd)
             lsa.lsa_gather_cold(B, N, w.row_bytes, self.cold, self.idx_new[l], self.cnt_new[l], self.cap,
                                 self.hot[l], self.status, stream=sd)
             if record:
-                e[3 + 2 * l].record(sd)
+                e["gather"][l][1].record(sd)
+        done = torch.cuda.Event()
+        done.record(sd)
+        m.wait_event(done)
+        if record:
+            self.timing.append(e)
+
+    def select_only(self):
+        """The main stream's part of a trigger alone (projection, scoring, union, fetch
+        lists, top-k), without the gathers."""
+        lsa, w, inp = self.lsa, self.w, self.inp
+        B, L, N = w.B, w.L, w.N
+        m = self.main
+        lsa.lsa_index_project(B, L, w.D, w.r, w.H, w.dI, self.wdt, inp["h"], inp["Wd"], inp["Wu"], inp["Ww"], -1,
+                              self.q, self.wv, self.ws_proj, stream=m)
+        lsa.lsa_index_score(B, L, N, w.D, w.r, w.H, w.dI, self.wdt, None, None, None, None, inp["bias"],
+                            self.kdt, inp["K"], inp["kscale"], -1, self.q, self.wv, None, None,
+                            self.mask, self.logit, None, self.ws_score, status=self.status, stream=m)
+        lsa.lsa_select_fetch(B, L, N, self.mask, self.U, self.new, self.cap, self.idx_new, self.cnt_new,
+                             self.idx_U, self.cnt_U, self.status, stream=m)
+        lsa.lsa_topk(B, L, N, w.k, self.idx_U, N, self.cnt_U, self.logit, self.topk, self.topk_cnt, self.ws_topk,
+                     stream=m)
+        torch.cuda.current_stream().wait_stream(m)
+
+    def run_per_layer(self, record=False):
+        """One trigger on the schedule the pages describe (the fetch asynchronous and
+        overlapped with compute): layer l is scored alone, its new rows are unioned and
+        compacted, and their gather starts on the side stream while layer l + 1 is
+        scored; the union's fetch list and the top-k follow the last layer."""
+        lsa, w, inp = self.lsa, self.w, self.inp
+        B, L, N = w.B, w.L, w.N
+        m, sd = self.main, self.side
+        e = self._events(record)
+        if record:
+            e["select"][0].record(m)
+        lsa.lsa_index_project(B, L, w.D, w.r, w.H, w.dI, self.wdt, inp["h"], inp["Wd"], inp["Wu"], inp["Ww"], -1,
+                              self.q, self.wv, self.ws_proj, stream=m)
+        with torch.cuda.stream(m):
+            self.U.zero_()
+        for l in range(L):
+            if record:
+                e["score"][l][0].record(m)
+            lsa.lsa_index_score(B, L, N, w.D, w.r, w.H, w.dI, self.wdt, None, None, None, None, inp["bias"],
+                                self.kdt, inp["K"], inp["kscale"], l, self.q, self.wv, None, None,
+                                self.mask, self.logit, None, self.ws_score, status=self.status, stream=m)
+            if record:
+                e["score"][l][1].record(m)
+            lsa.lsa_select_union(B, self.Nw, self.mask[l], self.U, self.new[l], stream=m)
+            lsa.lsa_compact(B, N, self.new[l], self.cap, self.idx_new[l], self.cnt_new[l], self.status, stream=m)
+            ready = torch.cuda.Event()
+            ready.record(m)
+            sd.wait_event(ready)
+            if record:
+                e["gather"][l][0].record(sd)
+            lsa.lsa_gather_cold(B, N, w.row_bytes, self.cold, self.idx_new[l], self.cnt_new[l], self.cap,
+                                self.hot[l], self.status, stream=sd)
+            if record:
+                e["gather"][l][1].record(sd)
+        lsa.lsa_compact(B, N, self.U, N, self.idx_U, self.cnt_U, self.status, stream=m)
+        lsa.lsa_topk(B, L, N, w.k, self.idx_U, N, self.cnt_U, self.logit, self.topk, self.topk_cnt, self.ws_topk,
+                     stream=m)
+        if record:
+            e["select"][1].record(m)
         done = torch.cuda.Event()
         done.record(sd)
         m.wait_event(done)
@@ -217,12 +296,11 @@ class Trigger:
             self.timing.append(e)
 
     def kernel_times_ms(self):
-        """Per step, in ms: the score launch; the gather launches; the main stream from
-        the projection through the top-k."""
-        L = self.w.L
-        score = [e[0].elapsed_time(e[1]) for e in self.timing]
-        gather = [sum(e[2 + 2 * l].elapsed_time(e[3 + 2 * l]) for l in range(L)) for e in self.timing]
-        select = [e[2 + 2 * L].elapsed_time(e[3 + 2 * L]) for e in self.timing]
+        """Per step, in ms: the score launches (summed); the gather launches (summed); the
+        main stream from the projection through the top-k."""
+        score = [sum(a.elapsed_time(b) for a, b in e["score"]) for e in self.timing]
+        gather = [sum(a.elapsed_time(b) for a, b in e["gather"]) for e in self.timing]
+        select = [e["select"][0].elapsed_time(e["select"][1]) for e in self.timing]
         return score, gather, select
 
 
@@ -460,16 +538,13 @@ def hot_pool_measure(lsa, trig, device, triggers=8, rho=0.9):
         lsa.lsa_index_score(B, L, N, w.D, w.r, w.H, w.dI, trig.wdt, None, None, None, None, inp["bias"],
                             trig.kdt, inp["K"], inp["kscale"], -1, trig.q, trig.wv, None, None,
                             trig.mask, trig.logit, None, trig.ws_score, status=status, stream=m)
-        with torch.cuda.stream(m):
-            trig.U.zero_()
-        for l in range(L):
-            lsa.lsa_select_union(B, trig.Nw, trig.mask[l], trig.U, None, stream=m)
+        lsa.lsa_select_fetch(B, L, N, trig.mask, trig.U, None, trig.cap, trig.idx_new, trig.cnt_new,
+                             trig.idx_U, trig.cnt_U, status, stream=m)
         ready = torch.cuda.Event()
         ready.record(m)
         sd.wait_event(ready)
         lsa.lsa_hot_pool_update(B, N, slots, w.row_bytes, t, trig.U, trig.cold, hot, state, moved, status, ws,
                                 stream=sd)
-        lsa.lsa_compact(B, N, trig.U, N, trig.idx_U, trig.cnt_U, status, stream=m)
         lsa.lsa_topk(B, L, N, w.k, trig.idx_U, N, trig.cnt_U, trig.logit, trig.topk, trig.topk_cnt, trig.ws_topk,
                      stream=m)
         done = torch.cuda.Event()
@@ -489,6 +564,60 @@ def hot_pool_measure(lsa, trig, device, triggers=8, rho=0.9):
             "first_trigger_ms": ms[0], "fetch_rows_per_trigger": mean(fetch_rows),
             "moved_rows_per_trigger": mean(moved_rows), "first_trigger_moved_rows": moved_rows[0],
             "host_link_bytes_per_trigger": mean(moved_rows) * w.row_bytes}
+
+
+def fine_measure(lsa, trig, device, steps=5):
+    """The native indexer's fine selection inside the fetched subset (lsa_fine_score over
+    each sequence's union fetch list, then lsa_topk with one layer of those scores) after
+    a trigger: per-token query and head weights from their own streams, layer 0's keys
+    standing in for the indexer's own.  Roofline: per candidate the key row and its scale,
+    its list index and its score write (dI + 12 bytes) against the measured HBM peak."""
+    w = trig.w
+    B, N = w.B, w.N
+    qf, wf = W.fine_query(w, device)
+    K0 = trig.inp["K"][0]
+    ks0 = trig.inp["kscale"][0] if trig.inp["kscale"] is not None else None
+    kdt = trig.kdt
+    score = torch.empty(B, N, dtype=torch.float32, device=device)
+    topk = torch.empty(B, w.k, dtype=torch.int32, device=device)
+    tcnt = torch.empty(B, dtype=torch.int32, device=device)
+    ws = lsa.workspace(lsa.lsa_fine_score_workspace_bytes(B, w.H, w.dI, kdt), device)
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    m = trig.main
+
+    def one():
+        lsa.lsa_fine_score(B, N, w.H, w.dI, lsa.LSA_BF16, qf, wf, kdt, K0, ks0, trig.idx_U, trig.cap, trig.cnt_U,
+                           score, ws, status=st, stream=m)
+        lsa.lsa_topk(B, 1, N, w.k, trig.idx_U, trig.cap, trig.cnt_U, score, topk, tcnt, trig.ws_topk, stream=m)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    score_ms = 0.0
+    total_ms = 0.0
+    for _ in range(steps):
+        e[0].record(m)
+        lsa.lsa_fine_score(B, N, w.H, w.dI, lsa.LSA_BF16, qf, wf, kdt, K0, ks0, trig.idx_U, trig.cap, trig.cnt_U,
+                           score, ws, status=st, stream=m)
+        e[1].record(m)
+        lsa.lsa_topk(B, 1, N, w.k, trig.idx_U, trig.cap, trig.cnt_U, score, topk, tcnt, trig.ws_topk, stream=m)
+        e[2].record(m)
+        torch.cuda.synchronize()
+        score_ms += e[0].elapsed_time(e[1])
+        total_ms += e[0].elapsed_time(e[2])
+    score_ms /= steps
+    total_ms /= steps
+    cands = int(trig.cnt_U.clamp(max=trig.cap).sum().item())
+    per = w.dI * K0.element_size() + (4 if ks0 is not None else 0) + 8
+    hbm_peak, peak_kind = measured_peaks()
+    achieved = cands * per / (score_ms * 1e-3) / 1e9
+    return {"workload": f"{w.name}: native-indexer fine top-{w.k} inside each sequence's union fetch list",
+            "candidates_per_step": cands, "status": int(st.item()), "score_ms": score_ms, "fine_topk_ms": total_ms,
+            "value": cands / (total_ms * 1e-3), "unit": "fetched entries scored+ranked/s",
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "bytes_per_candidate": per, "kernel": "score_tc (gathered)",
+                         "peak_kind": peak_kind}}
 
 
 def vote_measure(lsa, device, steps=5):
@@ -604,6 +733,7 @@ def our_arm(args):
     inp = device_inputs(w, device)
     cold = cold_pool(w, device)
     trig = Trigger(lsa, w, inp, cold, device)
+    trig.schedule = args.schedule
     torch.cuda.synchronize()
 
     for _ in range(max(args.warmup, 0)):
@@ -642,6 +772,27 @@ def our_arm(args):
     achieved = key_bytes / (score_avg * 1e-3) / 1e9
     link = host_link_gbs(device)
     gather_gbs = fetched_rows * w.row_bytes / (gather_ms[-1] * 1e-3) / 1e9
+
+    # the two fetch schedules side by side (device time per trigger, same run)
+    def time_schedule(fn, reps=3):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(trig.main)
+        for _ in range(reps):
+            fn()
+        b.record(trig.main)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+    overlap = {"batched_ms": time_schedule(trig.run_batched), "per_layer_ms": time_schedule(trig.run_per_layer),
+               "timed": args.schedule,
+               "batched": "all layers scored in one launch, the fused selection and the top-k, then the gathers "
+                          "on the side stream",
+               "per_layer": "layer l scored alone, its new rows unioned, compacted and gathered on the side stream "
+                            "while layer l+1 is scored; the union's list and the top-k after the last layer"}
+    if int(trig.status.item()) != 0:
+        raise SystemExit(f"device status {int(trig.status.item())} in the schedule comparison")
+    fine = fine_measure(lsa, trig, device) if rank == 0 else None
 
     # end to end: inputs from pinned host memory every step, result read back
     h_host = inp["h"].cpu().pin_memory()
@@ -698,7 +849,9 @@ def our_arm(args):
                        "parallelism": f"replica per GPU x{world}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": traffic_per_launch(),
-                         "kernel": "score_tc (lsa_index_score, all layers in one launch)",
+                         "kernel": ("score_tc (lsa_index_score, one launch per layer; achieved = all layers' "
+                                    "bytes over the sum of the three launch times)" if args.schedule == "per_layer"
+                                    else "score_tc (lsa_index_score, all layers in one launch)"),
                          "note": "the scoring launch, the kernel the metric's roofline is about; the step's "
                                  "longest kernel is the host-link gather, reported in roofline_gather",
                          "bytes_per_launch": key_bytes, "launch_ms": score_avg, "peak_kind": peak_kind},
@@ -715,7 +868,10 @@ def our_arm(args):
                                 "peak_kind": "measured here: pinned host->device cudaMemcpy, 1 GiB"},
             "select_path": {"value": sel_value, "unit": UNIT, "ms_per_step": sel_ms / args.steps,
                             "covers": "projection, scoring, union, compaction and top-k on the main stream of "
-                                      "each timed step (the step's gathers follow on the side stream)"},
+                                      "each timed step (per_layer: the layers' gathers run beside the later "
+                                      "layers' scoring on the side stream; batched: they follow the top-k)"},
+            "gather_overlap": overlap,
+            "fine_select": fine,
             "hot_pool": hot_pool,
             "vote_labels": vote,
         }
