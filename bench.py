@@ -55,6 +55,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-vote", action="store_true", help="skip the vote-label measurement")
     ap.add_argument("--no-hot-pool", action="store_true", help="skip the residency measurement")
+    ap.add_argument("--select-only", action="store_true",
+                    help="profiling mode: time only the main-stream part of the step (projection, scoring, "
+                         "selection, top-k) without the cold pool, the gathers or the secondary measurements")
     ap.add_argument("--schedule", choices=["batched", "per_layer"], default="batched",
                     help="fetch schedule of the timed step (batched: all layers scored in one launch, then the "
                          "selection, then the gathers; per_layer: each layer's gather runs beside the next "
@@ -168,6 +171,7 @@ class Trigger:
         self.ws_score = lsa.workspace(lsa.lsa_index_score_workspace_bytes(B, L, N, w.D, w.r, w.H, w.dI,
                                                                           self.wdt, self.kdt), device)
         self.ws_topk = lsa.workspace(lsa.lsa_topk_workspace_bytes(B, N), device)
+        self.ws_sel = lsa.workspace(lsa.lsa_select_fetch_workspace_bytes(B, N), device)
         # The main stream runs at a higher priority than the side stream: where the two
         # overlap (the residency measurement), the SMs a retiring gather block frees go to
         # the selection first.
@@ -212,7 +216,7 @@ class Trigger:
                 e["score"][l][0].record(m)
                 e["score"][l][1].record(m)
         lsa.lsa_select_fetch(B, L, N, self.mask, self.U, self.new, self.cap, self.idx_new, self.cnt_new,
-                             self.idx_U, self.cnt_U, self.status, stream=m)
+                             self.idx_U, self.cnt_U, self.ws_sel, status=self.status, stream=m)
         lsa.lsa_topk(B, L, N, w.k, self.idx_U, N, self.cnt_U, self.logit, self.topk, self.topk_cnt, self.ws_topk,
                      stream=m)
         if record:
@@ -245,7 +249,7 @@ class Trigger:
                             self.kdt, inp["K"], inp["kscale"], -1, self.q, self.wv, None, None,
                             self.mask, self.logit, None, self.ws_score, status=self.status, stream=m)
         lsa.lsa_select_fetch(B, L, N, self.mask, self.U, self.new, self.cap, self.idx_new, self.cnt_new,
-                             self.idx_U, self.cnt_U, self.status, stream=m)
+                             self.idx_U, self.cnt_U, self.ws_sel, status=self.status, stream=m)
         lsa.lsa_topk(B, L, N, w.k, self.idx_U, N, self.cnt_U, self.logit, self.topk, self.topk_cnt, self.ws_topk,
                      stream=m)
         torch.cuda.current_stream().wait_stream(m)
@@ -539,7 +543,7 @@ def hot_pool_measure(lsa, trig, device, triggers=8, rho=0.9):
                             trig.kdt, inp["K"], inp["kscale"], -1, trig.q, trig.wv, None, None,
                             trig.mask, trig.logit, None, trig.ws_score, status=status, stream=m)
         lsa.lsa_select_fetch(B, L, N, trig.mask, trig.U, None, trig.cap, trig.idx_new, trig.cnt_new,
-                             trig.idx_U, trig.cnt_U, status, stream=m)
+                             trig.idx_U, trig.cnt_U, trig.ws_sel, status=status, stream=m)
         ready = torch.cuda.Event()
         ready.record(m)
         sd.wait_event(ready)
@@ -881,10 +885,39 @@ def our_arm(args):
     return 0
 
 
+def select_only_arm(args):
+    """Profiling mode: the main-stream part of the step on the benchmark workload (no cold
+    pool, no gathers), K timed steps; prints a reduced JSON line.  Not the benchmark."""
+    import lookahead_sparse_kv_score_b200 as lsa
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    lsa.lib()
+    w = W.WORKLOADS[args.workload]
+    if args.batch is not None:
+        w = W.scaled(w, B=args.batch)
+    inp = device_inputs(w, device)
+    trig = Trigger(lsa, w, inp, None, device)
+    for _ in range(max(args.warmup, 0)):
+        trig.select_only()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(trig.main)
+    for _ in range(args.steps):
+        trig.select_only()
+    b.record(trig.main)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / max(args.steps, 1)
+    print(json.dumps({"mode": "select_only", "workload": w.name, "B": w.B, "steps": args.steps,
+                      "ms_per_step": ms, "status": int(trig.status.item())}), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return reference_arm(args)
+    if args.select_only:
+        return select_only_arm(args)
     return our_arm(args)
 
 

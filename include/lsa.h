@@ -179,11 +179,15 @@ int lsa_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32
  *   cnt_new [L][B], idx_U [B][cap], cnt_U [B] int32 outputs.  A count above cap is
  *   reported as is, only cap indices are written and *status (device int32 or NULL) is
  *   raised to LSA_ERR_CAPACITY.  1 <= L <= 8, else LSA_ERR_UNSUPPORTED.  Device
- *   pointers 16-byte aligned (counts 4-byte).  One launch per block of 65535 sequences.
+ *   pointers 16-byte aligned (counts 4-byte).  Two launches (per-chunk counts, then the
+ *   lists) per block of 65535 sequences.
+ * workspace: lsa_select_fetch_workspace_bytes(B, N) bytes, 256-byte aligned.
  * ---------------------------------------------------------------------------------- */
+size_t lsa_select_fetch_workspace_bytes(int B, int N);
+
 int lsa_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* new_l, int cap,
                      int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
-                     void* stream);
+                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * lsa_topk -- fine top-k inside the fetched subset ([SUMMARY] §2.1 hierarchical

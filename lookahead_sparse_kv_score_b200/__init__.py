@@ -122,9 +122,15 @@ def lsa_compact(B, N, bits, cap, idx, count, status=None, stream=None):
            "lsa_compact")
 
 
-def lsa_select_fetch(B, L, N, mask, U, new_l, cap, idx_new, cnt_new, idx_U, cnt_U, status=None, stream=None):
+def lsa_select_fetch_workspace_bytes(B, N) -> int:
+    return int(lib().lsa_select_fetch_workspace_bytes(B, N))
+
+
+def lsa_select_fetch(B, L, N, mask, U, new_l, cap, idx_new, cnt_new, idx_U, cnt_U, workspace, status=None,
+                     stream=None):
     _check(lib().lsa_select_fetch(B, L, N, _p(mask), _p(U), _p(new_l), cap, _p(idx_new), _p(cnt_new), _p(idx_U),
-                                  _p(cnt_U), _p(status), _stream(stream)), "lsa_select_fetch")
+                                  _p(cnt_U), _p(status), _p(workspace), 0 if workspace is None else workspace.numel(),
+                                  _stream(stream)), "lsa_select_fetch")
 
 
 def lsa_topk_workspace_bytes(B, cap) -> int:

@@ -256,9 +256,14 @@ int lsa_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32
   return launch_compact(B, N, bits, cap, idx, count, status, static_cast<cudaStream_t>(stream));
 }
 
+size_t lsa_select_fetch_workspace_bytes(int B, int N) {
+  if (B < 0 || N < 0) return 0;
+  return select_fetch_workspace_bytes(B, N) + 256;
+}
+
 int lsa_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* new_l, int cap,
                      int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
-                     void* stream) {
+                     void* workspace, size_t workspace_bytes, void* stream) {
   const CallRange range("lsa_select_fetch");
   g_err[0] = 0;
   if (B < 0 || L < 0 || N < 0 || cap < 0) return fail(LSA_ERR_INVALID_ARG, "select_fetch: negative size");
@@ -270,8 +275,11 @@ int lsa_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uin
       (idx_new && !aligned(idx_new, 16)) || (idx_U && !aligned(idx_U, 16)) || !aligned(cnt_new, 4) ||
       !aligned(cnt_U, 4))
     return fail(LSA_ERR_INVALID_ARG, "select_fetch: misaligned pointer");
+  const size_t need = lsa_select_fetch_workspace_bytes(B, N);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+    return fail(LSA_ERR_NOMEM, "select_fetch: workspace %zu bytes (need %zu)", workspace_bytes, need);
   return launch_select_fetch(B, L, N, mask, U, new_l, cap, idx_new, cnt_new, idx_U, cnt_U, status,
-                             static_cast<cudaStream_t>(stream));
+                             static_cast<int32_t*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
 // Workspace of lsa_fine_score: query images, folded head weights, tile prefix.

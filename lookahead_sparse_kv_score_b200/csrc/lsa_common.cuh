@@ -32,6 +32,32 @@ int check_launch(const char* what, int kernels = 1);   // LSA_OK or LSA_ERR_CUDA
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// ------------------------------------------------------------------ dependent launches
+// The kernels of the scoring and selection chain are launched as programmatic dependents of
+// the kernel before them on the stream: a kernel's blocks may be scheduled while its
+// predecessor's last blocks still run, and each such kernel waits at its first
+// instruction (pdl_wait) until the predecessor has completed and its writes are visible;
+// it then lets its own dependents be scheduled (pdl_trigger).  For a kernel launched
+// without the attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... Params, typename... Args>
+inline cudaError_t launch_dependent(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                    Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Params>(args)...);
+}
+
 // ------------------------------------------------------------------ device helpers
 __device__ __forceinline__ void raise_status(int32_t* status, int code) {
   if (status != nullptr) atomicMax(status, code);
@@ -132,9 +158,10 @@ int launch_fine_score_simt(const FineArgs& a, cudaStream_t s);
 int launch_union(int B, int Nw, const uint32_t* m, uint32_t* U, uint32_t* nw, cudaStream_t s);
 int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32_t* count,
                    int32_t* status, cudaStream_t s);
+size_t select_fetch_workspace_bytes(int B, int N);
 int launch_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* nw, int cap,
                         int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
-                        cudaStream_t s);
+                        int32_t* counts, cudaStream_t s);
 int launch_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
                 const float* logit, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws,
                 cudaStream_t s);

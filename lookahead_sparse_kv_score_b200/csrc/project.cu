@@ -183,6 +183,30 @@ __global__ void reduce_splits(const float* __restrict__ part, int S, size_t n, i
 
 unsigned grid_for(size_t n) { return static_cast<unsigned>(std::min<size_t>((n + 255) / 256, 148 * 16)); }
 
+// The two stage-A reductions of the tensor-core path in one launch: elements [0, nw) are
+// the head weights w (fp32 outputs), elements [nw, nw + nc) the elements of c (rounded to
+// bf16); each sums its S slices in order.
+__global__ void reduce_cw_kernel(const float* __restrict__ partW, size_t nw, float* __restrict__ w1,
+                                 float* __restrict__ w2, const float* __restrict__ partA, size_t nc,
+                                 __nv_bfloat16* __restrict__ c, int S) {
+  pdl_wait();
+  pdl_trigger();
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < nw + nc;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    if (i < nw) {
+      float v = 0.f;
+      for (int s = 0; s < S; ++s) v += partW[s * nw + i];
+      w1[i] = v;
+      if (w2) w2[i] = v;
+    } else {
+      const size_t k = i - nw;
+      float v = 0.f;
+      for (int s = 0; s < S; ++s) v += partA[s * nc + k];
+      c[k] = __float2bfloat16_rn(v);
+    }
+  }
+}
+
 template <typename WT>
 int project_typed(const ProjectArgs& a, cudaStream_t st) {
   const WT* h = static_cast<const WT*>(a.h) + static_cast<size_t>(a.l0) * a.B * a.D;
@@ -231,6 +255,14 @@ int project_splits_b(int K) { return (K + kSliceB - 1) / kSliceB; }
 // Fixed-order sums of S slices for the tensor-core path: w (fp32) and c (rounded to bf16,
 // stored as bf16 for q = c W_up).
 int launch_project_reductions(const ProjectArgs& a, int S, const ProjectTcBufs& t, cudaStream_t st) {
+  if (a.do_w && a.do_q) {
+    const size_t nw = static_cast<size_t>(a.nL) * a.B * a.H;
+    const size_t woff = static_cast<size_t>(a.l0) * a.B * a.H;
+    const size_t nc = static_cast<size_t>(a.nL) * a.B * a.r;
+    launch_dependent(reduce_cw_kernel, dim3(grid_for(nw + nc)), dim3(256), 0, st, a.partW, nw, a.w_ws + woff,
+                     a.w_out ? a.w_out + woff : nullptr, a.partA, nc, t.c_bf16, S);
+    return check_launch("project/reduce");
+  }
   int launches = 0;
   if (a.do_w) {
     const size_t nw = static_cast<size_t>(a.nL) * a.B * a.H;

@@ -106,6 +106,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 __global__ void __launch_bounds__(kPThreads, 1)
 proj_tc_kernel(const __grid_constant__ CUtensorMap mapW1, const __grid_constant__ CUtensorMap mapW2,
                const __grid_constant__ CUtensorMap mapX, const PjParams p) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smraw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   const int xbytes = p.npad * 128;
@@ -240,7 +242,7 @@ int launch_pj(const void* X, int B, int K, int L, int l0, int nL, const void* W1
   const int nb2 = W2 ? (M2 + kPM - 1) / kPM : 0;
   const int smem = pj_smem(npad);
   cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  proj_tc_kernel<<<dim3(p.nb1 + nb2, p.slices, nL), kPThreads, smem, st>>>(m1, m2, mx, p);
+  launch_dependent(proj_tc_kernel, dim3(p.nb1 + nb2, p.slices, nL), dim3(kPThreads), smem, st, m1, m2, mx, p);
   return check_launch("project_tc");
 }
 

@@ -159,6 +159,8 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t t0, uint32_t t1, float (&v0
 template <bool kFp8, int kH, int kKSteps, bool kGather>
 __global__ void __launch_bounds__(TcShape<kFp8, kH>::kThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
+  pdl_wait();
+  pdl_trigger();
   using S = TcShape<kFp8, kH>;
   constexpr int kN = S::kN, kNumAcc = S::kNumAcc;
   extern __shared__ uint8_t smem_raw[];
@@ -482,6 +484,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const TcParams p) {
 __global__ void build_qimg_bf16_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
                                        int B, int H, int dI, int l0, uint8_t* __restrict__ img,
                                        float* __restrict__ wfold) {
+  pdl_wait();
+  pdl_trigger();
   const size_t uabs = static_cast<size_t>(l0) * B + blockIdx.y;
   const int units = H * dI / 8;
   const int u = blockIdx.x * blockDim.x + threadIdx.x;
@@ -503,6 +507,8 @@ __global__ void build_qimg_bf16_kernel(const __nv_bfloat16* __restrict__ q, cons
 __global__ void build_qimg_fp8_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
                                       int B, int H, int dI, int l0, uint8_t* __restrict__ img,
                                       float* __restrict__ wfold) {
+  pdl_wait();
+  pdl_trigger();
   const size_t uabs = static_cast<size_t>(l0) * B + blockIdx.y;
   const int lane = threadIdx.x & 31;
   const int h = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -546,12 +552,12 @@ int launch_kernel(const CUtensorMap& map, const TcParams& p, const TcLayout& lay
   if (p.idx != nullptr) {
     auto kern = score_tc_kernel<kFp8, kH, kKSteps, true>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.smem);
-    kern<<<grid, TcShape<kFp8, kH>::kThreads, lay.smem, st>>>(map, p);
+    launch_dependent(kern, dim3(grid), dim3(TcShape<kFp8, kH>::kThreads), lay.smem, st, map, p);
     return check_launch("fine_score_tc");
   }
   auto kern = score_tc_kernel<kFp8, kH, kKSteps, false>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.smem);
-  kern<<<grid, TcShape<kFp8, kH>::kThreads, lay.smem, st>>>(map, p);
+  launch_dependent(kern, dim3(grid), dim3(TcShape<kFp8, kH>::kThreads), lay.smem, st, map, p);
   return check_launch("score_tc");
 }
 
@@ -585,6 +591,8 @@ int launch_h(const CUtensorMap& map, const TcParams& p, const TcLayout& lay, int
 
 // tile_start[b] = sum over b' < b of ceil(min(count[b'], cap) / 128), b = 0..B (one block).
 __global__ void tile_prefix_kernel(const int32_t* __restrict__ count, int B, int cap, int32_t* __restrict__ tile_start) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int wsum[32];
   __shared__ int carry;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -619,12 +627,12 @@ int launch_fine_score_tc(const FineArgs& a, cudaStream_t st) {
   const TcLayout lay = tc_layout(a.H, a.dI, fp8);
   const dim3 ig(fp8 ? (a.H + 7) / 8 : (a.H * a.dI / 8 + 255) / 256, a.B);
   if (fp8)
-    build_qimg_fp8_kernel<<<ig, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.q), a.w, a.B, a.H, a.dI, 0,
-                                              a.qimg, a.wfold);
+    launch_dependent(build_qimg_fp8_kernel, ig, dim3(256), 0, st, static_cast<const __nv_bfloat16*>(a.q), a.w, a.B,
+                     a.H, a.dI, 0, a.qimg, a.wfold);
   else
-    build_qimg_bf16_kernel<<<ig, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.q), a.w, a.B, a.H, a.dI, 0,
-                                               a.qimg, a.wfold);
-  tile_prefix_kernel<<<1, 1024, 0, st>>>(a.count, a.B, a.cap, a.tile_start);
+    launch_dependent(build_qimg_bf16_kernel, ig, dim3(256), 0, st, static_cast<const __nv_bfloat16*>(a.q), a.w, a.B,
+                     a.H, a.dI, 0, a.qimg, a.wfold);
+  launch_dependent(tile_prefix_kernel, dim3(1), dim3(1024), 0, st, a.count, a.B, a.cap, a.tile_start);
   int rc = check_launch("fine_score/query image and tile prefix", 2);
   if (rc != LSA_OK) return rc;
   EncodeTiledFn enc = encode_fn();
@@ -679,11 +687,11 @@ int launch_score_tc(const TcArgs& a, cudaStream_t st) {
   // query images and folded head weights for the processed layers
   const dim3 ig(fp8 ? (s.H + 7) / 8 : (s.H * s.dI / 8 + 255) / 256, s.B * s.nL);
   if (fp8)
-    build_qimg_fp8_kernel<<<ig, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(s.q), s.w, s.B, s.H, s.dI,
-                                              s.l0, a.qimg, a.wfold);
+    launch_dependent(build_qimg_fp8_kernel, ig, dim3(256), 0, st, static_cast<const __nv_bfloat16*>(s.q), s.w, s.B,
+                     s.H, s.dI, s.l0, a.qimg, a.wfold);
   else
-    build_qimg_bf16_kernel<<<ig, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(s.q), s.w, s.B, s.H, s.dI,
-                                               s.l0, a.qimg, a.wfold);
+    launch_dependent(build_qimg_bf16_kernel, ig, dim3(256), 0, st, static_cast<const __nv_bfloat16*>(s.q), s.w, s.B,
+                     s.H, s.dI, s.l0, a.qimg, a.wfold);
   int rc = check_launch("score_tc/query image");
   if (rc != LSA_OK) return rc;
 

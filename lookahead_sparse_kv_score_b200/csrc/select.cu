@@ -126,68 +126,37 @@ compact_kernel(const uint32_t* __restrict__ bits, int Nw, int cap, int32_t* __re
 }
 
 // ------------------------------------------------------------------ union + fetch lists
-// The whole selection of one trigger in one pass over the L layer masks: per word,
+// The whole selection of one trigger in two launches over the L layer masks: per word,
 // new_l = mask_l & ~(mask_0 | .. | mask_{l-1}) and U = mask_0 | .. | mask_{L-1}, and the
 // L + 1 fetch lists (new_0 .. new_{L-1}, U) with their counts.  Block (chunk, b) owns
-// words [chunk*kCompactWords, ...) of sequence b; the output bases of its lists are the
-// same popcounts over all earlier words of the sequence, recomputed from the masks
-// (re-read from L2).  Each thread writes its own word's indices; a warp's threads cover
-// one contiguous run of every list.
+// words [chunk*kCompactWords, ...) of sequence b.  The first launch writes each chunk's
+// popcounts of the L + 1 sets; the second takes its output bases from the earlier
+// chunks' counts, and each thread writes its own word's indices (a warp's threads cover
+// one contiguous run of every list).
 constexpr int kSelMaxLayers = 8;
 
+// Per (chunk, sequence): the popcounts of the chunk's words in the L new sets and the
+// union, written to counts[b][chunk][kSelMaxLayers + 1] (slot kSelMaxLayers = union).
 __global__ void __launch_bounds__(kCompactThreads)
-select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, int Nw, int cap,
-                    uint32_t* __restrict__ U, uint32_t* __restrict__ nw, int32_t* __restrict__ idx_new,
-                    int32_t* __restrict__ cnt_new, size_t cstride, int32_t* __restrict__ idx_U,
-                    int32_t* __restrict__ cnt_U, int32_t* status) {
+select_count_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, int Nw, int32_t* __restrict__ counts) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int sred[kSelMaxLayers + 1][kCompactThreads / 32];
-  __shared__ int wsum[kSelMaxLayers + 1][kCompactThreads / 32];
   const int b = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t* mb = mask + static_cast<size_t>(b) * Nw;
-  const int w0 = chunk * kCompactWords;
-  // bases: the lists' set bits in words [0, w0) of this sequence
+  const int wi = chunk * kCompactWords + tid;
   int pc[kSelMaxLayers + 1];
+  uint32_t acc = 0;
 #pragma unroll
-  for (int j = 0; j <= kSelMaxLayers; ++j) pc[j] = 0;
-  auto count_word = [&](const uint32_t* m) {
-    uint32_t acc = 0;
-#pragma unroll
-    for (int l = 0; l < kSelMaxLayers; ++l) {
-      if (l < L) {
-        pc[l] += __popc(m[l] & ~acc);
-        acc |= m[l];
-      }
-    }
-    pc[kSelMaxLayers] += __popc(acc);
-  };
-  if ((Nw & 3) == 0 && (lstride & 3) == 0) {
-    for (int i = tid; i < w0 / 4; i += kCompactThreads) {
-      uint4 v[kSelMaxLayers];
-#pragma unroll
-      for (int l = 0; l < kSelMaxLayers; ++l)
-        if (l < L) v[l] = __ldg(reinterpret_cast<const uint4*>(mb + l * lstride) + i);
-      uint32_t m[kSelMaxLayers];
-#pragma unroll
-      for (int l = 0; l < kSelMaxLayers; ++l) m[l] = v[l].x;
-      count_word(m);
-#pragma unroll
-      for (int l = 0; l < kSelMaxLayers; ++l) m[l] = v[l].y;
-      count_word(m);
-#pragma unroll
-      for (int l = 0; l < kSelMaxLayers; ++l) m[l] = v[l].z;
-      count_word(m);
-#pragma unroll
-      for (int l = 0; l < kSelMaxLayers; ++l) m[l] = v[l].w;
-      count_word(m);
-    }
-  } else {
-    for (int i = tid; i < w0; i += kCompactThreads) {
-      uint32_t m[kSelMaxLayers];
-#pragma unroll
-      for (int l = 0; l < kSelMaxLayers; ++l) m[l] = l < L ? __ldg(mb + l * lstride + i) : 0u;
-      count_word(m);
+  for (int l = 0; l < kSelMaxLayers; ++l) {
+    pc[l] = 0;
+    if (l < L && wi < Nw) {
+      const uint32_t m = __ldg(mb + l * lstride + wi);
+      pc[l] = __popc(m & ~acc);
+      acc |= m;
     }
   }
+  pc[kSelMaxLayers] = __popc(acc);
 #pragma unroll
   for (int j = 0; j <= kSelMaxLayers; ++j) {
 #pragma unroll
@@ -195,6 +164,32 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
     if (lane == 0) sred[j][warp] = pc[j];
   }
   __syncthreads();
+  if (tid <= kSelMaxLayers) {
+    int t = 0;
+    for (int w = 0; w < kCompactThreads / 32; ++w) t += sred[tid][w];
+    counts[(static_cast<size_t>(b) * gridDim.x + chunk) * (kSelMaxLayers + 1) + tid] = t;
+  }
+}
+
+__global__ void __launch_bounds__(kCompactThreads)
+select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, int Nw, int cap,
+                    const int32_t* __restrict__ counts, uint32_t* __restrict__ U, uint32_t* __restrict__ nw,
+                    int32_t* __restrict__ idx_new, int32_t* __restrict__ cnt_new, size_t cstride,
+                    int32_t* __restrict__ idx_U, int32_t* __restrict__ cnt_U, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int base_s[kSelMaxLayers + 1];
+  __shared__ int wsum[kSelMaxLayers + 1][kCompactThreads / 32];
+  const int b = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t* mb = mask + static_cast<size_t>(b) * Nw;
+  const int w0 = chunk * kCompactWords;
+  // bases: the lists' set bits in the earlier chunks of this sequence
+  if (tid <= kSelMaxLayers) {
+    int t = 0;
+    const int32_t* cb = counts + static_cast<size_t>(b) * gridDim.x * (kSelMaxLayers + 1) + tid;
+    for (int c = 0; c < chunk; ++c) t += __ldg(cb + c * (kSelMaxLayers + 1));
+    base_s[tid] = t;
+  }
   // own word
   const int wi = w0 + tid;
   uint32_t word[kSelMaxLayers + 1];
@@ -233,9 +228,9 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
 #pragma unroll 1
   for (int j = 0; j <= L; ++j) {
     const int jj = j == L ? kSelMaxLayers : j;
-    int base = 0, before = 0, total = 0;
+    const int base = base_s[jj];
+    int before = 0, total = 0;
     for (int w = 0; w < kCompactThreads / 32; ++w) {
-      base += sred[jj][w];
       const int ws = wsum[jj][w];
       before += w < warp ? ws : 0;
       total += ws;
@@ -269,13 +264,14 @@ __device__ __forceinline__ uint32_t order_key(float x) {
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kTopkSmemKeys = 45056;   // keys of one CTA's candidate slice held in shared memory
+constexpr int kTopkSmemKeys = 32768;   // keys of one CTA's candidate slice held in shared memory
+constexpr int kSubHists = 8;           // digit histograms, one per four warps (fewer same-bin collisions)
 constexpr int kDigitBins = 2048;       // radix digits of 11, 11 and 10 bits
 constexpr int kBinsPerThread = kDigitBins / kTopkThreads;
 static_assert(kBinsPerThread == 2, "two digit bins per thread");
 
 struct TopkShared {
-  int sub[2][kDigitBins];    // digit histograms, one per half of the warps
+  int sub[kSubHists][kDigitBins];   // digit histograms, one per four warps
   int hist[2][kDigitBins];   // this CTA's digit histogram by pass parity, read by the whole cluster
   int warp_tmp[32];
   int wgt[kTopkWarps], weq[kTopkWarps];   // per-warp counts of keys above T and equal to T
@@ -285,6 +281,7 @@ struct TopkShared {
   int kk;
   int total;
 };
+constexpr int kTopkStateBytes = (static_cast<int>(sizeof(TopkShared)) + 15) / 16 * 16;
 
 // Candidates and keys come in one of two ways.  Fetched-set mode: candidate j is entry
 // idx[b][j] (j < count[b]) with key order_key(max over layers of logit[l][b][entry]),
@@ -308,8 +305,12 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
                     const uint32_t* __restrict__ dkeys, const int32_t* __restrict__ kdev,
                     const int32_t* __restrict__ kept, int32_t* status,
                     uint32_t* __restrict__ keys_ws, int32_t* __restrict__ topk, int32_t* __restrict__ topk_count) {
-  extern __shared__ uint32_t skeys[];
-  __shared__ TopkShared sh;
+  pdl_wait();
+  pdl_trigger();
+  // dynamic shared memory: the shared state, then the key slice
+  extern __shared__ __align__(16) uint8_t topk_smem[];
+  TopkShared& sh = *reinterpret_cast<TopkShared*>(topk_smem);
+  uint32_t* skeys = reinterpret_cast<uint32_t*>(topk_smem + kTopkStateBytes);
   cg::cluster_group cl = cg::this_cluster();
   const int cs = static_cast<int>(cl.num_blocks());
   const int rank = static_cast<int>(cl.block_rank());
@@ -376,9 +377,9 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
   for (int pass = 0; pass < 3; ++pass) {
     const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
     const uint32_t dmask = pass == 2 ? 1023u : 2047u;
-    for (int i = tid; i < 2 * kDigitBins; i += kTopkThreads) (&sh.sub[0][0])[i] = 0;
+    for (int i = tid; i < kSubHists * kDigitBins; i += kTopkThreads) (&sh.sub[0][0])[i] = 0;
     __syncthreads();
-    int* mysub = sh.sub[warp & 1];
+    int* mysub = sh.sub[warp % kSubHists];
     for (int j = tid; j < mloc; j += kTopkThreads) {
       const uint32_t u = key[j];
       if ((u & himask) == prefix) atomicAdd(&mysub[(u >> shift) & dmask], 1);
@@ -387,7 +388,10 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
 #pragma unroll
     for (int q = 0; q < kBinsPerThread; ++q) {
       const int d = tid * kBinsPerThread + q;
-      sh.hist[pass & 1][d] = sh.sub[0][d] + sh.sub[1][d];
+      int h = 0;
+#pragma unroll
+      for (int c = 0; c < kSubHists; ++c) h += sh.sub[c][d];
+      sh.hist[pass & 1][d] = h;
     }
     // After this barrier every CTA's histogram of the pass is complete.  A CTA rewrites
     // hist[pass & 1] two passes later, after the next barrier, which no CTA passes
@@ -503,23 +507,32 @@ int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, in
   return check_launch("compact", launches);
 }
 
+size_t select_fetch_workspace_bytes(int B, int N) {
+  const int Nw = (N + 31) / 32;
+  const size_t chunks = std::max(1, (Nw + kCompactWords - 1) / kCompactWords);
+  return static_cast<size_t>(B) * chunks * (kSelMaxLayers + 1) * 4;
+}
+
 int launch_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* nw, int cap,
                         int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
-                        cudaStream_t s) {
+                        int32_t* counts, cudaStream_t s) {
   if (B == 0) return LSA_OK;
   const int Nw = (N + 31) / 32;
   const size_t lstride = static_cast<size_t>(B) * Nw;
+  const int chunks = std::max(1, (Nw + kCompactWords - 1) / kCompactWords);
   constexpr int kSeqPerLaunch = 65535;   // the sequence index is gridDim.y
   int launches = 0;
   for (int b0 = 0; b0 < B; b0 += kSeqPerLaunch) {
     const int nb = std::min(kSeqPerLaunch, B - b0);
-    const dim3 grid(std::max(1, (Nw + kCompactWords - 1) / kCompactWords), nb);
+    const dim3 grid(chunks, nb);
     const size_t o = static_cast<size_t>(b0) * Nw;
-    select_fetch_kernel<<<grid, kCompactThreads, 0, s>>>(
-        mask + o, L, lstride, Nw, cap, U ? U + o : nullptr, nw ? nw + o : nullptr,
-        idx_new + static_cast<size_t>(b0) * cap, cnt_new + b0, static_cast<size_t>(B),
-        idx_U + static_cast<size_t>(b0) * cap, cnt_U + b0, status);
-    ++launches;
+    int32_t* cnt = counts + static_cast<size_t>(b0) * chunks * (kSelMaxLayers + 1);
+    launch_dependent(select_count_kernel, grid, dim3(kCompactThreads), 0, s, mask + o, L, lstride, Nw, cnt);
+    launch_dependent(select_fetch_kernel, grid, dim3(kCompactThreads), 0, s, mask + o, L, lstride, Nw, cap,
+                     static_cast<const int32_t*>(cnt), U ? U + o : nullptr, nw ? nw + o : nullptr,
+                     idx_new + static_cast<size_t>(b0) * cap, cnt_new + b0, static_cast<size_t>(B),
+                     idx_U + static_cast<size_t>(b0) * cap, cnt_U + b0, status);
+    launches += 2;
   }
   return check_launch("select_fetch", launches);
 }
@@ -529,7 +542,7 @@ namespace {
 int launch_topk_cluster(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
                         const float* logit, const uint32_t* dkeys, const int32_t* kdev, const int32_t* kept,
                         int32_t* status, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws, cudaStream_t s) {
-  const int smem = kTopkSmemKeys * 4;
+  const int smem = kTopkStateBytes + kTopkSmemKeys * 4;
   cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
   int sms = 148, dev = 0;
@@ -542,13 +555,15 @@ int launch_topk_cluster(int B, int L, int N, int k, const int32_t* idx, int cap,
   while (cs > 1 && B * cs > sms) cs >>= 1;
   while (cs < 8 && (cap + cs - 1) / cs > kTopkSmemKeys) cs <<= 1;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // a dependent launch (pdl_wait in the kernel)
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(kTopkThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   for (;; cs >>= 1) {
     attr[0].val.clusterDim.x = cs;
     attr[0].val.clusterDim.y = 1;

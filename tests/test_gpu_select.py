@@ -111,7 +111,8 @@ def _select_fetch(marks, cap, want_words=True):
     idx_U = torch.full((B, capd), -7, dtype=torch.int32, device="cuda")
     cnt_U = torch.full((B,), -7, dtype=torch.int32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    lsa.lsa_select_fetch(B, L, N, mask, U, new, cap, idx_new, cnt_new, idx_U, cnt_U, st)
+    ws = lsa.workspace(lsa.lsa_select_fetch_workspace_bytes(B, N))
+    lsa.lsa_select_fetch(B, L, N, mask, U, new, cap, idx_new, cnt_new, idx_U, cnt_U, ws, status=st)
     torch.cuda.synchronize()
     out = dict(idx_new=idx_new.cpu().numpy(), cnt_new=cnt_new.cpu().numpy(), idx_U=idx_U.cpu().numpy(),
                cnt_U=cnt_U.cpu().numpy(), status=int(st.item()))

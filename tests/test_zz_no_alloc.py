@@ -80,13 +80,13 @@ def test_noalloc_matches_workspace_variant_twice():
 def test_noalloc_uses_the_whole_scratch_array_twice():
     """B = 16, cap = 2^19: B * cap is the array's full size, and each sequence's slice per
     CTA (up to 8 CTAs per sequence: 65,536 candidates) exceeds the shared-memory slice of
-    45,056 keys, so the keys live in the built-in array.  Two calls with different inputs
+    32,768 keys, so the keys live in the built-in array.  Two calls with different inputs
     in a row: the second runs over the first one's leftovers."""
     B, L, N, cap, k = 16, 3, 600000, 1 << 19, 2048
     assert B * cap == SCRATCH_SLOTS
     for seed in (3, 4):
         logit_np, idx_np, cnt_np, logit, idx, cnt = _case(seed, B, L, N, cap, lo=cap - 30000)
-        assert int(cnt_np.min()) > 8 * 45056          # the key slices go to the array
+        assert int(cnt_np.min()) > 8 * 32768          # the key slices go to the array
         ref, ref_n, got, got_n = _both(B, L, N, k, cap, logit, idx, cnt)
         assert np.array_equal(got_n, ref_n)
         assert np.array_equal(got, ref)
