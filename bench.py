@@ -163,6 +163,7 @@ class Trigger:
                     if cold is not None else None)
         self.idx_U = torch.empty(B, N, dtype=torch.int32, device=device)
         self.cnt_U = torch.zeros(B, dtype=torch.int32, device=device)
+        self.key_U = torch.empty(B, N, dtype=torch.int32, device=device)   # the union's top-k keys (uint32 bits)
         self.topk = torch.empty(B, w.k, dtype=torch.int32, device=device)
         self.topk_cnt = torch.zeros(B, dtype=torch.int32, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
@@ -194,9 +195,10 @@ class Trigger:
 
     def run_batched(self, record=False):
         """One trigger, all layers scored in one launch (HBM-bound, ~0.55 ms), then one
-        launch forms the union, the per-layer new sets and all fetch lists, and the top-k
-        runs (it ranks by the indexer logits, so it does not wait for the rows); then the
-        side stream gathers the new rows of each layer over the host link (tens of ms)."""
+        call forms the union, the per-layer new sets, all fetch lists and the union's top-k
+        keys, and the top-k runs on those keys (it ranks by the indexer logits, so it does
+        not wait for the rows); then the side stream gathers the new rows of each layer
+        over the host link (tens of ms)."""
         lsa, w, inp = self.lsa, self.w, self.inp
         B, L, N = w.B, w.L, w.N
         m, sd = self.main, self.side
@@ -216,9 +218,9 @@ class Trigger:
                 e["score"][l][0].record(m)
                 e["score"][l][1].record(m)
         lsa.lsa_select_fetch(B, L, N, self.mask, self.U, self.new, self.cap, self.idx_new, self.cnt_new,
-                             self.idx_U, self.cnt_U, self.ws_sel, status=self.status, stream=m)
-        lsa.lsa_topk(B, L, N, w.k, self.idx_U, N, self.cnt_U, self.logit, self.topk, self.topk_cnt, self.ws_topk,
-                     stream=m)
+                             self.idx_U, self.cnt_U, self.ws_sel, logit=self.logit, key_U=self.key_U,
+                             status=self.status, stream=m)
+        lsa.lsa_topk_keyed(B, w.k, self.idx_U, N, self.cnt_U, self.key_U, self.topk, self.topk_cnt, stream=m)
         if record:
             e["select"][1].record(m)
         selected = torch.cuda.Event()
@@ -249,9 +251,9 @@ class Trigger:
                             self.kdt, inp["K"], inp["kscale"], -1, self.q, self.wv, None, None,
                             self.mask, self.logit, None, self.ws_score, status=self.status, stream=m)
         lsa.lsa_select_fetch(B, L, N, self.mask, self.U, self.new, self.cap, self.idx_new, self.cnt_new,
-                             self.idx_U, self.cnt_U, self.ws_sel, status=self.status, stream=m)
-        lsa.lsa_topk(B, L, N, w.k, self.idx_U, N, self.cnt_U, self.logit, self.topk, self.topk_cnt, self.ws_topk,
-                     stream=m)
+                             self.idx_U, self.cnt_U, self.ws_sel, logit=self.logit, key_U=self.key_U,
+                             status=self.status, stream=m)
+        lsa.lsa_topk_keyed(B, w.k, self.idx_U, N, self.cnt_U, self.key_U, self.topk, self.topk_cnt, stream=m)
         torch.cuda.current_stream().wait_stream(m)
 
     def run_per_layer(self, record=False):
@@ -543,14 +545,14 @@ def hot_pool_measure(lsa, trig, device, triggers=8, rho=0.9):
                             trig.kdt, inp["K"], inp["kscale"], -1, trig.q, trig.wv, None, None,
                             trig.mask, trig.logit, None, trig.ws_score, status=status, stream=m)
         lsa.lsa_select_fetch(B, L, N, trig.mask, trig.U, None, trig.cap, trig.idx_new, trig.cnt_new,
-                             trig.idx_U, trig.cnt_U, trig.ws_sel, status=status, stream=m)
+                             trig.idx_U, trig.cnt_U, trig.ws_sel, logit=trig.logit, key_U=trig.key_U,
+                             status=status, stream=m)
         ready = torch.cuda.Event()
         ready.record(m)
         sd.wait_event(ready)
         lsa.lsa_hot_pool_update(B, N, slots, w.row_bytes, t, trig.U, trig.cold, hot, state, moved, status, ws,
                                 stream=sd)
-        lsa.lsa_topk(B, L, N, w.k, trig.idx_U, N, trig.cnt_U, trig.logit, trig.topk, trig.topk_cnt, trig.ws_topk,
-                     stream=m)
+        lsa.lsa_topk_keyed(B, w.k, trig.idx_U, N, trig.cnt_U, trig.key_U, trig.topk, trig.topk_cnt, stream=m)
         done = torch.cuda.Event()
         done.record(sd)
         m.wait_event(done)

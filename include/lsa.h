@@ -178,7 +178,11 @@ int lsa_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32
  *   leaves them); U [B][Nw] and new_l [L][B][Nw] outputs or NULL; idx_new [L][B][cap],
  *   cnt_new [L][B], idx_U [B][cap], cnt_U [B] int32 outputs.  A count above cap is
  *   reported as is, only cap indices are written and *status (device int32 or NULL) is
- *   raised to LSA_ERR_CAPACITY.  1 <= L <= 8, else LSA_ERR_UNSUPPORTED.  Device
+ *   raised to LSA_ERR_CAPACITY.  logit [L][B][N] fp32 and key_U [B][cap] uint32, both
+ *   or neither: key_U[b][j] = order key of max over layers of logit[l][b][idx_U[b][j]]
+ *   (the float's sign-magnitude bits mapped so that larger floats give larger keys),
+ *   the keys lsa_topk ranks by, for lsa_topk_keyed.
+ *   1 <= L <= 8, else LSA_ERR_UNSUPPORTED.  Device
  *   pointers 16-byte aligned (counts 4-byte).  Two launches (per-chunk counts, then the
  *   lists) per block of 65535 sequences.
  * workspace: lsa_select_fetch_workspace_bytes(B, N) bytes, 256-byte aligned.
@@ -186,8 +190,21 @@ int lsa_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32
 size_t lsa_select_fetch_workspace_bytes(int B, int N);
 
 int lsa_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* new_l, int cap,
-                     int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
-                     void* workspace, size_t workspace_bytes, void* stream);
+                     int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, const float* logit,
+                     uint32_t* key_U, int32_t* status, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * lsa_topk_keyed -- lsa_topk with the candidates' keys given: candidate j of sequence b
+ * is entry idx[b][j] with key key[b][j] (an unsigned integer; larger ranks first, equal
+ * keys by ascending j, i.e. ascending entry for an ascending list), j < min(count[b],
+ * cap).  Results as lsa_topk: the first min(k, n) in ascending entry order in
+ * topk[b][0..], -1 after them, topk_count[b] = min(k, n).  With key_U from
+ * lsa_select_fetch it returns exactly what lsa_topk returns on the same lists and
+ * logits ([SUMMARY] §2.1 hierarchical selection), without gathering the logits again.
+ *   idx, key [B][cap], count [B], topk [B][k], topk_count [B] or NULL.  No workspace.
+ * ---------------------------------------------------------------------------------- */
+int lsa_topk_keyed(int B, int k, const int32_t* idx, int cap, const int32_t* count, const uint32_t* key,
+                   int32_t* topk, int32_t* topk_count, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * lsa_topk -- fine top-k inside the fetched subset ([SUMMARY] §2.1 hierarchical

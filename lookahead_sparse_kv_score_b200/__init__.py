@@ -126,11 +126,16 @@ def lsa_select_fetch_workspace_bytes(B, N) -> int:
     return int(lib().lsa_select_fetch_workspace_bytes(B, N))
 
 
-def lsa_select_fetch(B, L, N, mask, U, new_l, cap, idx_new, cnt_new, idx_U, cnt_U, workspace, status=None,
-                     stream=None):
+def lsa_select_fetch(B, L, N, mask, U, new_l, cap, idx_new, cnt_new, idx_U, cnt_U, workspace, logit=None,
+                     key_U=None, status=None, stream=None):
     _check(lib().lsa_select_fetch(B, L, N, _p(mask), _p(U), _p(new_l), cap, _p(idx_new), _p(cnt_new), _p(idx_U),
-                                  _p(cnt_U), _p(status), _p(workspace), 0 if workspace is None else workspace.numel(),
-                                  _stream(stream)), "lsa_select_fetch")
+                                  _p(cnt_U), _p(logit), _p(key_U), _p(status), _p(workspace),
+                                  0 if workspace is None else workspace.numel(), _stream(stream)), "lsa_select_fetch")
+
+
+def lsa_topk_keyed(B, k, idx, cap, count, key, topk, topk_count, stream=None):
+    _check(lib().lsa_topk_keyed(B, k, _p(idx), cap, _p(count), _p(key), _p(topk), _p(topk_count), _stream(stream)),
+           "lsa_topk_keyed")
 
 
 def lsa_topk_workspace_bytes(B, cap) -> int:

@@ -29,7 +29,8 @@ SIGNATURES = {
     "lsa_compact": (c_int, [c_int, c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "lsa_select_fetch_workspace_bytes": (c_size_t, [c_int, c_int]),
     "lsa_select_fetch": (c_int, [c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p,
-                                 c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+                                 c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "lsa_topk_keyed": (c_int, [c_int, c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "lsa_topk_workspace_bytes": (c_size_t, [c_int, c_int]),
     "lsa_topk": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
                          c_void_p, c_void_p, c_size_t, c_void_p]),

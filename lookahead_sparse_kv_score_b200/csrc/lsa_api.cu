@@ -262,8 +262,8 @@ size_t lsa_select_fetch_workspace_bytes(int B, int N) {
 }
 
 int lsa_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* new_l, int cap,
-                     int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
-                     void* workspace, size_t workspace_bytes, void* stream) {
+                     int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, const float* logit,
+                     uint32_t* key_U, int32_t* status, void* workspace, size_t workspace_bytes, void* stream) {
   const CallRange range("lsa_select_fetch");
   g_err[0] = 0;
   if (B < 0 || L < 0 || N < 0 || cap < 0) return fail(LSA_ERR_INVALID_ARG, "select_fetch: negative size");
@@ -273,13 +273,27 @@ int lsa_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uin
     return fail(LSA_ERR_INVALID_ARG, "select_fetch: null pointer");
   if ((mask && !aligned(mask, 16)) || (U && !aligned(U, 16)) || (new_l && !aligned(new_l, 16)) ||
       (idx_new && !aligned(idx_new, 16)) || (idx_U && !aligned(idx_U, 16)) || !aligned(cnt_new, 4) ||
-      !aligned(cnt_U, 4))
+      !aligned(cnt_U, 4) || (key_U && !aligned(key_U, 16)) || (logit && !aligned(logit, 4)))
     return fail(LSA_ERR_INVALID_ARG, "select_fetch: misaligned pointer");
+  if (key_U && cap > 0 && !logit) return fail(LSA_ERR_INVALID_ARG, "select_fetch: key_U needs the logits");
   const size_t need = lsa_select_fetch_workspace_bytes(B, N);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
     return fail(LSA_ERR_NOMEM, "select_fetch: workspace %zu bytes (need %zu)", workspace_bytes, need);
   return launch_select_fetch(B, L, N, mask, U, new_l, cap, idx_new, cnt_new, idx_U, cnt_U, status,
-                             static_cast<int32_t*>(workspace), static_cast<cudaStream_t>(stream));
+                             static_cast<int32_t*>(workspace), logit, key_U, static_cast<cudaStream_t>(stream));
+}
+
+int lsa_topk_keyed(int B, int k, const int32_t* idx, int cap, const int32_t* count, const uint32_t* key,
+                   int32_t* topk, int32_t* topk_count, void* stream) {
+  const CallRange range("lsa_topk_keyed");
+  g_err[0] = 0;
+  if (B < 0 || k < 0 || cap < 0) return fail(LSA_ERR_INVALID_ARG, "topk_keyed: negative size");
+  if (B == 0) return LSA_OK;
+  if (!count || (cap > 0 && (!idx || !key)) || (k > 0 && !topk))
+    return fail(LSA_ERR_INVALID_ARG, "topk_keyed: null pointer");
+  if ((idx && !aligned(idx, 4)) || (key && !aligned(key, 4)) || !aligned(count, 4))
+    return fail(LSA_ERR_INVALID_ARG, "topk_keyed: misaligned pointer");
+  return launch_topk_keyed(B, k, idx, cap, count, key, topk, topk_count, static_cast<cudaStream_t>(stream));
 }
 
 // Workspace of lsa_fine_score: query images, folded head weights, tile prefix.

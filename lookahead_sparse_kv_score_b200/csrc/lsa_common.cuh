@@ -161,7 +161,10 @@ int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, in
 size_t select_fetch_workspace_bytes(int B, int N);
 int launch_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* nw, int cap,
                         int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
-                        int32_t* counts, cudaStream_t s);
+                        int32_t* counts, const float* logit, uint32_t* key_U, cudaStream_t s);
+// The top-k with given per-candidate order keys (keys[b][j] for candidate idx[b][j]).
+int launch_topk_keyed(int B, int k, const int32_t* idx, int cap, const int32_t* count, const uint32_t* keys,
+                      int32_t* topk, int32_t* topk_count, cudaStream_t s);
 int launch_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const int32_t* count,
                 const float* logit, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws,
                 cudaStream_t s);

@@ -125,14 +125,20 @@ compact_kernel(const uint32_t* __restrict__ bits, int Nw, int cap, int32_t* __re
   }
 }
 
+// Order-preserving integer image of a float key: larger float -> larger key.
+__device__ __forceinline__ uint32_t order_key(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // ------------------------------------------------------------------ union + fetch lists
 // The whole selection of one trigger in two launches over the L layer masks: per word,
 // new_l = mask_l & ~(mask_0 | .. | mask_{l-1}) and U = mask_0 | .. | mask_{L-1}, and the
 // L + 1 fetch lists (new_0 .. new_{L-1}, U) with their counts.  Block (chunk, b) owns
 // words [chunk*kCompactWords, ...) of sequence b.  The first launch writes each chunk's
 // popcounts of the L + 1 sets; the second takes its output bases from the earlier
-// chunks' counts, and each thread writes its own word's indices (a warp's threads cover
-// one contiguous run of every list).
+// chunks' counts; each warp stages its run of every list in shared memory and copies it
+// out with full stores.
 constexpr int kSelMaxLayers = 8;
 
 // Per (chunk, sequence): the popcounts of the chunk's words in the L new sets and the
@@ -175,11 +181,13 @@ __global__ void __launch_bounds__(kCompactThreads)
 select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, int Nw, int cap,
                     const int32_t* __restrict__ counts, uint32_t* __restrict__ U, uint32_t* __restrict__ nw,
                     int32_t* __restrict__ idx_new, int32_t* __restrict__ cnt_new, size_t cstride,
-                    int32_t* __restrict__ idx_U, int32_t* __restrict__ cnt_U, int32_t* status) {
+                    int32_t* __restrict__ idx_U, int32_t* __restrict__ cnt_U, int32_t* status,
+                    const float* __restrict__ logit, int Bfull, int b_off, int N, uint32_t* __restrict__ key_U) {
   pdl_wait();
   pdl_trigger();
   __shared__ int base_s[kSelMaxLayers + 1];
   __shared__ int wsum[kSelMaxLayers + 1][kCompactThreads / 32];
+  __shared__ int32_t wstage[kCompactThreads / 32][32 * 32];   // one warp's words hold at most 1024 indices
   const int b = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t* mb = mask + static_cast<size_t>(b) * Nw;
   const int w0 = chunk * kCompactWords;
@@ -210,8 +218,8 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
   }
   const bool last = chunk == static_cast<int>(gridDim.x) - 1;
   // every list's offsets for the block in one pass: warp prefix sums of the popcounts,
-  // one barrier, then the warps' bases; each thread writes its word's indices directly
-  // (a warp's threads cover one contiguous run of each list)
+  // one barrier, then the warps' bases (a warp's threads cover one contiguous run of
+  // each list)
   int incl[kSelMaxLayers + 1];
 #pragma unroll
   for (int q = 0; q <= kSelMaxLayers; ++q) {
@@ -240,14 +248,38 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
 #pragma unroll
     for (int q = 0; q <= kSelMaxLayers; ++q)
       if (q == jj) { bits = word[q]; inc = incl[q]; }
-    int pos = base + before + inc - __popc(bits);
-    int32_t* out = (j == L ? idx_U + static_cast<size_t>(b) * cap : idx_new + j * cstride * cap + static_cast<size_t>(b) * cap);
+    // the warp's run of this list: staged in its own shared buffer in list order, then
+    // copied out with full 128-byte stores
+    int32_t* stage = wstage[warp];
+    int wp = inc - __popc(bits);                     // this lane's offset inside the warp's run
     while (bits) {
       const int bit = __ffs(bits) - 1;
       bits &= bits - 1;
-      if (pos < cap) out[pos] = wi * 32 + bit;
-      ++pos;
+      stage[wp++] = wi * 32 + bit;
     }
+    __syncwarp();
+    const int wtot = __shfl_sync(0xffffffffu, inc, 31);
+    const int wbase = base + before;
+    int32_t* out = (j == L ? idx_U + static_cast<size_t>(b) * cap : idx_new + j * cstride * cap + static_cast<size_t>(b) * cap);
+    if (j == L && key_U) {
+      // the union's candidates also get their top-k key: the order image of the largest
+      // logit over the layers (read in list order, i.e. ascending entries)
+      uint32_t* kout = key_U + static_cast<size_t>(b) * cap;
+      const float* lb = logit + static_cast<size_t>(b_off + b) * N;
+      const size_t lstep = static_cast<size_t>(Bfull) * N;
+      for (int i = lane; i < wtot; i += 32) {
+        if (wbase + i >= cap) break;
+        const int e = stage[i];
+        float z = __ldg(lb + e);
+        for (int l = 1; l < L; ++l) z = fmaxf(z, __ldg(lb + l * lstep + e));
+        out[wbase + i] = e;
+        kout[wbase + i] = order_key(z);
+      }
+    } else {
+      for (int i = lane; i < wtot; i += 32)
+        if (wbase + i < cap) out[wbase + i] = stage[i];
+    }
+    __syncwarp();
     if (last && tid == 0) {
       int32_t* cnt = j == L ? cnt_U + b : cnt_new + j * cstride + b;
       *cnt = base + total;
@@ -257,10 +289,6 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
 }
 
 // ------------------------------------------------------------------ top-k
-__device__ __forceinline__ uint32_t order_key(float x) {
-  const uint32_t u = __float_as_uint(x);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);   // larger float -> larger key
-}
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
@@ -316,7 +344,8 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
   const int rank = static_cast<int>(cl.block_rank());
   const int b = blockIdx.x / cs;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const bool direct = dkeys != nullptr;
+  const bool direct = dkeys != nullptr && idx == nullptr;   // keys given per slot, outputs are slots
+  const bool keyed = dkeys != nullptr && idx != nullptr;     // keys given per candidate of idx
   int n, kb;                         // candidates and keys to keep for this sequence
   if (direct) {
     n = cap;
@@ -341,9 +370,15 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
   }
   const int m = (n + cs - 1) / cs;
   const int j0 = min(n, rank * m), mloc = min(n, j0 + m) - j0;
-  uint32_t* key = m <= kTopkSmemKeys ? skeys : keys_ws + static_cast<size_t>(b) * cap + j0;
-  if (direct) {
-    for (int j = tid; j < mloc; j += kTopkThreads) key[j] = __ldg(dkeys + static_cast<size_t>(b) * cap + j0 + j);
+  // the slice's keys: in shared memory when they fit; otherwise read in place (given keys)
+  // or computed into the key workspace
+  const bool in_smem = m <= kTopkSmemKeys;
+  uint32_t* key = in_smem ? skeys
+                          : ((direct || keyed) ? const_cast<uint32_t*>(dkeys) + static_cast<size_t>(b) * cap + j0
+                                               : keys_ws + static_cast<size_t>(b) * cap + j0);
+  if (direct || keyed) {
+    if (in_smem)
+      for (int j = tid; j < mloc; j += kTopkThreads) key[j] = __ldg(dkeys + static_cast<size_t>(b) * cap + j0 + j);
   } else {
     // eight candidates per thread in flight: their entries first, then every layer's logits
     constexpr int kBatch = 8;
@@ -515,7 +550,7 @@ size_t select_fetch_workspace_bytes(int B, int N) {
 
 int launch_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* nw, int cap,
                         int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
-                        int32_t* counts, cudaStream_t s) {
+                        int32_t* counts, const float* logit, uint32_t* key_U, cudaStream_t s) {
   if (B == 0) return LSA_OK;
   const int Nw = (N + 31) / 32;
   const size_t lstride = static_cast<size_t>(B) * Nw;
@@ -531,7 +566,8 @@ int launch_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, 
     launch_dependent(select_fetch_kernel, grid, dim3(kCompactThreads), 0, s, mask + o, L, lstride, Nw, cap,
                      static_cast<const int32_t*>(cnt), U ? U + o : nullptr, nw ? nw + o : nullptr,
                      idx_new + static_cast<size_t>(b0) * cap, cnt_new + b0, static_cast<size_t>(B),
-                     idx_U + static_cast<size_t>(b0) * cap, cnt_U + b0, status);
+                     idx_U + static_cast<size_t>(b0) * cap, cnt_U + b0, status, logit, B, b0, N,
+                     key_U ? key_U + static_cast<size_t>(b0) * cap : nullptr);
     launches += 2;
   }
   return check_launch("select_fetch", launches);
@@ -547,13 +583,16 @@ int launch_topk_cluster(int B, int L, int N, int k, const int32_t* idx, int cap,
   cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // CTAs per sequence: as many as keep B x cs within one wave, at most 8 (portable), but
-  // at least enough that a full list (cap candidates) keeps every CTA's slice in shared
-  // memory: the busiest sequence sets the kernel's time, and a slice in global memory
-  // costs more than a second wave of clusters.
+  // CTAs per sequence: as many as keep B x cs within one wave, at most 8 (portable); when
+  // the keys are computed from the logits, at least enough that a full list (cap
+  // candidates) keeps every CTA's slice in shared memory (the busiest sequence sets the
+  // kernel's time, and computing a slice into global memory costs more than a second
+  // wave of clusters).
   int cs = 8;
   while (cs > 1 && B * cs > sms) cs >>= 1;
-  while (cs < 8 && (cap + cs - 1) / cs > kTopkSmemKeys) cs <<= 1;
+  // keys computed here must fit in shared memory; given keys can be read in place
+  if (dkeys == nullptr)
+    while (cs < 8 && (cap + cs - 1) / cs > kTopkSmemKeys) cs <<= 1;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -587,6 +626,13 @@ int launch_topk(int B, int L, int N, int k, const int32_t* idx, int cap, const i
   if (B == 0) return LSA_OK;
   return launch_topk_cluster(B, L, N, k, idx, cap, count, logit, nullptr, nullptr, nullptr, nullptr, topk,
                              topk_count, keys_ws, s);
+}
+
+int launch_topk_keyed(int B, int k, const int32_t* idx, int cap, const int32_t* count, const uint32_t* keys,
+                      int32_t* topk, int32_t* topk_count, cudaStream_t s) {
+  if (B == 0) return LSA_OK;
+  return launch_topk_cluster(B, 1, 0, k, idx, cap, count, nullptr, keys, nullptr, nullptr, nullptr, topk, topk_count,
+                             nullptr, s);
 }
 
 int launch_select_keys(int B, int n, const uint32_t* keys, const int32_t* kdev, const int32_t* kept,

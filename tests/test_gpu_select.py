@@ -188,6 +188,43 @@ def test_select_fetch_more_sequences_than_one_launch():
     assert (out["cnt_U"] == marks.any(axis=0).sum(axis=1)).all()
 
 
+@pytest.mark.parametrize("B,N,k", [(5, 40000, 512), (3, 262144, 2048), (2, 3000, 5000)])
+def test_topk_keyed_with_selection_keys_equals_topk(B, N, k):
+    """The union's keys written by lsa_select_fetch and lsa_topk_keyed on them give
+    exactly lsa_topk's result (keys over the logits of every layer) and the oracle's."""
+    g = np.random.default_rng(N + k)
+    L = 3
+    marks = g.random((L, B, N)) < 0.25
+    logits = np.round(g.standard_normal((L, B, N)) * 4, 1).astype(np.float32)   # ties
+    Nw = (N + 31) // 32
+    mask = torch.from_numpy(O.pack_bits(marks).view(np.int32).copy()).cuda()
+    lg = torch.from_numpy(logits).cuda()
+    idx_new = torch.empty(L, B, N, dtype=torch.int32, device="cuda")
+    cnt_new = torch.empty(L, B, dtype=torch.int32, device="cuda")
+    idx_U = torch.empty(B, N, dtype=torch.int32, device="cuda")
+    cnt_U = torch.empty(B, dtype=torch.int32, device="cuda")
+    key_U = torch.empty(B, N, dtype=torch.int32, device="cuda")
+    ws = lsa.workspace(lsa.lsa_select_fetch_workspace_bytes(B, N))
+    lsa.lsa_select_fetch(B, L, N, mask, None, None, N, idx_new, cnt_new, idx_U, cnt_U, ws, logit=lg, key_U=key_U)
+    got = torch.full((B, k), -9, dtype=torch.int32, device="cuda")
+    got_n = torch.full((B,), -9, dtype=torch.int32, device="cuda")
+    lsa.lsa_topk_keyed(B, k, idx_U, N, cnt_U, key_U, got, got_n)
+    ref = torch.full((B, k), -9, dtype=torch.int32, device="cuda")
+    ref_n = torch.full((B,), -9, dtype=torch.int32, device="cuda")
+    wst = lsa.workspace(lsa.lsa_topk_workspace_bytes(B, N))
+    lsa.lsa_topk(B, L, N, k, idx_U, N, cnt_U, lg, ref, ref_n, wst)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref) and torch.equal(got_n, ref_n)
+    got, got_n = got.cpu().numpy(), got_n.cpu().numpy()
+    for b in range(B):
+        U = marks[:, b].any(axis=0)
+        fetched = O.compact(U)
+        key = O.fetched_key(logits[:, b].astype(np.float64), np.ones((L, N), dtype=bool))
+        want = O.topk_in_fetched(fetched, key, k)
+        assert got_n[b] == want.size
+        assert np.array_equal(got[b, : want.size], want), b
+
+
 def run_topk(idx_list, logits, k, N):
     L, B = logits.shape[0], len(idx_list)
     cap = max(1, max(len(x) for x in idx_list))
