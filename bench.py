@@ -40,6 +40,8 @@ DEFAULT_WORKLOAD = "lsa_step_1m_b32_fp8"
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "score_tc_fp8_1m_b32_traffic.txt")
 # the score kernel's source: the kernel file and the tcgen05 / TMA wrappers it includes
 SCORE_SRC = [os.path.join(ROOT, "lookahead_sparse_kv_score_b200", "csrc", f) for f in ("score_tc.cu", "tc_ptx.cuh")]
+PROFILE_GATHER = os.path.join(ROOT, "profiles", "gather_cold_1m_host_link.txt")
+GATHER_SRC = [os.path.join(ROOT, "lookahead_sparse_kv_score_b200", "csrc", "gather.cu")]
 
 
 def parse_args(argv=None):
@@ -385,29 +387,47 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def score_source_sha() -> str:
+def source_sha(files) -> str:
     h = hashlib.sha256()
-    for f in SCORE_SRC:
+    for f in files:
         h.update(open(f, "rb").read())
     return h.hexdigest()
+
+
+def score_source_sha() -> str:
+    return source_sha(SCORE_SRC)
+
+
+def profile_fields(path, files):
+    """The key: value lines of a committed ncu summary, or None when it is missing or was
+    taken on another version of the kernel source (its source_sha256 field)."""
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    for line in open(path):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    return kv if kv.get("source_sha256") == source_sha(files) else None
 
 
 def traffic_per_launch():
     """DRAM bytes per score launch from the committed ncu summary, if it was taken on
     the current kernel source (else None)."""
-    if not os.path.exists(PROFILE_TRAFFIC):
-        return None
-    kv = {}
-    for line in open(PROFILE_TRAFFIC):
-        if ":" in line:
-            k, v = line.split(":", 1)
-            kv[k.strip()] = v.strip()
-    sha = score_source_sha()
-    if kv.get("source_sha256") != sha:
-        return None
+    kv = profile_fields(PROFILE_TRAFFIC, SCORE_SRC)
     try:
         return int(kv["dram_bytes_read_per_launch"]) + int(kv["dram_bytes_write_per_launch"])
-    except (KeyError, ValueError):
+    except (KeyError, ValueError, TypeError):
+        return None
+
+
+def gather_link_traffic(payload_bytes):
+    """Host-link bytes a gather of payload_bytes moves, from the committed ncu summary's
+    ratio of PCIe read bytes to payload bytes (None if missing or on other source)."""
+    kv = profile_fields(PROFILE_GATHER, GATHER_SRC)
+    try:
+        return int(round(float(kv["pcie_read_bytes_per_payload_byte"]) * payload_bytes))
+    except (KeyError, ValueError, TypeError):
         return None
 
 
@@ -867,7 +887,9 @@ def our_arm(args):
             "clocks": clk,
             "gpu_launches": launches,
             "roofline_gather": {"bound": "host_link", "achieved": gather_gbs, "peak": link, "unit": "GB/s",
-                                "frac": gather_gbs / link, "traffic": None,
+                                "frac": gather_gbs / link,
+                                "traffic": gather_link_traffic(fetched_rows * w.row_bytes),
+                                "traffic_kind": "PCIe read bytes per step (ncu ratio to payload bytes)",
                                 "kernel": "gather_cold (zero-copy reads of pinned host rows)",
                                 "bytes_per_step": fetched_rows * w.row_bytes, "rows_per_step": fetched_rows,
                                 "ms_per_step": gather_avg,

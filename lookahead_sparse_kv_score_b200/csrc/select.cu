@@ -6,6 +6,7 @@
 // (every entry with I >= 0.5 is fetched) and "hierarchical selection" (a top-k runs
 // inside the fetched subset once it is in GPU memory).
 #include <algorithm>
+#include <type_traits>
 
 #include <cooperative_groups.h>
 
@@ -143,18 +144,20 @@ constexpr int kSelMaxLayers = 8;
 
 // Per (chunk, sequence): the popcounts of the chunk's words in the L new sets and the
 // union, written to counts[b][chunk][kSelMaxLayers + 1] (slot kSelMaxLayers = union).
+// kML >= L bounds the layers the kernel is compiled for (3 or kSelMaxLayers).
+template <int kML>
 __global__ void __launch_bounds__(kCompactThreads)
 select_count_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, int Nw, int32_t* __restrict__ counts) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int sred[kSelMaxLayers + 1][kCompactThreads / 32];
+  __shared__ int sred[kML + 1][kCompactThreads / 32];
   const int b = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t* mb = mask + static_cast<size_t>(b) * Nw;
   const int wi = chunk * kCompactWords + tid;
-  int pc[kSelMaxLayers + 1];
+  int pc[kML + 1];
   uint32_t acc = 0;
 #pragma unroll
-  for (int l = 0; l < kSelMaxLayers; ++l) {
+  for (int l = 0; l < kML; ++l) {
     pc[l] = 0;
     if (l < L && wi < Nw) {
       const uint32_t m = __ldg(mb + l * lstride + wi);
@@ -162,22 +165,24 @@ select_count_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
       acc |= m;
     }
   }
-  pc[kSelMaxLayers] = __popc(acc);
+  pc[kML] = __popc(acc);
 #pragma unroll
-  for (int j = 0; j <= kSelMaxLayers; ++j) {
+  for (int j = 0; j <= kML; ++j) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) pc[j] += __shfl_xor_sync(0xffffffffu, pc[j], o);
     if (lane == 0) sred[j][warp] = pc[j];
   }
   __syncthreads();
-  if (tid <= kSelMaxLayers) {
+  if (tid <= kML) {
     int t = 0;
     for (int w = 0; w < kCompactThreads / 32; ++w) t += sred[tid][w];
-    counts[(static_cast<size_t>(b) * gridDim.x + chunk) * (kSelMaxLayers + 1) + tid] = t;
+    const int slot = tid == kML ? kSelMaxLayers : tid;
+    counts[(static_cast<size_t>(b) * gridDim.x + chunk) * (kSelMaxLayers + 1) + slot] = t;
   }
 }
 
-__global__ void __launch_bounds__(kCompactThreads)
+template <int kML>
+__global__ void __launch_bounds__(kCompactThreads, 4)
 select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, int Nw, int cap,
                     const int32_t* __restrict__ counts, uint32_t* __restrict__ U, uint32_t* __restrict__ nw,
                     int32_t* __restrict__ idx_new, int32_t* __restrict__ cnt_new, size_t cstride,
@@ -185,26 +190,31 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
                     const float* __restrict__ logit, int Bfull, int b_off, int N, uint32_t* __restrict__ key_U) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int base_s[kSelMaxLayers + 1];
-  __shared__ int wsum[kSelMaxLayers + 1][kCompactThreads / 32];
+  __shared__ int base_s[kML + 1];
+  __shared__ int wsum[kML + 1][kCompactThreads / 32];
   __shared__ int32_t wstage[kCompactThreads / 32][32 * 32];   // one warp's words hold at most 1024 indices
   const int b = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t* mb = mask + static_cast<size_t>(b) * Nw;
   const int w0 = chunk * kCompactWords;
-  // bases: the lists' set bits in the earlier chunks of this sequence
-  if (tid <= kSelMaxLayers) {
+  // bases: the lists' set bits in the earlier chunks of this sequence (list q, q = kML
+  // the union, summed by warp q mod 8, its lanes over the chunks, so no load waits on
+  // another)
+  for (int q = warp; q <= kML; q += kCompactThreads / 32) {
+    const int slot = q == kML ? kSelMaxLayers : q;
     int t = 0;
-    const int32_t* cb = counts + static_cast<size_t>(b) * gridDim.x * (kSelMaxLayers + 1) + tid;
-    for (int c = 0; c < chunk; ++c) t += __ldg(cb + c * (kSelMaxLayers + 1));
-    base_s[tid] = t;
+    const int32_t* cb = counts + static_cast<size_t>(b) * gridDim.x * (kSelMaxLayers + 1) + slot;
+    for (int c = lane; c < chunk; c += 32) t += __ldg(cb + c * (kSelMaxLayers + 1));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (lane == 0) base_s[q] = t;
   }
   // own word
   const int wi = w0 + tid;
-  uint32_t word[kSelMaxLayers + 1];
+  uint32_t word[kML + 1];
   {
     uint32_t acc = 0;
 #pragma unroll
-    for (int l = 0; l < kSelMaxLayers; ++l) {
+    for (int l = 0; l < kML; ++l) {
       word[l] = 0u;
       if (l < L && wi < Nw) {
         const uint32_t m = __ldg(mb + l * lstride + wi);
@@ -213,17 +223,17 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
         if (nw) nw[l * lstride + static_cast<size_t>(b) * Nw + wi] = word[l];
       }
     }
-    word[kSelMaxLayers] = acc;
+    word[kML] = acc;
     if (U && wi < Nw) U[static_cast<size_t>(b) * Nw + wi] = acc;
   }
   const bool last = chunk == static_cast<int>(gridDim.x) - 1;
   // every list's offsets for the block in one pass: warp prefix sums of the popcounts,
   // one barrier, then the warps' bases (a warp's threads cover one contiguous run of
   // each list)
-  int incl[kSelMaxLayers + 1];
+  int incl[kML + 1];
 #pragma unroll
-  for (int q = 0; q <= kSelMaxLayers; ++q) {
-    const int v = (q < L || q == kSelMaxLayers) ? __popc(word[q]) : 0;
+  for (int q = 0; q <= kML; ++q) {
+    const int v = (q < L || q == kML) ? __popc(word[q]) : 0;
     incl[q] = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -235,7 +245,7 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
   __syncthreads();
 #pragma unroll 1
   for (int j = 0; j <= L; ++j) {
-    const int jj = j == L ? kSelMaxLayers : j;
+    const int jj = j == L ? kML : j;
     const int base = base_s[jj];
     int before = 0, total = 0;
     for (int w = 0; w < kCompactThreads / 32; ++w) {
@@ -246,8 +256,9 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
     uint32_t bits = 0;
     int inc = 0;
 #pragma unroll
-    for (int q = 0; q <= kSelMaxLayers; ++q)
+    for (int q = 0; q <= kML; ++q)
       if (q == jj) { bits = word[q]; inc = incl[q]; }
+    const uint32_t lbits = bits;
     // the warp's run of this list: staged in its own shared buffer in list order, then
     // copied out with full 128-byte stores
     int32_t* stage = wstage[warp];
@@ -261,23 +272,51 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
     const int wtot = __shfl_sync(0xffffffffu, inc, 31);
     const int wbase = base + before;
     int32_t* out = (j == L ? idx_U + static_cast<size_t>(b) * cap : idx_new + j * cstride * cap + static_cast<size_t>(b) * cap);
+    for (int i = lane; i < wtot; i += 32)
+      if (wbase + i < cap) out[wbase + i] = stage[i];
     if (j == L && key_U) {
-      // the union's candidates also get their top-k key: the order image of the largest
-      // logit over the layers (read in list order, i.e. ascending entries)
+      // The union's candidates also get their top-k key, the order image of the largest
+      // logit over the layers.  The warp's 1024 entries are read densely (lane t: the
+      // float4 of entries 128 k + 4 t), skipping groups with no candidate, and each
+      // candidate's list position comes from its word's offset in the warp's run.
       uint32_t* kout = key_U + static_cast<size_t>(b) * cap;
       const float* lb = logit + static_cast<size_t>(b_off + b) * N;
       const size_t lstep = static_cast<size_t>(Bfull) * N;
-      for (int i = lane; i < wtot; i += 32) {
-        if (wbase + i >= cap) break;
-        const int e = stage[i];
-        float z = __ldg(lb + e);
-        for (int l = 1; l < L; ++l) z = fmaxf(z, __ldg(lb + l * lstep + e));
-        out[wbase + i] = e;
-        kout[wbase + i] = order_key(z);
+      const bool vec = (N % 4 == 0) && (reinterpret_cast<uintptr_t>(logit) % 16 == 0);
+      const int ex = inc - __popc(lbits);             // exclusive offset of this lane's word
+      const int e_warp = (w0 + warp * 32) * 32;       // the warp's first entry
+      const int sh = (lane & 7) * 4;                  // bit of entry 128 k + 4 lane in its word
+#pragma unroll 2
+      for (int k = 0; k < 8; ++k) {
+        const int src = 4 * k + (lane >> 3);          // the word holding those entries
+        const uint32_t uw = __shfl_sync(0xffffffffu, lbits, src);
+        const int off = __shfl_sync(0xffffffffu, ex, src);
+        const uint32_t nib = (uw >> sh) & 0xFu;
+        const int e0 = e_warp + 128 * k + 4 * lane;
+        float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (nib) {
+#pragma unroll
+          for (int l = 0; l < kML; ++l) {
+            if (l >= L) break;
+            const float* src_l = lb + l * lstep + e0;
+            if (vec && e0 + 3 < N) {
+              const float4 v = __ldg(reinterpret_cast<const float4*>(src_l));
+              m[0] = fmaxf(m[0], v.x); m[1] = fmaxf(m[1], v.y); m[2] = fmaxf(m[2], v.z); m[3] = fmaxf(m[3], v.w);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                if (((nib >> i) & 1u) && e0 + i < N) m[i] = fmaxf(m[i], __ldg(src_l + i));
+            }
+          }
+        }
+        int pos = wbase + off + __popc(uw & ((1u << sh) - 1u));
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if ((nib >> i) & 1u) {
+            if (pos < cap) kout[pos] = order_key(m[i]);
+            ++pos;
+          }
       }
-    } else {
-      for (int i = lane; i < wtot; i += 32)
-        if (wbase + i < cap) out[wbase + i] = stage[i];
     }
     __syncwarp();
     if (last && tid == 0) {
@@ -295,6 +334,7 @@ constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkSmemKeys = 32768;   // keys of one CTA's candidate slice held in shared memory
 constexpr int kSubHists = 8;           // digit histograms, one per four warps (fewer same-bin collisions)
 constexpr int kDigitBins = 2048;       // radix digits of 11, 11 and 10 bits
+constexpr int kKeyBatch = 8;           // keys a thread loads before using any
 constexpr int kBinsPerThread = kDigitBins / kTopkThreads;
 static_assert(kBinsPerThread == 2, "two digit bins per thread");
 
@@ -377,8 +417,22 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
                           : ((direct || keyed) ? const_cast<uint32_t*>(dkeys) + static_cast<size_t>(b) * cap + j0
                                                : keys_ws + static_cast<size_t>(b) * cap + j0);
   if (direct || keyed) {
-    if (in_smem)
-      for (int j = tid; j < mloc; j += kTopkThreads) key[j] = __ldg(dkeys + static_cast<size_t>(b) * cap + j0 + j);
+    if (in_smem) {
+      const uint32_t* src = dkeys + static_cast<size_t>(b) * cap + j0;
+      for (int jb = 0; jb < mloc; jb += kKeyBatch * kTopkThreads) {
+        uint32_t v[kKeyBatch];
+#pragma unroll
+        for (int u = 0; u < kKeyBatch; ++u) {
+          const int j = jb + u * kTopkThreads + tid;
+          v[u] = j < mloc ? __ldg(src + j) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kKeyBatch; ++u) {
+          const int j = jb + u * kTopkThreads + tid;
+          if (j < mloc) key[j] = v[u];
+        }
+      }
+    }
   } else {
     // eight candidates per thread in flight: their entries first, then every layer's logits
     constexpr int kBatch = 8;
@@ -415,9 +469,18 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
     for (int i = tid; i < kSubHists * kDigitBins; i += kTopkThreads) (&sh.sub[0][0])[i] = 0;
     __syncthreads();
     int* mysub = sh.sub[warp % kSubHists];
-    for (int j = tid; j < mloc; j += kTopkThreads) {
-      const uint32_t u = key[j];
-      if ((u & himask) == prefix) atomicAdd(&mysub[(u >> shift) & dmask], 1);
+    for (int jb = 0; jb < mloc; jb += kKeyBatch * kTopkThreads) {
+      uint32_t v[kKeyBatch];   // loaded before use: slices in global memory stay latency-hidden
+#pragma unroll
+      for (int u = 0; u < kKeyBatch; ++u) {
+        const int j = jb + u * kTopkThreads + tid;
+        v[u] = j < mloc ? key[j] : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kKeyBatch; ++u) {
+        const int j = jb + u * kTopkThreads + tid;
+        if (j < mloc && (v[u] & himask) == prefix) atomicAdd(&mysub[(v[u] >> shift) & dmask], 1);
+      }
     }
     __syncthreads();
 #pragma unroll
@@ -464,10 +527,19 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
   const int w0 = min(mloc, warp * per), w1 = min(mloc, w0 + per);
   {
     int gt = 0, eq = 0;
-    for (int j = w0 + lane; j < w1; j += 32) {
-      const uint32_t u = key[j];
-      gt += u > T;
-      eq += u == T;
+    for (int jb = w0; jb < w1; jb += 32 * kKeyBatch) {
+      uint32_t v[kKeyBatch];
+#pragma unroll
+      for (int u = 0; u < kKeyBatch; ++u) {
+        const int j = jb + u * 32 + lane;
+        v[u] = j < w1 ? key[j] : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kKeyBatch; ++u) {
+        const int j = jb + u * 32 + lane;
+        gt += j < w1 && v[u] > T;
+        eq += j < w1 && v[u] == T;
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -501,17 +573,26 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
   int gt_before = sh.gbase, eq_before = sh.ebase;
   for (int w = 0; w < warp; ++w) { gt_before += sh.wgt[w]; eq_before += sh.weq[w]; }
   const uint32_t lt = (1u << lane) - 1u;
-  for (int jb = w0; jb < w1; jb += 32) {
-    const int j = jb + lane;
-    const uint32_t u = j < w1 ? key[j] : 0u;
-    const bool g = j < w1 && u > T, q = j < w1 && u == T;
-    const uint32_t gm = __ballot_sync(0xffffffffu, g), qm = __ballot_sync(0xffffffffu, q);
-    const int gb = gt_before + __popc(gm & lt), qb = eq_before + __popc(qm & lt);
-    const int c = j0 + j;
-    if (g) ob[gb + min(qb, kk)] = direct ? c : __ldg(ib + c);
-    else if (q && qb < kk) ob[gb + qb] = direct ? c : __ldg(ib + c);
-    gt_before += __popc(gm);
-    eq_before += __popc(qm);
+  constexpr int kOutBatch = 4;
+  for (int jb0 = w0; jb0 < w1; jb0 += 32 * kOutBatch) {
+    uint32_t v[kOutBatch];
+#pragma unroll
+    for (int u = 0; u < kOutBatch; ++u) {
+      const int j = jb0 + u * 32 + lane;
+      v[u] = j < w1 ? key[j] : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kOutBatch; ++u) {
+      const int j = jb0 + u * 32 + lane;
+      const bool g = j < w1 && v[u] > T, q = j < w1 && v[u] == T;
+      const uint32_t gm = __ballot_sync(0xffffffffu, g), qm = __ballot_sync(0xffffffffu, q);
+      const int gb = gt_before + __popc(gm & lt), qb = eq_before + __popc(qm & lt);
+      const int c = j0 + j;
+      if (g) ob[gb + min(qb, kk)] = direct ? c : __ldg(ib + c);
+      else if (q && qb < kk) ob[gb + qb] = direct ? c : __ldg(ib + c);
+      gt_before += __popc(gm);
+      eq_before += __popc(qm);
+    }
   }
   if (rank == 0 && tid == 0 && topk_count) topk_count[b] = kb;
 }
@@ -562,12 +643,19 @@ int launch_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, 
     const dim3 grid(chunks, nb);
     const size_t o = static_cast<size_t>(b0) * Nw;
     int32_t* cnt = counts + static_cast<size_t>(b0) * chunks * (kSelMaxLayers + 1);
-    launch_dependent(select_count_kernel, grid, dim3(kCompactThreads), 0, s, mask + o, L, lstride, Nw, cnt);
-    launch_dependent(select_fetch_kernel, grid, dim3(kCompactThreads), 0, s, mask + o, L, lstride, Nw, cap,
-                     static_cast<const int32_t*>(cnt), U ? U + o : nullptr, nw ? nw + o : nullptr,
-                     idx_new + static_cast<size_t>(b0) * cap, cnt_new + b0, static_cast<size_t>(B),
-                     idx_U + static_cast<size_t>(b0) * cap, cnt_U + b0, status, logit, B, b0, N,
-                     key_U ? key_U + static_cast<size_t>(b0) * cap : nullptr);
+    auto go = [&](auto ml) {
+      constexpr int kML = decltype(ml)::value;
+      launch_dependent(select_count_kernel<kML>, grid, dim3(kCompactThreads), 0, s, mask + o, L, lstride, Nw, cnt);
+      launch_dependent(select_fetch_kernel<kML>, grid, dim3(kCompactThreads), 0, s, mask + o, L, lstride, Nw, cap,
+                       static_cast<const int32_t*>(cnt), U ? U + o : nullptr, nw ? nw + o : nullptr,
+                       idx_new + static_cast<size_t>(b0) * cap, cnt_new + b0, static_cast<size_t>(B),
+                       idx_U + static_cast<size_t>(b0) * cap, cnt_U + b0, status, logit, B, b0, N,
+                       key_U ? key_U + static_cast<size_t>(b0) * cap : nullptr);
+    };
+    if (L <= 3)
+      go(std::integral_constant<int, 3>{});
+    else
+      go(std::integral_constant<int, kSelMaxLayers>{});
     launches += 2;
   }
   return check_launch("select_fetch", launches);

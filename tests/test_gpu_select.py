@@ -188,12 +188,13 @@ def test_select_fetch_more_sequences_than_one_launch():
     assert (out["cnt_U"] == marks.any(axis=0).sum(axis=1)).all()
 
 
-@pytest.mark.parametrize("B,N,k", [(5, 40000, 512), (3, 262144, 2048), (2, 3000, 5000)])
-def test_topk_keyed_with_selection_keys_equals_topk(B, N, k):
+@pytest.mark.parametrize("B,N,k,L", [(5, 40000, 512, 3), (3, 262144, 2048, 3), (2, 3000, 5000, 3),
+                                     (4, 3001, 100, 5), (3, 7777, 64, 1)])
+def test_topk_keyed_with_selection_keys_equals_topk(B, N, k, L):
     """The union's keys written by lsa_select_fetch and lsa_topk_keyed on them give
-    exactly lsa_topk's result (keys over the logits of every layer) and the oracle's."""
+    exactly lsa_topk's result (keys over the logits of every layer) and the oracle's;
+    N not a multiple of 4 reads the logits one by one, L > 3 takes the wider kernel."""
     g = np.random.default_rng(N + k)
-    L = 3
     marks = g.random((L, B, N)) < 0.25
     logits = np.round(g.standard_normal((L, B, N)) * 4, 1).astype(np.float32)   # ties
     Nw = (N + 31) // 32
