@@ -184,7 +184,8 @@ int lsa_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, int32
  *   the keys lsa_topk ranks by, for lsa_topk_keyed.
  *   1 <= L <= 8, else LSA_ERR_UNSUPPORTED.  Device
  *   pointers 16-byte aligned (counts 4-byte).  Two launches (per-chunk counts, then the
- *   lists) per block of 65535 sequences.
+ *   lists), and a third for key_U (the keys, from dense reads of the logits), per block
+ *   of 65535 sequences.
  * workspace: lsa_select_fetch_workspace_bytes(B, N) bytes, 256-byte aligned.
  * ---------------------------------------------------------------------------------- */
 size_t lsa_select_fetch_workspace_bytes(int B, int N);

@@ -82,6 +82,15 @@ __device__ __forceinline__ float load_elem(const uint8_t* p, size_t i) { return 
 
 __device__ __forceinline__ float sigmoid_f(float z) { return 1.0f / (1.0f + __expf(-z)); }
 
+// Order-preserving integer image of a float: x < y  <=>  order_key(x) < order_key(y)
+// (the two zeros map to one key; non-negative x map to keys >= 2^31, so 0 is below
+// every non-negative logit's key).
+__device__ __forceinline__ uint32_t order_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // ------------------------------------------------------------------ internal launches
 // Projection: fills q_ws ([L][B][H][dI], wdt) and w_ws ([L][B][H] fp32) for layers
 // l0 .. l0+nL-1.  Scratch regions come from the caller's workspace.
@@ -161,7 +170,7 @@ int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, in
 size_t select_fetch_workspace_bytes(int B, int N);
 int launch_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* nw, int cap,
                         int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
-                        int32_t* counts, const float* logit, uint32_t* key_U, cudaStream_t s);
+                        int32_t* ws, const float* logit, uint32_t* key_U, cudaStream_t s);
 // The top-k with given per-candidate order keys (keys[b][j] for candidate idx[b][j]).
 int launch_topk_keyed(int B, int k, const int32_t* idx, int cap, const int32_t* count, const uint32_t* keys,
                       int32_t* topk, int32_t* topk_count, cudaStream_t s);

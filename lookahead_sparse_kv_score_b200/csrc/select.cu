@@ -126,12 +126,6 @@ compact_kernel(const uint32_t* __restrict__ bits, int Nw, int cap, int32_t* __re
   }
 }
 
-// Order-preserving integer image of a float key: larger float -> larger key.
-__device__ __forceinline__ uint32_t order_key(float x) {
-  const uint32_t u = __float_as_uint(x);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
 // ------------------------------------------------------------------ union + fetch lists
 // The whole selection of one trigger in two launches over the L layer masks: per word,
 // new_l = mask_l & ~(mask_0 | .. | mask_{l-1}) and U = mask_0 | .. | mask_{L-1}, and the
@@ -155,15 +149,17 @@ select_count_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
   const uint32_t* mb = mask + static_cast<size_t>(b) * Nw;
   const int wi = chunk * kCompactWords + tid;
   int pc[kML + 1];
+  uint32_t mw[kML];
+#pragma unroll
+  for (int l = 0; l < kML; ++l) {            // every layer's word loaded before any is used
+    mw[l] = 0u;
+    if (l < L && wi < Nw) mw[l] = __ldg(mb + l * lstride + wi);
+  }
   uint32_t acc = 0;
 #pragma unroll
   for (int l = 0; l < kML; ++l) {
-    pc[l] = 0;
-    if (l < L && wi < Nw) {
-      const uint32_t m = __ldg(mb + l * lstride + wi);
-      pc[l] = __popc(m & ~acc);
-      acc |= m;
-    }
+    pc[l] = __popc(mw[l] & ~acc);
+    acc |= mw[l];
   }
   pc[kML] = __popc(acc);
 #pragma unroll
@@ -187,7 +183,7 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
                     const int32_t* __restrict__ counts, uint32_t* __restrict__ U, uint32_t* __restrict__ nw,
                     int32_t* __restrict__ idx_new, int32_t* __restrict__ cnt_new, size_t cstride,
                     int32_t* __restrict__ idx_U, int32_t* __restrict__ cnt_U, int32_t* status,
-                    const float* __restrict__ logit, int Bfull, int b_off, int N, uint32_t* __restrict__ key_U) {
+                    int32_t* __restrict__ ubase) {
   pdl_wait();
   pdl_trigger();
   __shared__ int base_s[kML + 1];
@@ -212,16 +208,18 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
   const int wi = w0 + tid;
   uint32_t word[kML + 1];
   {
+    uint32_t mw[kML];
+#pragma unroll
+    for (int l = 0; l < kML; ++l) {          // every layer's word loaded before any is used
+      mw[l] = 0u;
+      if (l < L && wi < Nw) mw[l] = __ldg(mb + l * lstride + wi);
+    }
     uint32_t acc = 0;
 #pragma unroll
     for (int l = 0; l < kML; ++l) {
-      word[l] = 0u;
-      if (l < L && wi < Nw) {
-        const uint32_t m = __ldg(mb + l * lstride + wi);
-        word[l] = m & ~acc;
-        acc |= m;
-        if (nw) nw[l * lstride + static_cast<size_t>(b) * Nw + wi] = word[l];
-      }
+      word[l] = mw[l] & ~acc;
+      acc |= mw[l];
+      if (nw && l < L && wi < Nw) nw[l * lstride + static_cast<size_t>(b) * Nw + wi] = word[l];
     }
     word[kML] = acc;
     if (U && wi < Nw) U[static_cast<size_t>(b) * Nw + wi] = acc;
@@ -258,7 +256,6 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
 #pragma unroll
     for (int q = 0; q <= kML; ++q)
       if (q == jj) { bits = word[q]; inc = incl[q]; }
-    const uint32_t lbits = bits;
     // the warp's run of this list: staged in its own shared buffer in list order, then
     // copied out with full 128-byte stores
     int32_t* stage = wstage[warp];
@@ -274,50 +271,8 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
     int32_t* out = (j == L ? idx_U + static_cast<size_t>(b) * cap : idx_new + j * cstride * cap + static_cast<size_t>(b) * cap);
     for (int i = lane; i < wtot; i += 32)
       if (wbase + i < cap) out[wbase + i] = stage[i];
-    if (j == L && key_U) {
-      // The union's candidates also get their top-k key, the order image of the largest
-      // logit over the layers.  The warp's 1024 entries are read densely (lane t: the
-      // float4 of entries 128 k + 4 t), skipping groups with no candidate, and each
-      // candidate's list position comes from its word's offset in the warp's run.
-      uint32_t* kout = key_U + static_cast<size_t>(b) * cap;
-      const float* lb = logit + static_cast<size_t>(b_off + b) * N;
-      const size_t lstep = static_cast<size_t>(Bfull) * N;
-      const bool vec = (N % 4 == 0) && (reinterpret_cast<uintptr_t>(logit) % 16 == 0);
-      const int ex = inc - __popc(lbits);             // exclusive offset of this lane's word
-      const int e_warp = (w0 + warp * 32) * 32;       // the warp's first entry
-      const int sh = (lane & 7) * 4;                  // bit of entry 128 k + 4 lane in its word
-#pragma unroll 2
-      for (int k = 0; k < 8; ++k) {
-        const int src = 4 * k + (lane >> 3);          // the word holding those entries
-        const uint32_t uw = __shfl_sync(0xffffffffu, lbits, src);
-        const int off = __shfl_sync(0xffffffffu, ex, src);
-        const uint32_t nib = (uw >> sh) & 0xFu;
-        const int e0 = e_warp + 128 * k + 4 * lane;
-        float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        if (nib) {
-#pragma unroll
-          for (int l = 0; l < kML; ++l) {
-            if (l >= L) break;
-            const float* src_l = lb + l * lstep + e0;
-            if (vec && e0 + 3 < N) {
-              const float4 v = __ldg(reinterpret_cast<const float4*>(src_l));
-              m[0] = fmaxf(m[0], v.x); m[1] = fmaxf(m[1], v.y); m[2] = fmaxf(m[2], v.z); m[3] = fmaxf(m[3], v.w);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                if (((nib >> i) & 1u) && e0 + i < N) m[i] = fmaxf(m[i], __ldg(src_l + i));
-            }
-          }
-        }
-        int pos = wbase + off + __popc(uw & ((1u << sh) - 1u));
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if ((nib >> i) & 1u) {
-            if (pos < cap) kout[pos] = order_key(m[i]);
-            ++pos;
-          }
-      }
-    }
+    if (j == L && ubase && lane == 0) ubase[static_cast<size_t>(b) * (gridDim.x * (kCompactThreads / 32)) +
+                                          chunk * (kCompactThreads / 32) + warp] = wbase;
     __syncwarp();
     if (last && tid == 0) {
       int32_t* cnt = j == L ? cnt_U + b : cnt_new + j * cstride + b;
@@ -325,6 +280,98 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
       if (base + total > cap) raise_status(status, LSA_ERR_CAPACITY);
     }
   }
+}
+
+// The union's top-k keys: key_U[b][j] = order_key(max over layers of logit[l][b][e]) for
+// the j-th union entry e.  One warp per 32 union words (1024 entries), independent of
+// the others: its run of the union list starts at ubase[b][warp] (from the fetch
+// kernel), each word's offset is a warp prefix sum of the popcounts, and the logits are
+// read densely (lane t: the four entries 128 k + 4 t, k = 0..7; groups without a
+// candidate are skipped), every load of the warp issued before the first is used; the
+// keys are staged in shared memory in list order and written out with full stores.
+template <int kML>
+__global__ void __launch_bounds__(256)
+select_keys_kernel(const uint32_t* __restrict__ U, int Nw, int L, int N, int cap, const int32_t* __restrict__ ubase,
+                   int wpb, const float* __restrict__ logit, int Bfull, int b_off, uint32_t* __restrict__ key_U) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ uint32_t kstage[8][32 * 32];          // a warp's keys in list order, then copied out
+  const int b = blockIdx.y, lane = threadIdx.x & 31;
+  const int wg = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);   // warp of words [32 wg, 32 wg + 32)
+  if (wg * 32 >= Nw) return;
+  uint32_t* stage = kstage[threadIdx.x >> 5];
+  const int wi = wg * 32 + lane;
+  const uint32_t uw = wi < Nw ? __ldg(U + static_cast<size_t>(b) * Nw + wi) : 0u;
+  const int base = __ldg(ubase + static_cast<size_t>(b) * wpb + wg);
+  int inc = __popc(uw);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  const int ex = inc - __popc(uw);
+  const float* lb = logit + static_cast<size_t>(b_off + b) * N;
+  const size_t lstep = static_cast<size_t>(Bfull) * N;
+  uint32_t* kout = key_U + static_cast<size_t>(b) * cap;
+  const bool vec = (N % 4 == 0) && (reinterpret_cast<uintptr_t>(logit) % 16 == 0);
+  const int sh = (lane & 7) * 4;                    // bit of entry 128 k + 4 lane in its word
+  constexpr int kGroups = 8;
+  constexpr int kHalf = kML <= 3 ? 4 : 1;          // groups whose loads are in flight together
+#pragma unroll
+  for (int k0 = 0; k0 < kGroups; k0 += kHalf) {
+    uint32_t wd[kHalf], nib[kHalf];
+    int off[kHalf];
+    float m[kHalf][4];
+#pragma unroll
+    for (int u = 0; u < kHalf; ++u) {
+      const int src = 4 * (k0 + u) + (lane >> 3);   // the word holding those entries
+      wd[u] = __shfl_sync(0xffffffffu, uw, src);
+      off[u] = __shfl_sync(0xffffffffu, ex, src);
+      nib[u] = (wd[u] >> sh) & 0xFu;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m[u][i] = -INFINITY;
+    }
+    if (vec) {
+      // every load first (predicated, no branch between a load and its use), then the maxima
+      float4 v[kHalf][kML];
+#pragma unroll
+      for (int l = 0; l < kML; ++l)
+#pragma unroll
+        for (int u = 0; u < kHalf; ++u) {
+          const int e0 = wg * 1024 + 128 * (k0 + u) + 4 * lane;
+          v[u][l] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+          if (l < L && nib[u] != 0u && e0 < N)
+            v[u][l] = __ldg(reinterpret_cast<const float4*>(lb + l * lstep + e0));
+        }
+#pragma unroll
+      for (int l = 0; l < kML; ++l)
+#pragma unroll
+        for (int u = 0; u < kHalf; ++u) {
+          m[u][0] = fmaxf(m[u][0], v[u][l].x); m[u][1] = fmaxf(m[u][1], v[u][l].y);
+          m[u][2] = fmaxf(m[u][2], v[u][l].z); m[u][3] = fmaxf(m[u][3], v[u][l].w);
+        }
+    } else {
+      for (int l = 0; l < L; ++l)
+#pragma unroll
+        for (int u = 0; u < kHalf; ++u) {
+          const int e0 = wg * 1024 + 128 * (k0 + u) + 4 * lane;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (((nib[u] >> i) & 1u) && e0 + i < N) m[u][i] = fmaxf(m[u][i], __ldg(lb + l * lstep + e0 + i));
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kHalf; ++u) {
+      int pos = off[u] + __popc(wd[u] & ((1u << sh) - 1u));   // offset in the warp's run
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if ((nib[u] >> i) & 1u) stage[pos++] = order_key(m[u][i]);
+    }
+  }
+  __syncwarp();
+  const int wtot = __shfl_sync(0xffffffffu, inc, 31);
+  for (int i = lane; i < wtot; i += 32)
+    if (base + i < cap) kout[base + i] = stage[i];
 }
 
 // ------------------------------------------------------------------ top-k
@@ -623,19 +670,39 @@ int launch_compact(int B, int N, const uint32_t* bits, int cap, int32_t* idx, in
   return check_launch("compact", launches);
 }
 
-size_t select_fetch_workspace_bytes(int B, int N) {
+// Workspace: per-chunk counts [B][chunks][kSelMaxLayers + 1], the union list's base of
+// every warp of words [B][chunks * 8], and room for the union words [B][Nw] when the
+// caller does not ask for them (the key kernel reads them).
+struct SelWs {
+  size_t counts, ubase, U, total;
+};
+static SelWs sel_ws(int B, int N) {
   const int Nw = (N + 31) / 32;
   const size_t chunks = std::max(1, (Nw + kCompactWords - 1) / kCompactWords);
-  return static_cast<size_t>(B) * chunks * (kSelMaxLayers + 1) * 4;
+  SelWs w{};
+  w.counts = 0;
+  w.ubase = align_up(static_cast<size_t>(B) * chunks * (kSelMaxLayers + 1) * 4, 256);
+  w.U = align_up(w.ubase + static_cast<size_t>(B) * chunks * (kCompactThreads / 32) * 4, 256);
+  w.total = align_up(w.U + static_cast<size_t>(B) * Nw * 4, 256);
+  return w;
 }
+
+size_t select_fetch_workspace_bytes(int B, int N) { return sel_ws(B, N).total; }
 
 int launch_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, uint32_t* nw, int cap,
                         int32_t* idx_new, int32_t* cnt_new, int32_t* idx_U, int32_t* cnt_U, int32_t* status,
-                        int32_t* counts, const float* logit, uint32_t* key_U, cudaStream_t s) {
+                        int32_t* ws, const float* logit, uint32_t* key_U, cudaStream_t s) {
   if (B == 0) return LSA_OK;
   const int Nw = (N + 31) / 32;
   const size_t lstride = static_cast<size_t>(B) * Nw;
   const int chunks = std::max(1, (Nw + kCompactWords - 1) / kCompactWords);
+  const int wpb = chunks * (kCompactThreads / 32);             // warps of words per sequence
+  const SelWs lay = sel_ws(B, N);
+  uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
+  int32_t* counts = reinterpret_cast<int32_t*>(wsb + lay.counts);
+  int32_t* ubase = key_U ? reinterpret_cast<int32_t*>(wsb + lay.ubase) : nullptr;
+  // the key kernel reads the union words: the caller's, else a workspace copy
+  uint32_t* Uw = U ? U : (key_U ? reinterpret_cast<uint32_t*>(wsb + lay.U) : nullptr);
   constexpr int kSeqPerLaunch = 65535;   // the sequence index is gridDim.y
   int launches = 0;
   for (int b0 = 0; b0 < B; b0 += kSeqPerLaunch) {
@@ -647,16 +714,23 @@ int launch_select_fetch(int B, int L, int N, const uint32_t* mask, uint32_t* U, 
       constexpr int kML = decltype(ml)::value;
       launch_dependent(select_count_kernel<kML>, grid, dim3(kCompactThreads), 0, s, mask + o, L, lstride, Nw, cnt);
       launch_dependent(select_fetch_kernel<kML>, grid, dim3(kCompactThreads), 0, s, mask + o, L, lstride, Nw, cap,
-                       static_cast<const int32_t*>(cnt), U ? U + o : nullptr, nw ? nw + o : nullptr,
+                       static_cast<const int32_t*>(cnt), Uw ? Uw + o : nullptr, nw ? nw + o : nullptr,
                        idx_new + static_cast<size_t>(b0) * cap, cnt_new + b0, static_cast<size_t>(B),
-                       idx_U + static_cast<size_t>(b0) * cap, cnt_U + b0, status, logit, B, b0, N,
-                       key_U ? key_U + static_cast<size_t>(b0) * cap : nullptr);
+                       idx_U + static_cast<size_t>(b0) * cap, cnt_U + b0, status,
+                       ubase ? ubase + static_cast<size_t>(b0) * wpb : nullptr);
+      launches += 2;
+      if (key_U) {
+        const dim3 kgrid((wpb + 7) / 8, nb);
+        launch_dependent(select_keys_kernel<kML>, kgrid, dim3(256), 0, s, static_cast<const uint32_t*>(Uw + o), Nw,
+                         L, N, cap, static_cast<const int32_t*>(ubase + static_cast<size_t>(b0) * wpb), wpb, logit,
+                         B, b0, key_U + static_cast<size_t>(b0) * cap);
+        ++launches;
+      }
     };
     if (L <= 3)
       go(std::integral_constant<int, 3>{});
     else
       go(std::integral_constant<int, kSelMaxLayers>{});
-    launches += 2;
   }
   return check_launch("select_fetch", launches);
 }
@@ -667,10 +741,41 @@ int launch_topk_cluster(int B, int L, int N, int k, const int32_t* idx, int cap,
                         const float* logit, const uint32_t* dkeys, const int32_t* kdev, const int32_t* kept,
                         int32_t* status, int32_t* topk, int32_t* topk_count, uint32_t* keys_ws, cudaStream_t s) {
   const int smem = kTopkStateBytes + kTopkSmemKeys * 4;
-  cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
-  int sms = 148, dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // per device, once: the kernel's attributes, the SM count and the largest cluster size
+  // the occupancy calculator accepts (kept so that a launch makes no query calls)
+  constexpr int kMaxDevices = 64;
+  static int dev_sms[kMaxDevices] = {}, dev_max_cs[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+  if (dev_sms[dev] == 0) {
+    cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+    int n = 148;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    int best = 1;
+    for (int c = 8; c > 1; c >>= 1) {
+      cudaLaunchConfig_t q = {};
+      cudaLaunchAttribute qa[1];
+      qa[0].id = cudaLaunchAttributeClusterDimension;
+      qa[0].val.clusterDim.x = c;
+      qa[0].val.clusterDim.y = 1;
+      qa[0].val.clusterDim.z = 1;
+      q.gridDim = dim3(c);
+      q.blockDim = dim3(kTopkThreads);
+      q.dynamicSmemBytes = smem;
+      q.attrs = qa;
+      q.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, topk_cluster_kernel, &q) == cudaSuccess && clusters > 0) {
+        best = c;
+        break;
+      }
+      cudaGetLastError();
+    }
+    dev_max_cs[dev] = best;
+    dev_sms[dev] = n;
+  }
+  const int sms = dev_sms[dev];
   // CTAs per sequence: as many as keep B x cs within one wave, at most 8 (portable); when
   // the keys are computed from the logits, at least enough that a full list (cap
   // candidates) keeps every CTA's slice in shared memory (the busiest sequence sets the
@@ -691,16 +796,11 @@ int launch_topk_cluster(int B, int L, int N, int k, const int32_t* idx, int cap,
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  for (;; cs >>= 1) {
-    attr[0].val.clusterDim.x = cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(B * cs);
-    if (cs == 1) break;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, topk_cluster_kernel, &cfg) == cudaSuccess && clusters > 0) break;
-    cudaGetLastError();
-  }
+  cs = std::min(cs, dev_max_cs[dev]);
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(B * cs);
   cudaLaunchKernelEx(&cfg, topk_cluster_kernel, B, L, N, k, idx, cap, count, logit, dkeys, kdev, kept, status,
                      keys_ws, topk, topk_count);
   return check_launch("topk");

@@ -42,11 +42,6 @@ static_assert(kFineBins % kRowThreads == 0, "bins per thread");
 static_assert(kSubBins % kRowThreads == 0, "sub-bins per thread");
 static_assert(kSubBins * 12 <= kHistInts * 4, "sub-bins reuse the histogram");
 
-__device__ __forceinline__ uint32_t order_key(float x) {
-  uint32_t u = __float_as_uint(x);
-  if (u == 0x80000000u) u = 0u;       // -0 and +0 are the same logit
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
