@@ -548,8 +548,12 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
 #pragma unroll
     for (int q = 0; q < kBinsPerThread; ++q) {
       const int d = kDigitBins - 1 - (tid * kBinsPerThread + q);
+      int v[8];                 // every rank's count loaded before any is added
+#pragma unroll
+      for (int r = 0; r < 8; ++r) v[r] = r < cs ? cl.map_shared_rank(&sh.hist[pass & 1][0], r)[d] : 0;
       int t = 0;
-      for (int r = 0; r < cs; ++r) t += cl.map_shared_rank(&sh.hist[pass & 1][0], r)[d];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) t += v[r];
       tot[q] = t;
       mine += t;
     }
@@ -605,15 +609,19 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
       if (lane == 0) { sh.cnt[0] = g; sh.cnt[1] = q; }
     }
     cl.sync();
-    if (tid == 0) {
+    if (warp == 0) {            // lane r reads rank r's counts; the lower ranks' are summed
       int g = 0, q = 0;
-      for (int r = 0; r < rank; ++r) {
-        const int* rc = cl.map_shared_rank(&sh.cnt[0], r);
-        g += rc[0];
-        q += rc[1];
+      if (lane < rank) {
+        const int* rc = cl.map_shared_rank(&sh.cnt[0], lane);
+        g = rc[0];
+        q = rc[1];
       }
-      sh.gbase = g;
-      sh.ebase = q;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        g += __shfl_xor_sync(0xffffffffu, g, o);
+        q += __shfl_xor_sync(0xffffffffu, q, o);
+      }
+      if (lane == 0) { sh.gbase = g; sh.ebase = q; }
     }
     cl.sync();   // no CTA leaves while another may still read its shared memory
   }
