@@ -65,6 +65,13 @@ constexpr float kLog2e = 1.4426950408889634f;
 // row's window path (Z, the mass above the run, the run's entries) uses this one form.
 __device__ __forceinline__ float win_term(float x, float nm) { return ex2_approx(fmaf(x, kLog2e, nm)); }
 
+// max(a, b, c) in one instruction; like fmaxf, a NaN operand is ignored.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // One count into the shared-memory histogram at a 32-bit shared address.
 __device__ __forceinline__ void red_shared_inc(uint32_t addr) {
   asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
@@ -454,10 +461,14 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
       constexpr bool kFull = decltype(full)::value;
       const float xs[4] = {v.x, v.y, v.z, v.w};
       float ez = 0.f;              // at most four terms <= e^4
+      if constexpr (kFull) {       // two three-input maxima per four logits
+        mloc = fmax3(mloc, xs[0], xs[1]);
+        mloc = fmax3(mloc, xs[2], xs[3]);
+      }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         if (kFull || s + j < N) {
-          mloc = fmaxf(mloc, xs[j]);
+          if constexpr (!kFull) mloc = fmaxf(mloc, xs[j]);
           ez += ex2_approx(fmaf(xs[j], kLog2e, nm));
           const float u = __saturatef(fmaf(xs[j], c1, c0));
           red_shared_inc(__float_as_uint(__fmaf_rd(u, static_cast<float>(kFineBins), 8388608.f)) * 4u + hbase);
@@ -562,38 +573,20 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
       const float xs[4] = {v.x, v.y, v.z, v.w};   // NaN past N: neither above nor in the run
       float ea = 0.f;
       uint32_t wd[4];
-      bool run[4];
-      bool any_run = false;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const bool up = (kFull || s + j < N) && xs[j] > xu;
         wd[j] = __ballot_sync(0xffffffffu, up);
-        run[j] = !up && xs[j] > xl;
-        any_run |= run[j];
         const float e = ex2_approx(fmaf(xs[j], kLog2e, nm));
         ea += up ? e : 0.f;
+        // the run's entries (a fraction of a percent): each takes its own list slot
+        if (!up && xs[j] > xl) {
+          const int at = atomicAdd(&sh.count, 1);
+          if (at < kListCap)
+            list[at] = (static_cast<unsigned long long>(~order_key(xs[j])) << 32) | static_cast<uint32_t>(s + j);
+        }
       }
       if (lane == 0 && s < N) *reinterpret_cast<uint4*>(out + 4 * (s >> 7)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-      if (__any_sync(0xffffffffu, any_run)) {
-        uint32_t rb[4];
-        int tot = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          rb[j] = __ballot_sync(0xffffffffu, run[j]);
-          tot += __popc(rb[j]);
-        }
-        int pos = 0;
-        if (lane == 0) pos = atomicAdd(&sh.count, tot);
-        pos = __shfl_sync(0xffffffffu, pos, 0);
-        const uint32_t lt = (1u << lane) - 1u;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int at = pos + __popc(rb[j] & lt);
-          if (run[j] && at < kListCap)
-            list[at] = (static_cast<unsigned long long>(~order_key(xs[j])) << 32) | static_cast<uint32_t>(s + j);
-          pos += __popc(rb[j]);
-        }
-      }
       return ea;
     };
     int g0 = tid;
