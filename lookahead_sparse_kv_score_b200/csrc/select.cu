@@ -382,8 +382,10 @@ constexpr int kTopkSmemKeys = 32768;   // keys of one CTA's candidate slice held
 constexpr int kSubHists = 8;           // digit histograms, one per four warps (fewer same-bin collisions)
 constexpr int kDigitBins = 2048;       // radix digits of 11, 11 and 10 bits
 constexpr int kKeyBatch = 8;           // keys a thread loads before using any
+constexpr int kKeptCap = 512;          // positions of kept keys a warp records (in the digit histograms' space)
 constexpr int kBinsPerThread = kDigitBins / kTopkThreads;
 static_assert(kBinsPerThread == 2, "two digit bins per thread");
+static_assert(kTopkWarps * kKeptCap <= kSubHists * kDigitBins, "kept positions fit in the digit histograms");
 
 struct TopkShared {
   int sub[kSubHists][kDigitBins];   // digit histograms, one per four warps
@@ -576,6 +578,12 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
   // this warp's contiguous part of the slice
   const int per = (mloc + kTopkWarps - 1) / kTopkWarps;
   const int w0 = min(mloc, warp * per), w1 = min(mloc, w0 + per);
+  // The warp counts its keys above and equal to T and records where they are (ascending,
+  // in the digit histograms' space, free after the last pass), so that the output needs
+  // no second pass over the part unless more than kKeptCap of them fell in it.
+  const uint32_t lt = (1u << lane) - 1u;
+  int* wpos = &sh.sub[0][0] + warp * kKeptCap;
+  int nk = 0;
   {
     int gt = 0, eq = 0;
     for (int jb = w0; jb < w1; jb += 32 * kKeyBatch) {
@@ -588,14 +596,15 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
 #pragma unroll
       for (int u = 0; u < kKeyBatch; ++u) {
         const int j = jb + u * 32 + lane;
-        gt += j < w1 && v[u] > T;
-        eq += j < w1 && v[u] == T;
+        const bool g = j < w1 && v[u] > T, q = j < w1 && v[u] == T;
+        const uint32_t gm = __ballot_sync(0xffffffffu, g), qm = __ballot_sync(0xffffffffu, q);
+        const uint32_t km = gm | qm;
+        const int at = nk + __popc(km & lt);
+        if ((g || q) && at < kKeptCap) wpos[at] = j;
+        nk += __popc(km);
+        gt += __popc(gm);
+        eq += __popc(qm);
       }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      gt += __shfl_xor_sync(0xffffffffu, gt, o);
-      eq += __shfl_xor_sync(0xffffffffu, eq, o);
     }
     if (lane == 0) { sh.wgt[warp] = gt; sh.weq[warp] = eq; }
     __syncthreads();
@@ -627,7 +636,23 @@ topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx,
   }
   int gt_before = sh.gbase, eq_before = sh.ebase;
   for (int w = 0; w < warp; ++w) { gt_before += sh.wgt[w]; eq_before += sh.weq[w]; }
-  const uint32_t lt = (1u << lane) - 1u;
+  if (nk <= kKeptCap) {
+    for (int i0 = 0; i0 < nk; i0 += 32) {
+      const int i = i0 + lane;
+      const int j = i < nk ? wpos[i] : 0;
+      const uint32_t u = i < nk ? key[j] : 0u;
+      const bool g = i < nk && u > T, q = i < nk && u == T;
+      const uint32_t gm = __ballot_sync(0xffffffffu, g), qm = __ballot_sync(0xffffffffu, q);
+      const int gb = gt_before + __popc(gm & lt), qb = eq_before + __popc(qm & lt);
+      const int c = j0 + j;
+      if (g) ob[gb + min(qb, kk)] = direct ? c : __ldg(ib + c);
+      else if (q && qb < kk) ob[gb + qb] = direct ? c : __ldg(ib + c);
+      gt_before += __popc(gm);
+      eq_before += __popc(qm);
+    }
+    if (rank == 0 && tid == 0 && topk_count) topk_count[b] = kb;
+    return;
+  }
   constexpr int kOutBatch = 4;
   for (int jb0 = w0; jb0 < w1; jb0 += 32 * kOutBatch) {
     uint32_t v[kOutBatch];

@@ -299,6 +299,21 @@ def test_topk_negative_keys_and_all_equal():
     assert np.array_equal(topk[1, :100], np.arange(0, 300, 3))
 
 
+def test_topk_all_equal_long_list_and_mixed_ties():
+    """600,000 equal keys (every warp's part holds more keys at the threshold than it
+    records, so the output rescans the part) and a list of 20 distinct large keys among
+    ties: the kept entries are the large keys and then the lowest-index ties."""
+    L, B, N, k = 1, 2, 600000, 2048
+    logits = np.full((L, B, N), 1.25, dtype=np.float32)
+    big = np.array([7, 1000, 99999, 123456, 599999] + list(range(300000, 300015)))
+    logits[0, 1, big] = 5.0 + np.arange(big.size, dtype=np.float32)
+    idx = [np.arange(N), np.arange(N)]
+    topk, tc = run_topk(idx, logits, k, N)
+    assert tc[0] == k and np.array_equal(topk[0, :k], np.arange(k))
+    want = np.sort(np.concatenate([big, np.setdiff1d(np.arange(N), big)[: k - big.size]]))
+    assert tc[1] == k and np.array_equal(topk[1, :k], want)
+
+
 def test_gather_bytes_exact_and_range_status():
     g = np.random.default_rng(2)
     B, N, R = 3, 4000, 1152
