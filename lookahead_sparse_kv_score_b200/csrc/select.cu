@@ -192,6 +192,16 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
   const int b = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t* mb = mask + static_cast<size_t>(b) * Nw;
   const int w0 = chunk * kCompactWords;
+  // own word: every layer's word loaded first, so that these loads and the bases' below
+  // are in flight together
+  const int wi = w0 + tid;
+  uint32_t word[kML + 1];
+  uint32_t mw[kML];
+#pragma unroll
+  for (int l = 0; l < kML; ++l) {
+    mw[l] = 0u;
+    if (l < L && wi < Nw) mw[l] = __ldg(mb + l * lstride + wi);
+  }
   // bases: the lists' set bits in the earlier chunks of this sequence (list q, q = kML
   // the union, summed by warp q mod 8, its lanes over the chunks, so no load waits on
   // another)
@@ -204,16 +214,7 @@ select_fetch_kernel(const uint32_t* __restrict__ mask, int L, size_t lstride, in
     for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
     if (lane == 0) base_s[q] = t;
   }
-  // own word
-  const int wi = w0 + tid;
-  uint32_t word[kML + 1];
   {
-    uint32_t mw[kML];
-#pragma unroll
-    for (int l = 0; l < kML; ++l) {          // every layer's word loaded before any is used
-      mw[l] = 0u;
-      if (l < L && wi < Nw) mw[l] = __ldg(mb + l * lstride + wi);
-    }
     uint32_t acc = 0;
 #pragma unroll
     for (int l = 0; l < kML; ++l) {
