@@ -573,18 +573,23 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
       const float xs[4] = {v.x, v.y, v.z, v.w};   // NaN past N: neither above nor in the run
       float ea = 0.f;
       uint32_t wd[4];
+      uint32_t runm = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const bool up = (kFull || s + j < N) && xs[j] > xu;
         wd[j] = __ballot_sync(0xffffffffu, up);
         const float e = ex2_approx(fmaf(xs[j], kLog2e, nm));
-        ea += up ? e : 0.f;
-        // the run's entries (a fraction of a percent): each takes its own list slot
-        if (!up && xs[j] > xl) {
-          const int at = atomicAdd(&sh.count, 1);
-          if (at < kListCap)
-            list[at] = (static_cast<unsigned long long>(~order_key(xs[j])) << 32) | static_cast<uint32_t>(s + j);
-        }
+        if (up) ea += e;
+        runm |= (!up && xs[j] > xl) ? (1u << j) : 0u;
+      }
+      if (runm) {   // the run's entries (a fraction of a percent): each takes its own list slot
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (runm & (1u << j)) {
+            const int at = atomicAdd(&sh.count, 1);
+            if (at < kListCap)
+              list[at] = (static_cast<unsigned long long>(~order_key(xs[j])) << 32) | static_cast<uint32_t>(s + j);
+          }
       }
       if (lane == 0 && s < N) *reinterpret_cast<uint4*>(out + 4 * (s >> 7)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
       return ea;
