@@ -65,6 +65,28 @@ constexpr float kLog2e = 1.4426950408889634f;
 // row's window path (Z, the mass above the run, the run's entries) uses this one form.
 __device__ __forceinline__ float win_term(float x, float nm) { return ex2_approx(fmaf(x, kLog2e, nm)); }
 
+// Paired fp32 arithmetic (one instruction for two lanes of values, each rounded as the
+// scalar instruction rounds it).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  unsigned long long ra, rb, rc, rd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rc) : "f"(c.x), "f"(c.y));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+  float2 d;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  unsigned long long ra, rb, rd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
+  float2 d;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+  return d;
+}
+
 // max(a, b, c) in one instruction; like fmaxf, a NaN operand is ignored.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
@@ -461,15 +483,23 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
       constexpr bool kFull = decltype(full)::value;
       const float xs[4] = {v.x, v.y, v.z, v.w};
       float ez = 0.f;              // at most four terms <= e^4
-      if constexpr (kFull) {       // two three-input maxima per four logits
+      if constexpr (kFull) {
+        // two three-input maxima, the exponents' arguments and the sum in pairs
         mloc = fmax3(mloc, xs[0], xs[1]);
         mloc = fmax3(mloc, xs[2], xs[3]);
+        const float2 l2 = make_float2(kLog2e, kLog2e), n2 = make_float2(nm, nm);
+        const float2 a01 = ffma2(make_float2(xs[0], xs[1]), l2, n2), a23 = ffma2(make_float2(xs[2], xs[3]), l2, n2);
+        const float2 e = fadd2(make_float2(ex2_approx(a01.x), ex2_approx(a01.y)),
+                               make_float2(ex2_approx(a23.x), ex2_approx(a23.y)));
+        ez = e.x + e.y;
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         if (kFull || s + j < N) {
-          if constexpr (!kFull) mloc = fmaxf(mloc, xs[j]);
-          ez += ex2_approx(fmaf(xs[j], kLog2e, nm));
+          if constexpr (!kFull) {
+            mloc = fmaxf(mloc, xs[j]);
+            ez += ex2_approx(fmaf(xs[j], kLog2e, nm));
+          }
           const float u = __saturatef(fmaf(xs[j], c1, c0));
           red_shared_inc(__float_as_uint(__fmaf_rd(u, static_cast<float>(kFineBins), 8388608.f)) * 4u + hbase);
         }
@@ -574,11 +604,14 @@ __device__ bool window_nucleus(const float* x, int N, bool vec, float top_p, flo
       float ea = 0.f;
       uint32_t wd[4];
       uint32_t runm = 0;
+      const float2 l2 = make_float2(kLog2e, kLog2e), n2 = make_float2(nm, nm);
+      const float2 a01 = ffma2(make_float2(xs[0], xs[1]), l2, n2), a23 = ffma2(make_float2(xs[2], xs[3]), l2, n2);
+      const float arg[4] = {a01.x, a01.y, a23.x, a23.y};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const bool up = (kFull || s + j < N) && xs[j] > xu;
         wd[j] = __ballot_sync(0xffffffffu, up);
-        const float e = ex2_approx(fmaf(xs[j], kLog2e, nm));
+        const float e = ex2_approx(arg[j]);
         if (up) ea += e;
         runm |= (!up && xs[j] > xl) ? (1u << j) : 0u;
       }
