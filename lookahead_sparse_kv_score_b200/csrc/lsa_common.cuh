@@ -232,7 +232,7 @@ struct VoteArgs {
   double* loss;
   uint32_t* selbits;    // workspace [L][P][Nw]
   float* rowparam;      // workspace [L][P][4]
-  double* lossacc;      // workspace [2]
+  double* lossacc;      // workspace: [2] loss sums, then the loss blocks' counter
 };
 int launch_vote(const VoteArgs& a, cudaStream_t s);
 

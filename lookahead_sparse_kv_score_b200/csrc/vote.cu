@@ -830,10 +830,15 @@ __global__ void vote_count_kernel(const uint32_t* __restrict__ selbits, int L, i
     }
   };
   int l = 0;
-  for (; l + 2 <= L; l += 2) {
-    const uint4 b0 = __ldg(src + l * stride), b1 = __ldg(src + (l + 1) * stride);
-    add(b0.x, pl[0]); add(b0.y, pl[1]); add(b0.z, pl[2]); add(b0.w, pl[3]);
-    add(b1.x, pl[0]); add(b1.y, pl[1]); add(b1.z, pl[2]); add(b1.w, pl[3]);
+  constexpr int kLoads = 8;    // layers' words in flight together
+  for (; l + kLoads <= L; l += kLoads) {
+    uint4 bw[kLoads];
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i) bw[i] = __ldg(src + (l + i) * stride);
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i) {
+      add(bw[i].x, pl[0]); add(bw[i].y, pl[1]); add(bw[i].z, pl[2]); add(bw[i].w, pl[3]);
+    }
   }
   for (; l < L; ++l) {
     const uint4 b = __ldg(src + l * stride);
@@ -911,8 +916,9 @@ __device__ __forceinline__ float focal_pow(float q, float gamma) {
   return gamma == 2.f ? q * q : (gamma == 1.f ? q : (gamma == 0.f ? 1.f : powf(q, gamma)));
 }
 
+// acc [2] doubles, then a block counter: the last block to finish writes the means.
 __global__ void vote_loss_kernel(const float* __restrict__ scores, const uint32_t* __restrict__ golden, int P,
-                                 int N, float gamma, double* __restrict__ acc) {
+                                 int N, float gamma, double* __restrict__ acc, double* __restrict__ loss) {
   __shared__ double tmp[2][32];
   const int Nw = (N + 31) / 32;
   const int p = blockIdx.y;
@@ -931,22 +937,35 @@ __global__ void vote_loss_kernel(const float* __restrict__ scores, const uint32_
   const int stride = gridDim.x * blockDim.x;
   if ((N & 7) == 0 && (reinterpret_cast<uintptr_t>(sc) & 15) == 0) {
     const int G = N >> 3;       // groups of eight entries: two float4 and one byte of labels
-    for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < G; g += stride) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(sc) + 2 * g);
-      const float4 c = __ldg(reinterpret_cast<const float4*>(sc) + 2 * g + 1);
-      const uint32_t bits = __ldg(gw + (g >> 2)) >> (8 * (g & 3));
-      gb = 0.f;
-      gf = 0.f;
-      term(a.x, bits & 1u);
-      term(a.y, (bits >> 1) & 1u);
-      term(a.z, (bits >> 2) & 1u);
-      term(a.w, (bits >> 3) & 1u);
-      term(c.x, (bits >> 4) & 1u);
-      term(c.y, (bits >> 5) & 1u);
-      term(c.z, (bits >> 6) & 1u);
-      term(c.w, (bits >> 7) & 1u);
-      bce += static_cast<double>(gb);
-      fl += static_cast<double>(gf);
+    constexpr int kGroups = 2;  // groups whose loads are in flight together
+    for (int g0 = blockIdx.x * blockDim.x + threadIdx.x; g0 < G; g0 += kGroups * stride) {
+      float4 a[kGroups], c[kGroups];
+      uint32_t bits[kGroups];
+#pragma unroll
+      for (int u = 0; u < kGroups; ++u) {
+        const int g = g0 + u * stride;
+        if (g < G) {
+          a[u] = __ldg(reinterpret_cast<const float4*>(sc) + 2 * g);
+          c[u] = __ldg(reinterpret_cast<const float4*>(sc) + 2 * g + 1);
+          bits[u] = __ldg(gw + (g >> 2)) >> (8 * (g & 3));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kGroups; ++u) {
+        if (g0 + u * stride >= G) break;
+        gb = 0.f;
+        gf = 0.f;
+        term(a[u].x, bits[u] & 1u);
+        term(a[u].y, (bits[u] >> 1) & 1u);
+        term(a[u].z, (bits[u] >> 2) & 1u);
+        term(a[u].w, (bits[u] >> 3) & 1u);
+        term(c[u].x, (bits[u] >> 4) & 1u);
+        term(c[u].y, (bits[u] >> 5) & 1u);
+        term(c[u].z, (bits[u] >> 6) & 1u);
+        term(c[u].w, (bits[u] >> 7) & 1u);
+        bce += static_cast<double>(gb);
+        fl += static_cast<double>(gf);
+      }
     }
   } else {
     for (int s = blockIdx.x * blockDim.x + threadIdx.x; s < N; s += stride) {
@@ -970,12 +989,15 @@ __global__ void vote_loss_kernel(const float* __restrict__ scores, const uint32_
     for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) { a += tmp[0][w]; b += tmp[1][w]; }
     atomicAdd(&acc[0], a);
     atomicAdd(&acc[1], b);
+    __threadfence();
+    unsigned int* done = reinterpret_cast<unsigned int*>(acc + 2);
+    if (atomicAdd(done, 1u) == gridDim.x * gridDim.y - 1) {   // every other block's sums are in
+      __threadfence();
+      const double n = static_cast<double>(P) * N;
+      loss[0] = *reinterpret_cast<volatile double*>(&acc[0]) / n;
+      loss[1] = *reinterpret_cast<volatile double*>(&acc[1]) / n;
+    }
   }
-}
-
-__global__ void vote_loss_finalize(const double* __restrict__ acc, double n, double* __restrict__ loss) {
-  loss[0] = acc[0] / n;
-  loss[1] = acc[1] / n;
 }
 
 }  // namespace
@@ -1007,13 +1029,12 @@ int launch_vote(const VoteArgs& a, cudaStream_t st) {
     vote_count_kernel<8><<<cgrid, kCountThreads, 0, st>>>(a.selbits, a.L, a.P, a.N, a.theta, a.golden, a.counts);
   if ((rc = check_launch("vote_labels/count")) != LSA_OK) return rc;
   if (a.scores) {
-    cudaMemsetAsync(a.lossacc, 0, 2 * sizeof(double), st);
+    cudaMemsetAsync(a.lossacc, 0, 3 * sizeof(double), st);   // the two sums and the block counter
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int per_row = std::max(1, std::min((a.N + 1023) / 1024, (4 * sms + a.P - 1) / a.P));
-    vote_loss_kernel<<<dim3(per_row, a.P), 256, 0, st>>>(a.scores, a.golden, a.P, a.N, a.gamma, a.lossacc);
-    vote_loss_finalize<<<1, 1, 0, st>>>(a.lossacc, static_cast<double>(a.P) * a.N, a.loss);
-    if ((rc = check_launch("vote_labels/loss", 2)) != LSA_OK) return rc;
+    vote_loss_kernel<<<dim3(per_row, a.P), 256, 0, st>>>(a.scores, a.golden, a.P, a.N, a.gamma, a.lossacc, a.loss);
+    if ((rc = check_launch("vote_labels/loss")) != LSA_OK) return rc;
   }
   return LSA_OK;
 }
