@@ -127,13 +127,14 @@ compact_kernel(const uint32_t* __restrict__ bits, int Nw, int cap, int32_t* __re
 }
 
 // ------------------------------------------------------------------ union + fetch lists
-// The whole selection of one trigger in two launches over the L layer masks: per word,
-// new_l = mask_l & ~(mask_0 | .. | mask_{l-1}) and U = mask_0 | .. | mask_{L-1}, and the
-// L + 1 fetch lists (new_0 .. new_{L-1}, U) with their counts.  Block (chunk, b) owns
-// words [chunk*kCompactWords, ...) of sequence b.  The first launch writes each chunk's
-// popcounts of the L + 1 sets; the second takes its output bases from the earlier
-// chunks' counts; each warp stages its run of every list in shared memory and copies it
-// out with full stores.
+// The whole selection of one trigger in two launches over the L layer masks (three with
+// the union's top-k keys): per word, new_l = mask_l & ~(mask_0 | .. | mask_{l-1}) and
+// U = mask_0 | .. | mask_{L-1}, and the L + 1 fetch lists (new_0 .. new_{L-1}, U) with
+// their counts.  Block (chunk, b) owns words [chunk*kCompactWords, ...) of sequence b.
+// The first launch writes each chunk's popcounts of the L + 1 sets; the second takes its
+// output bases from the earlier chunks' counts; each warp stages its run of every list in
+// shared memory and copies it out with full stores; the third (select_keys_kernel) forms
+// the keys of the union's list.
 constexpr int kSelMaxLayers = 8;
 
 // Per (chunk, sequence): the popcounts of the chunk's words in the L new sets and the
