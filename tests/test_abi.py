@@ -112,3 +112,31 @@ def test_workspace_queries(lib):
     assert 0 < n < 64 << 20
     assert lib.lsa_topk_workspace_bytes(32, 262144) >= 32 * 262144 * 4
     assert lib.lsa_vote_labels_workspace_bytes(24, 64, 131072) >= 24 * 64 * 4096 * 4
+
+
+def test_selection_and_keyed_topk_argument_errors(lib):
+    """The fused selection and the keyed top-k refuse bad arguments on the host (fake,
+    aligned device addresses; every case returns before a launch)."""
+    A = 256                                   # an aligned non-null address, never dereferenced
+    B, L, N = 2, 3, 4096
+    ws_need = lib.lsa_select_fetch_workspace_bytes(B, N)
+    Nw = (N + 31) // 32
+    # the per-chunk counts, the union's warp bases and a copy of the union words fit
+    assert ws_need >= B * Nw * 4 + B * ((Nw + 255) // 256) * 9 * 4
+    sf = lib.lsa_select_fetch
+    args = lambda **kw: [kw.get("B", B), kw.get("L", L), N, A, None, None, N, A, A, A, A,
+                         kw.get("logit", None), kw.get("key_U", None), None, kw.get("ws", A),
+                         kw.get("wsb", ws_need), None]
+    assert sf(*args(L=9)) == lsa.LSA_ERR_UNSUPPORTED and b"1 to 8" in lib.lsa_last_error()
+    assert sf(*args(B=-1)) == lsa.LSA_ERR_INVALID_ARG
+    assert sf(*args(key_U=A)) == lsa.LSA_ERR_INVALID_ARG and b"needs the logits" in lib.lsa_last_error()
+    assert sf(*args(logit=A, key_U=A + 4)) == lsa.LSA_ERR_INVALID_ARG      # key_U not 16-byte aligned
+    assert sf(*args(wsb=ws_need - 1)) == lsa.LSA_ERR_NOMEM
+    assert sf(*args(ws=A + 16)) == lsa.LSA_ERR_NOMEM                       # workspace not 256-byte aligned
+    assert sf(*args(B=0)) == lsa.LSA_OK
+    tk = lib.lsa_topk_keyed
+    assert tk(-1, 8, A, N, A, A, A, A, None) == lsa.LSA_ERR_INVALID_ARG
+    assert tk(B, 8, A, N, None, A, A, A, None) == lsa.LSA_ERR_INVALID_ARG   # no counts
+    assert tk(B, 8, A, N, A, A, None, A, None) == lsa.LSA_ERR_INVALID_ARG   # k > 0 without an output
+    assert tk(B, 8, A, N, A, A + 2, A, A, None) == lsa.LSA_ERR_INVALID_ARG  # keys not 4-byte aligned
+    assert tk(0, 8, A, N, A, A, A, A, None) == lsa.LSA_OK
