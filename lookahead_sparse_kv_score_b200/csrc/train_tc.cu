@@ -440,33 +440,47 @@ outer_acc_kernel(const __nv_bfloat16* __restrict__ X, int M, const float* __rest
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  // The next stage's values are loaded into registers while the current one is used
+  // (thread t: X positions t / 16, values (t % 16) * 8 .. + 7; Y two float4).
+  const int xk = threadIdx.x >> 4, xc = (threadIdx.x & 15) * 8;
+  auto load_x = [&](int p0) {
+    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+    const int pp = p0 + xk, m = m0 + xc;
+    if (pp < P && m < M) raw = *reinterpret_cast<const uint4*>(X + static_cast<size_t>(pp) * M + m);   // M % 8 == 0
+    return raw;
+  };
+  auto load_y = [&](int p0, int u) {
+    const int t = threadIdx.x + u * 256;
+    const int kk = t / (kOT / 4), c = (t % (kOT / 4)) * 4;
+    const int pp = p0 + kk, n = n0 + c;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (pp < P && n < Nn) v = *reinterpret_cast<const float4*>(Y + static_cast<size_t>(pp) * Nn + n);
+    return v;
+  };
+  static_assert(kOK * kOT / 4 == 2 * 256, "two float4 of Y per thread and stage");
+  uint4 xr = load_x(0);
+  float4 yr0 = load_y(0, 0), yr1 = load_y(0, 1);
   for (int p0 = 0; p0 < P; p0 += kOK) {
-    {   // X: 16 positions x 128 values, one 16-byte load (8 bf16) per thread
-      const int kk = threadIdx.x >> 4, c = (threadIdx.x & 15) * 8;
-      const int pp = p0 + kk, m = m0 + c;
+    {   // X: bf16 -> fp32 is exact
+      const uint32_t wv[4] = {xr.x, xr.y, xr.z, xr.w};
       float v[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = 0.f;
-      if (pp < P && m < M) {   // M % 8 == 0: the eight values are all in range
-        const uint4 raw = *reinterpret_cast<const uint4*>(X + static_cast<size_t>(pp) * M + m);
-        const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          v[2 * e] = __uint_as_float(wv[e] << 16);            // bf16 -> fp32 is exact
-          v[2 * e + 1] = __uint_as_float(wv[e] & 0xffff0000u);
-        }
+      for (int e = 0; e < 4; ++e) {
+        v[2 * e] = __uint_as_float(wv[e] << 16);
+        v[2 * e + 1] = __uint_as_float(wv[e] & 0xffff0000u);
       }
-      *reinterpret_cast<float4*>(&xs[kk][c]) = make_float4(v[0], v[1], v[2], v[3]);
-      *reinterpret_cast<float4*>(&xs[kk][c + 4]) = make_float4(v[4], v[5], v[6], v[7]);
-    }
-    for (int t = threadIdx.x; t < kOK * kOT / 4; t += 256) {   // Y: two float4 per thread
-      const int kk = t / (kOT / 4), c = (t % (kOT / 4)) * 4;
-      const int pp = p0 + kk, n = n0 + c;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (pp < P && n < Nn) v = *reinterpret_cast<const float4*>(Y + static_cast<size_t>(pp) * Nn + n);
-      *reinterpret_cast<float4*>(&ys[kk][c]) = v;
+      *reinterpret_cast<float4*>(&xs[xk][xc]) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4*>(&xs[xk][xc + 4]) = make_float4(v[4], v[5], v[6], v[7]);
+      const int t0 = threadIdx.x, t1 = threadIdx.x + 256;
+      *reinterpret_cast<float4*>(&ys[t0 / (kOT / 4)][(t0 % (kOT / 4)) * 4]) = yr0;
+      *reinterpret_cast<float4*>(&ys[t1 / (kOT / 4)][(t1 % (kOT / 4)) * 4]) = yr1;
     }
     __syncthreads();
+    if (p0 + kOK < P) {
+      xr = load_x(p0 + kOK);
+      yr0 = load_y(p0 + kOK, 0);
+      yr1 = load_y(p0 + kOK, 1);
+    }
 #pragma unroll
     for (int k = 0; k < kOK; ++k) {
       const float4 a0 = *reinterpret_cast<const float4*>(&xs[k][ty * 4]);
@@ -496,41 +510,97 @@ outer_acc_kernel(const __nv_bfloat16* __restrict__ X, int M, const float* __rest
   }
 }
 
-// dc[p][i] = sum_j dq[p][j] W_up[i][j]  (W_up bf16 [r][J]).  Tiles of 64 positions x 64
-// rows i, the reduction split into kDcSplits slices written as partial sums and added in
-// a fixed order by dc_reduce_kernel.
+// dc[p][i] = sum_j dq[p][j] W_up[i][j]  (W_up bf16 [r][J]).  Tiles of 64 positions x 256
+// rows i, 8 x 8 outputs per thread (two float4 of each operand per reduction step), the
+// reduction split into kDcSplits slices written as partial sums and added in a fixed order
+// by dc_reduce_kernel; within a slice j ascends, so the tile shape changes no result bit.
+// The next 32-wide chunk of both operands is loaded into registers while the current one
+// is used.
 constexpr int kDcSplits = 64;
+constexpr int kDcP = 64, kDcI = 256, kDcJ = 32;
 
 __global__ void __launch_bounds__(256)
 dc_kernel(const float* __restrict__ dq, int P, int J, const __nv_bfloat16* __restrict__ Wu, int r,
           float* __restrict__ part) {
-  __shared__ float as[32][65], bs[32][65];     // [j][p], [j][i]
-  const int i0 = blockIdx.x * 64, p0 = blockIdx.y * 64, sl = blockIdx.z;
+  __shared__ __align__(16) float as[kDcJ][kDcP];   // [j][p]
+  __shared__ __align__(16) float bs[kDcJ][kDcI];   // [j][i]
+  const int i0 = blockIdx.x * kDcI, p0 = blockIdx.y * kDcP, sl = blockIdx.z;
   const int js = (J * sl) / kDcSplits, je = (J * (sl + 1)) / kDcSplits;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4] = {};
-  for (int j0 = js; j0 < je; j0 += 32) {
-    for (int t = threadIdx.x; t < 64 * 32; t += 256) {
-      const int row = t / 32, jj = t % 32, j = j0 + jj;
-      as[jj][row] = (p0 + row < P && j < je) ? dq[static_cast<size_t>(p0 + row) * J + j] : 0.f;
-      bs[jj][row] = (i0 + row < r && j < je) ? __bfloat162float(Wu[static_cast<size_t>(i0 + row) * J + j]) : 0.f;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // i groups of 4 (x2), p groups of 4 (x2)
+  float acc[8][8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+  // thread t loads dq float4 f = t + 256 u (row f % 64, j f / 64 * 4) and W_up 8-wide
+  // pieces f = t + 256 u (row f % 256, j f / 256 * 8); positions past P, rows past r and
+  // columns past the slice read zero (J % 8 == 0, so a piece is all in or all out)
+  auto load_a = [&](int j0, int u) {
+    const int f = threadIdx.x + 256 * u, row = f % kDcP, j = j0 + (f / kDcP) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p0 + row < P && j < je) v = *reinterpret_cast<const float4*>(dq + static_cast<size_t>(p0 + row) * J + j);
+    return v;
+  };
+  auto load_b = [&](int j0, int u) {
+    const int f = threadIdx.x + 256 * u, row = f % kDcI, j = j0 + (f / kDcI) * 8;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (i0 + row < r && j < je) v = *reinterpret_cast<const uint4*>(Wu + static_cast<size_t>(i0 + row) * J + j);
+    return v;
+  };
+  float4 ar[2];
+  uint4 br[4];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) ar[u] = load_a(js, u);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) br[u] = load_b(js, u);
+  for (int j0 = js; j0 < je; j0 += kDcJ) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int f = threadIdx.x + 256 * u, row = f % kDcP, jj = (f / kDcP) * 4;
+      as[jj][row] = ar[u].x; as[jj + 1][row] = ar[u].y; as[jj + 2][row] = ar[u].z; as[jj + 3][row] = ar[u].w;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int f = threadIdx.x + 256 * u, row = f % kDcI, jj = (f / kDcI) * 8;
+      const uint32_t wv[4] = {br[u].x, br[u].y, br[u].z, br[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        bs[jj + 2 * e][row] = __uint_as_float(wv[e] << 16);              // bf16 -> fp32 is exact
+        bs[jj + 2 * e + 1][row] = __uint_as_float(wv[e] & 0xffff0000u);
+      }
     }
     __syncthreads();
-#pragma unroll 8
-    for (int k = 0; k < 32; ++k)
+    if (j0 + kDcJ < je) {
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int u = 0; u < 2; ++u) ar[u] = load_a(j0 + kDcJ, u);
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(as[k][ty * 4 + a], bs[k][tx * 4 + b], acc[a][b]);
+      for (int u = 0; u < 4; ++u) br[u] = load_b(j0 + kDcJ, u);
+    }
+    const int kn = min(kDcJ, je - j0);
+    for (int k = 0; k < kn; ++k) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&as[k][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&as[k][32 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&bs[k][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&bs[k][128 + tx * 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(av[a], bv[b], acc[a][b]);
+    }
     __syncthreads();
   }
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < 8; ++a) {
+    const int pp = p0 + (a >> 2) * 32 + ty * 4 + (a & 3);
+    if (pp >= P) continue;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int pp = p0 + ty * 4 + a, i = i0 + tx * 4 + b;
-      if (pp < P && i < r) part[(static_cast<size_t>(sl) * P + pp) * r + i] = acc[a][b];
+    for (int b = 0; b < 8; ++b) {
+      const int i = i0 + (b >> 2) * 128 + tx * 4 + (b & 3);
+      if (i < r) part[(static_cast<size_t>(sl) * P + pp) * r + i] = acc[a][b];
     }
+  }
 }
 
 __global__ void dc_reduce_kernel(const float* __restrict__ part, size_t n, float* __restrict__ dc) {
@@ -635,7 +705,7 @@ int launch_train(const TrainArgs& a, cudaStream_t st) {
   outer_acc_kernel<<<dim3(static_cast<unsigned>((HD + kOT - 1) / kOT), (a.r + kOT - 1) / kOT), 256, 0, st>>>(
       c, a.r, dq, static_cast<int>(HD), a.P, a.dW_up);
   float* dcpart = reinterpret_cast<float*>(ws + lay.dcpart);
-  dc_kernel<<<dim3((a.r + 63) / 64, (a.P + 63) / 64, kDcSplits), 256, 0, st>>>(
+  dc_kernel<<<dim3((a.r + kDcI - 1) / kDcI, (a.P + kDcP - 1) / kDcP, kDcSplits), 256, 0, st>>>(
       dq, a.P, static_cast<int>(HD), static_cast<const __nv_bfloat16*>(a.W_up), a.r, dcpart);
   const size_t ndc = static_cast<size_t>(a.P) * a.r;
   dc_reduce_kernel<<<static_cast<unsigned>(std::min<size_t>((ndc + 255) / 256, 1184)), 256, 0, st>>>(dcpart, ndc, dc);
