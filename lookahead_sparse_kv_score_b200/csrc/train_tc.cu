@@ -607,7 +607,8 @@ __global__ void dc_reduce_kernel(const float* __restrict__ part, size_t n, float
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     float v = 0.f;
-    for (int s = 0; s < kDcSplits; ++s) v += part[s * n + i];
+#pragma unroll 16
+    for (int s = 0; s < kDcSplits; ++s) v += part[s * n + i];   // loads issued ahead, sums in slice order
     dc[i] = v;
   }
 }
