@@ -388,27 +388,32 @@ __global__ void train_qimg_kernel(const __nv_bfloat16* __restrict__ q, int P, in
 }
 
 // U = sum over chunks; dq = w U ([P][H*dI]); dw = q . U ([P][H]).  One block per (p, h).
-__global__ void train_finish_kernel(const float* __restrict__ Upart, int chunks, int rows, int dI,
-                                    const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
-                                    float* __restrict__ dq, float* __restrict__ dw) {
-  __shared__ float tmp[32];
-  const int row = blockIdx.x;
+// One warp per (position, head) row: U = the chunks' partial sums in chunk order, dq = w U,
+// dw = q . U; block 0's first thread also writes the loss means and the bias gradient
+// (the fused kernel's sums are complete when this launch runs).
+__global__ void __launch_bounds__(256)
+train_finish_kernel(const float* __restrict__ Upart, int chunks, int rows, int dI,
+                    const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
+                    float* __restrict__ dq, float* __restrict__ dw, const double* __restrict__ acc, double n,
+                    double* __restrict__ loss, double* __restrict__ dbias) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (loss) { loss[0] = acc[0] / n; loss[1] = acc[1] / n; }
+    if (dbias) dbias[0] = acc[2];
+  }
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float wr = w[row];
   float part = 0.f;
-  for (int d = threadIdx.x; d < dI; d += blockDim.x) {
+  for (int d = lane; d < dI; d += 32) {
     float u = 0.f;
     for (int c = 0; c < chunks; ++c) u += Upart[(static_cast<size_t>(c) * rows + row) * dI + d];
-    dq[static_cast<size_t>(row) * dI + d] = w[row] * u;
+    dq[static_cast<size_t>(row) * dI + d] = wr * u;
     part = fmaf(__bfloat162float(q[static_cast<size_t>(row) * dI + d]), u, part);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-  if ((threadIdx.x & 31) == 0) tmp[threadIdx.x >> 5] = part;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float s = 0.f;
-    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) s += tmp[i];
-    dw[row] = s;
-  }
+  if (lane == 0) dw[row] = part;
 }
 
 // out[m][n] = sum_p X[p][m] Y[p][n]  (X bf16 [P][M], Y fp32 [P][Nn]; M % 8 == 0, Nn % 4 == 0,
@@ -613,12 +618,6 @@ __global__ void dc_reduce_kernel(const float* __restrict__ part, size_t n, float
   }
 }
 
-__global__ void train_loss_kernel(const double* __restrict__ acc, double n, double* __restrict__ loss,
-                                  double* __restrict__ dbias) {
-  if (loss) { loss[0] = acc[0] / n; loss[1] = acc[1] / n; }
-  if (dbias) dbias[0] = acc[2];
-}
-
 int train_smem(int dI) {
   return kTStages * (dI / 64) * kTE * 128 + kTR * dI * 2 + kGBufs * 2 * kTR * kTE * 2 + kTR * 4 + 2 * 4 * 4 * 32 * 4 +
          1024 + 1024;
@@ -697,8 +696,10 @@ int launch_train(const TrainArgs& a, cudaStream_t st) {
     default: return fail(LSA_ERR_UNSUPPORTED, "train: H=%d dI=%d", a.H, a.dI);
   }
   if ((rc = check_launch("train/fused")) != LSA_OK) return rc;
-  train_finish_kernel<<<a.P * a.H, 128, 0, st>>>(Upart, kTChunks, a.P * a.H, a.dI,
-                                                 static_cast<const __nv_bfloat16*>(a.q), a.w, dq, dw);
+  const int frows = a.P * a.H;
+  train_finish_kernel<<<(frows + 7) / 8, 256, 0, st>>>(Upart, kTChunks, frows, a.dI,
+                                                       static_cast<const __nv_bfloat16*>(a.q), a.w, dq, dw, acc,
+                                                       static_cast<double>(a.P) * a.N, a.loss, a.dbias);
   if ((rc = check_launch("train/finish")) != LSA_OK) return rc;
   // projection gradients
   const __nv_bfloat16* c = static_cast<const __nv_bfloat16*>(a.c);
@@ -713,8 +714,7 @@ int launch_train(const TrainArgs& a, cudaStream_t st) {
   const int nb_r = (a.r + kOT - 1) / kOT, nb_h = (a.H + kOT - 1) / kOT;   // dW_down and dW_w in one launch
   outer_acc_kernel<<<dim3(nb_r + nb_h, (a.D + kOT - 1) / kOT), 256, 0, st>>>(h, a.D, dc, a.r, a.P, a.dW_down, nb_r,
                                                                            dw, a.H, a.dW_w);
-  train_loss_kernel<<<1, 1, 0, st>>>(acc, static_cast<double>(a.P) * a.N, a.loss, a.dbias);
-  return check_launch("train/projection gradients", 5);
+  return check_launch("train/projection gradients", 4);
 }
 
 }  // namespace lsa
