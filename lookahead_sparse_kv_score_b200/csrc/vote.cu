@@ -186,27 +186,6 @@ __device__ __forceinline__ float4 ldg4_hint(const float4* p, uint64_t pol) {
   return v;
 }
 
-// Calls f(value, index) for every logit of the row, four loads in flight per thread.
-template <typename F>
-__device__ __forceinline__ void row_for_each(const float* x, int N, bool vec, F&& f) {
-  const int G = (N + 3) >> 2;
-  int g = threadIdx.x;
-  auto run = [&](const float4& v, int s) {
-    f(v.x, s);
-    if (s + 1 < N) f(v.y, s + 1);
-    if (s + 2 < N) f(v.z, s + 2);
-    if (s + 3 < N) f(v.w, s + 3);
-  };
-  for (; g + 3 * kRowThreads < G; g += 4 * kRowThreads) {
-    float4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) v[u] = load4(x, 4 * (g + u * kRowThreads), N, vec);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) run(v[u], 4 * (g + u * kRowThreads));
-  }
-  for (; g < G; g += kRowThreads) run(load4(x, 4 * g, N, vec), 4 * g);
-}
-
 // Ascending bitonic sort of n entries (n a power of two, >= 64).  Stages whose partner
 // distance is below 64 stay inside 64-entry blocks, one warp per block, with warp
 // barriers only.
