@@ -402,22 +402,25 @@ struct TopkShared {
 };
 constexpr int kTopkStateBytes = (static_cast<int>(sizeof(TopkShared)) + 15) / 16 * 16;
 
-// Candidates and keys come in one of two ways.  Fetched-set mode: candidate j is entry
+// Candidates and keys come in one of three ways.  Fetched-set mode: candidate j is entry
 // idx[b][j] (j < count[b]) with key order_key(max over layers of logit[l][b][entry]),
-// and k is the same for every sequence.  Direct mode (dkeys != nullptr): candidate j is
-// j itself for j < cap, its key is dkeys[b][j], and sequence b keeps kdev[b] of them,
-// or none (raising LSA_ERR_CAPACITY) when kdev[b] exceeds cap - kept[b]; the output row
-// stride is then cap.
+// and k is the same for every sequence.  Keyed mode (idx and dkeys given): the same
+// candidates with the keys given per candidate, dkeys[b][j].  Direct mode (dkeys without
+// idx): candidate j is j itself for j < cap, its key is dkeys[b][j], and sequence b keeps
+// kdev[b] of them, or none (raising LSA_ERR_CAPACITY) when kdev[b] exceeds cap - kept[b];
+// the output row stride is then cap.
 //
 // One thread-block cluster per sequence; CTA `rank` owns the contiguous candidate slice
-// [rank m, (rank + 1) m), m = ceil(n / cluster size).  Its keys go to shared memory (to
-// the key workspace when the slice exceeds kTopkSmemKeys).  Three radix passes (digits
-// of 11, 11 and 10 bits, most significant first) find the k-th largest key T and the
-// number kk of keys equal to T to keep; each pass adds the CTAs' digit histograms
-// through distributed shared memory and picks the digit with one block-wide scan.  The
-// kept entries, all keys above T and the kk lowest-index ties, are written in ascending
-// candidate (= entry) order: each warp owns a contiguous part of its CTA's slice, and
-// its output offset comes from the counts of the CTAs and warps before it.
+// [rank m, (rank + 1) m), m = ceil(n / cluster size).  Its keys go to shared memory when
+// the slice fits in kTopkSmemKeys; otherwise given keys are read in place and computed
+// keys go to the key workspace.  Three radix passes (digits of 11, 11 and 10 bits, most
+// significant first) find the k-th largest key T and the number kk of keys equal to T to
+// keep; each pass adds the CTAs' digit histograms through distributed shared memory and
+// picks the digit with one block-wide scan.  The kept entries, all keys above T and the
+// kk lowest-index ties, are written in ascending candidate (= entry) order: each warp
+// owns a contiguous part of its CTA's slice, records where its keys at or above T are
+// while counting them, and takes its output offset from the counts of the CTAs and warps
+// before it.
 __global__ void __launch_bounds__(kTopkThreads, 1)
 topk_cluster_kernel(int B, int L, int N, int k, const int32_t* __restrict__ idx, int cap,
                     const int32_t* __restrict__ count, const float* __restrict__ logit,
