@@ -296,6 +296,21 @@ def test_fetched_key_is_max_over_marking_layers():
     assert O.fetched_key(z, m).tolist() == [5.0, 2.0, -np.inf]
 
 
+def test_fetched_key_equals_the_largest_logit_when_marks_are_the_threshold():
+    """With the marks the threshold makes (z >= 0), a layer that does not mark an entry has
+    a logit below every marking layer's, so for every fetched entry the key over the
+    marking layers equals the largest logit over all layers (the form the fused selection
+    computes its keys in); entries no layer marks have no key."""
+    g = np.random.default_rng(11)
+    z = np.round(g.standard_normal((4, 5000)) * 2, 1)     # ties and exact zeros included
+    z[:, :10] = 0.0
+    m = z >= 0
+    key = O.fetched_key(z, m)
+    fetched = m.any(axis=0)
+    assert np.array_equal(key[fetched], z.max(axis=0)[fetched])
+    assert np.all(np.isneginf(key[~fetched]))
+
+
 def test_step_select_composes_the_set_operations():
     """The step's selection from per-layer marks and logits, by brute force: the top-k
     runs over the union of all layers (not one layer's new set), keyed by the largest
